@@ -1,0 +1,221 @@
+"""Python binding of libckl.so: the fused chunked KL-distillation loss on B200.
+
+Argument marshalling only.  Every step of the loss runs in the CUDA library
+(``csrc/``, declared in ``include/ckl.h``); PyTorch supplies device memory,
+streams and events.  There is no CPU path: importing this package fails when
+the library has not been built, and every call fails when no sm_100 device
+is present.
+
+    import chunked_kl_loss_ckl_b200 as ckl
+    loss, lse = ckl.forward(H, W, idx, logp, mask, chunk=1024)
+    dH, dW = ckl.backward(H, W, idx, logp, mask, lse, chunk=1024)
+    loss = ckl.chunked_kl_loss(H, W, idx, logp, mask, chunk=1024)  # autograd
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "LIB_PATH", "CklError", "Trace", "KERNEL_NAMES", "lib", "workspace_bytes", "new_workspace",
+    "forward", "backward", "read_device_status", "status_string", "chunked_kl_loss",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libckl.so")
+
+CKL_OK = 0
+STATUS_NAMES = {
+    0: "CKL_OK", 1: "CKL_ERR_INVALID_ARG", 2: "CKL_ERR_UNSUPPORTED", 3: "CKL_ERR_WORKSPACE",
+    4: "CKL_ERR_CUDA", 5: "CKL_ERR_BAD_INDEX", 6: "CKL_ERR_BAD_LOGP", 7: "CKL_ERR_TIMEOUT",
+}
+KERNEL_NAMES = {1: "prep", 2: "fwd_gemm", 3: "fwd_combine", 4: "bwd_dz", 5: "bwd_dhdw", 6: "other"}
+
+
+class CklError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {STATUS_NAMES.get(code, code)} ({status_string(code)})")
+
+
+class _Trace(ctypes.Structure):
+    _fields_ = [("capacity", ctypes.c_int32), ("count", ctypes.c_int32),
+                ("events", ctypes.POINTER(ctypes.c_void_p)),
+                ("kernel_id", ctypes.POINTER(ctypes.c_int32))]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m chunked_kl_loss_ckl_b200._build` (nvcc, sm_100a)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+    tr = ctypes.POINTER(_Trace)
+    L.ckl_workspace_bytes.argtypes = [i64, i64, i64, i32, i64]
+    L.ckl_workspace_bytes.restype = sz
+    L.ckl_forward.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i64, vp, vp, vp, sz, vp, tr]
+    L.ckl_forward.restype = ctypes.c_int
+    L.ckl_backward.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i64, vp, vp, vp, vp, i32,
+                               vp, sz, vp, tr]
+    L.ckl_backward.restype = ctypes.c_int
+    L.ckl_read_device_status.argtypes = [vp, vp, ctypes.POINTER(i32)]
+    L.ckl_read_device_status.restype = ctypes.c_int
+    L.ckl_status_string.argtypes = [i32]
+    L.ckl_status_string.restype = ctypes.c_char_p
+    L.ckl_version.argtypes = []
+    L.ckl_version.restype = i32
+    return L
+
+
+lib = _load()
+
+
+def status_string(code: int) -> str:
+    return lib.ckl_status_string(int(code)).decode()
+
+
+class Trace:
+    """Per-launch CUDA events recorded by the library around each kernel.
+
+    ``durations()`` returns [(kernel name, ms)] after the stream has been
+    synchronised.  Call ``reset()`` between steps to reuse the events.
+    """
+
+    def __init__(self, capacity: int = 256):
+        self.capacity = capacity
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(2 * capacity)]
+        for e in self.events:  # create the underlying cudaEvent_t now
+            e.record()
+        torch.cuda.synchronize()
+        self._handles = (ctypes.c_void_p * (2 * capacity))(*[e.cuda_event for e in self.events])
+        self._ids = (ctypes.c_int32 * capacity)()
+        self.c = _Trace(capacity, 0, ctypes.cast(self._handles, ctypes.POINTER(ctypes.c_void_p)),
+                        ctypes.cast(self._ids, ctypes.POINTER(ctypes.c_int32)))
+
+    def reset(self) -> None:
+        self.c.count = 0
+
+    @property
+    def count(self) -> int:
+        return int(self.c.count)
+
+    def durations(self):
+        return [(KERNEL_NAMES.get(self._ids[i], str(self._ids[i])),
+                 self.events[2 * i].elapsed_time(self.events[2 * i + 1]))
+                for i in range(self.count)]
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _trace_ptr(trace):
+    return None if trace is None else ctypes.byref(trace.c)
+
+
+def _check_inputs(H, W, idx, logp, mask):
+    for name, t, dts in (("H", H, (torch.bfloat16, torch.int16, torch.uint16)),
+                         ("W", W, (torch.bfloat16, torch.int16, torch.uint16)),
+                         ("topk_idx", idx, (torch.int32,)), ("topk_logp", logp, (torch.float32,))):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if t.dtype not in dts:
+            raise TypeError(f"{name} has dtype {t.dtype}, expected one of {dts}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if mask is not None and (not mask.is_cuda or mask.dtype not in (torch.uint8, torch.bool)
+                             or not mask.is_contiguous()):
+        raise ValueError("mask must be a contiguous CUDA uint8/bool tensor")
+    T, d = H.shape
+    V, d2 = W.shape
+    if d2 != d or idx.shape != logp.shape or idx.shape[0] != T:
+        raise ValueError("shape mismatch: H [T,d], W [V,d], topk_idx/topk_logp [T,K]")
+    if mask is not None and mask.shape != (T,):
+        raise ValueError("mask must have shape [T]")
+    return T, d, V, idx.shape[1]
+
+
+def workspace_bytes(T: int, d: int, V: int, K: int, chunk: int) -> int:
+    n = lib.ckl_workspace_bytes(T, d, V, K, chunk)
+    if n == 0:
+        raise CklError(1, "ckl_workspace_bytes")
+    return int(n)
+
+
+def new_workspace(T: int, d: int, V: int, K: int, chunk: int, device=None) -> torch.Tensor:
+    n = workspace_bytes(T, d, V, K, chunk)
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def forward(H, W, idx, logp, mask=None, chunk: int = 1024, workspace=None, stream=None,
+            trace: Trace | None = None, out_loss=None, out_lse=None):
+    """Mean KL over the positions that count, and lse for every row."""
+    T, d, V, K = _check_inputs(H, W, idx, logp, mask)
+    if workspace is None:
+        workspace = new_workspace(T, d, V, K, chunk, H.device)
+    loss = out_loss if out_loss is not None else torch.empty(1, dtype=torch.float32, device=H.device)
+    lse = out_lse if out_lse is not None else torch.empty(T, dtype=torch.float32, device=H.device)
+    rc = lib.ckl_forward(_ptr(H), _ptr(W), _ptr(idx), _ptr(logp), _ptr(mask), T, d, V, K, chunk,
+                         _ptr(loss), _ptr(lse), _ptr(workspace), workspace.numel(),
+                         _stream_handle(stream), _trace_ptr(trace))
+    if rc != CKL_OK:
+        raise CklError(rc, "ckl_forward")
+    return loss, lse
+
+
+def backward(H, W, idx, logp, mask, lse, grad_loss=None, chunk: int = 1024, dW=None,
+             accumulate_dW: bool = False, workspace=None, stream=None,
+             trace: Trace | None = None, out_dH=None):
+    """dH (bf16, like H) and dW (fp32) by chunked recomputation."""
+    T, d, V, K = _check_inputs(H, W, idx, logp, mask)
+    if workspace is None:
+        workspace = new_workspace(T, d, V, K, chunk, H.device)
+    dH = out_dH if out_dH is not None else torch.empty(T, d, dtype=torch.bfloat16, device=H.device)
+    if dW is None:
+        dW = torch.empty(V, d, dtype=torch.float32, device=H.device)
+        accumulate_dW = False
+    if grad_loss is not None and (grad_loss.dtype != torch.float32 or not grad_loss.is_cuda):
+        raise TypeError("grad_loss must be a CUDA float32 tensor")
+    rc = lib.ckl_backward(_ptr(H), _ptr(W), _ptr(idx), _ptr(logp), _ptr(mask), T, d, V, K, chunk,
+                          _ptr(lse), _ptr(grad_loss), _ptr(dH), _ptr(dW), int(bool(accumulate_dW)),
+                          _ptr(workspace), workspace.numel(), _stream_handle(stream),
+                          _trace_ptr(trace))
+    if rc != CKL_OK:
+        raise CklError(rc, "ckl_backward")
+    return dH, dW
+
+
+def read_device_status(workspace, stream=None):
+    """(status code, raw device word) of the last call that used ``workspace``."""
+    word = ctypes.c_int32(0)
+    rc = lib.ckl_read_device_status(_ptr(workspace), _stream_handle(stream), ctypes.byref(word))
+    return int(rc), int(word.value)
+
+
+class _ChunkedKL(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, H, W, idx, logp, mask, chunk):
+        loss, lse = forward(H, W, idx, logp, mask, chunk)
+        ctx.save_for_backward(H, W, idx, logp, lse)
+        ctx.mask = mask
+        ctx.chunk = chunk
+        return loss.reshape(())
+
+    @staticmethod
+    def backward(ctx, g):
+        H, W, idx, logp, lse = ctx.saved_tensors
+        gl = g.reshape(1).to(torch.float32).contiguous()
+        dH, dW = backward(H, W, idx, logp, ctx.mask, lse, grad_loss=gl, chunk=ctx.chunk)
+        return dH.to(H.dtype), dW.to(W.dtype), None, None, None, None
+
+
+def chunked_kl_loss(H, W, idx, logp, mask=None, chunk: int = 1024):
+    """Differentiable loss (gradients w.r.t. H and W; dW cast to W's dtype)."""
+    return _ChunkedKL.apply(H, W, idx, logp, mask, chunk)

@@ -1,0 +1,414 @@
+// Host side of libckl.so: argument checks, workspace layout, the chunk
+// scheduler and the kernel launches.  See include/ckl.h for the contract.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/ckl.h"
+#include "ckl_kernels.cuh"
+
+namespace {
+
+using ckl::TcParams;
+
+constexpr int32_t kVersion = 100;  // 0.1.0
+constexpr int kMaxSplits = 64;     // vocabulary splits per row in the forward
+constexpr size_t kHeaderBytes = 256;
+
+// Header words at the start of the workspace.
+struct Header {
+  int32_t status;   // CKL_DEV_* bits
+  int32_t countN;   // positions that count
+  uint32_t ticket;  // combine: blocks finished
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+struct Layout {
+  size_t pairs, hp, partials, blocksums, dz, total;
+  int64_t ldz;  // dZ row pitch in elements
+};
+
+Layout layout(int64_t T, int64_t V, int32_t K, int64_t chunk) {
+  Layout L{};
+  size_t off = kHeaderBytes;
+  L.pairs = off;
+  off += align256(static_cast<size_t>(T) * K * 8);
+  L.hp = off;
+  off += align256(static_cast<size_t>(T) * 4);
+  L.partials = off;
+  off += align256(static_cast<size_t>(T) * kMaxSplits * 16);
+  L.blocksums = off;
+  off += align256(static_cast<size_t>(cdiv(T, ckl::COMBINE_THREADS)) * 8);
+  L.ldz = cdiv(V, 8) * 8;
+  L.dz = off;
+  off += align256(static_cast<size_t>(std::min(chunk, std::max<int64_t>(T, 1))) * L.ldz * 2);
+  L.total = off;
+  return L;
+}
+
+bool sizes_ok(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk) {
+  const int64_t lim = (int64_t(1) << 31) - 1;
+  return T >= 0 && T < lim && d >= 8 && d % 8 == 0 && d < lim && V >= 1 && V < lim && K >= 1 &&
+         chunk >= 1;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// ---- driver entry point for tensor-map encoding (no link-time libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D tiled tensor map over a row-major [outer, inner] array.
+bool map2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner,
+           uint64_t outer, uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer,
+           CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {pitch_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct DevInfo {
+  int sms = 0;
+  int major = 0;
+  bool attrs_set = false;
+};
+
+bool device_info(DevInfo& out) {
+  static std::mutex mu;
+  static DevInfo cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  DevInfo& di = cache[dev];
+  if (di.sms == 0) {
+    if (cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return false;
+    if (cudaDeviceGetAttribute(&di.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+      return false;
+  }
+  if (!di.attrs_set && di.major == 10) {
+    if (cudaFuncSetAttribute(ckl::tc_kernel<ckl::MODE_FWD>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, ckl::SMEM_ALLOC) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(ckl::tc_kernel<ckl::MODE_DZ>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, ckl::SMEM_ALLOC) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(ckl::tc_kernel<ckl::MODE_DHDW>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, ckl::SMEM_ALLOC) !=
+            cudaSuccess)
+      return false;
+    di.attrs_set = true;
+  }
+  out = di;
+  return true;
+}
+
+// Records launch events around one kernel.
+struct TraceScope {
+  ckl_trace* tr;
+  cudaStream_t st;
+  int slot = -1;
+  TraceScope(ckl_trace* t, cudaStream_t s, int kid) : tr(t), st(s) {
+    if (tr && tr->events && tr->count < tr->capacity) {
+      slot = tr->count;
+      cudaEventRecord(static_cast<cudaEvent_t>(tr->events[2 * slot]), st);
+      if (tr->kernel_id) tr->kernel_id[slot] = kid;
+    }
+  }
+  ~TraceScope() {
+    if (slot >= 0) {
+      cudaEventRecord(static_cast<cudaEvent_t>(tr->events[2 * slot + 1]), st);
+      tr->count = slot + 1;
+    }
+  }
+};
+
+// Vocabulary splits S for n_rb row blocks: the most even makespan over the
+// SMs (every unit = one row block x one contiguous run of vocabulary tiles).
+int choose_splits(int64_t n_rb, int64_t n_vt, int sms) {
+  int best = 1;
+  double best_cost = 1e300;
+  const int smax = static_cast<int>(std::min<int64_t>(kMaxSplits, n_vt));
+  for (int S = 1; S <= smax; ++S) {
+    const int64_t units = n_rb * S;
+    const int64_t waves = cdiv(units, sms);
+    const double per_unit = static_cast<double>(cdiv(n_vt, S)) + 0.25;  // +: unit set-up
+    const double cost = static_cast<double>(waves) * per_unit;
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = S;
+    }
+  }
+  return best;
+}
+
+int pick_bn(int64_t d) {
+  int best = 256;
+  int64_t best_waste = cdiv(d, 256) * 256 - d;
+  for (int bn : {192, 128, 64}) {
+    const int64_t w = cdiv(d, bn) * bn - d;
+    if (w < best_waste) {
+      best_waste = w;
+      best = bn;
+    }
+  }
+  return best;
+}
+
+int status_from_word(int32_t w) {
+  if (w & CKL_DEV_BAD_INDEX) return CKL_ERR_BAD_INDEX;
+  if (w & CKL_DEV_BAD_LOGP) return CKL_ERR_BAD_LOGP;
+  if (w & CKL_DEV_TIMEOUT) return CKL_ERR_TIMEOUT;
+  return CKL_OK;
+}
+
+// Shared front half of forward and backward: checks, header reset, prep.
+int common_prep(const uint16_t* H, const uint16_t* W, const int32_t* idx, const float* logp,
+                const uint8_t* mask, int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk,
+                void* ws, size_t ws_bytes, cudaStream_t st, ckl_trace* trace, DevInfo& di,
+                Layout& L) {
+  if (!sizes_ok(T, d, V, K, chunk)) return CKL_ERR_INVALID_ARG;
+  // H, topk_idx and topk_logp may be NULL only for an empty batch.
+  if (!W || !ws || (T > 0 && (!H || !idx || !logp))) return CKL_ERR_INVALID_ARG;
+  if (!aligned16(H) || !aligned16(W) || !aligned16(ws) || !aligned4(idx) || !aligned4(logp))
+    return CKL_ERR_INVALID_ARG;
+  if (K > ckl::PREP_MAXK) return CKL_ERR_UNSUPPORTED;
+  L = layout(T, V, K, chunk);
+  if (ws_bytes < L.total) return CKL_ERR_WORKSPACE;
+  if (!device_info(di)) return CKL_ERR_CUDA;
+  if (di.major != 10) return CKL_ERR_UNSUPPORTED;
+  if (!encode_fn()) return CKL_ERR_CUDA;
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  if (cudaMemsetAsync(w8, 0, kHeaderBytes, st) != cudaSuccess) return CKL_ERR_CUDA;
+  if (T > 0) {
+    Header* hdr = reinterpret_cast<Header*>(w8);
+    TraceScope ts(trace, st, CKL_KERNEL_PREP);
+    const unsigned grid = static_cast<unsigned>(cdiv(T, ckl::PREP_WARPS));
+    ckl::prep_kernel<<<grid, ckl::PREP_WARPS * 32, 0, st>>>(
+        idx, logp, mask, T, K, V, reinterpret_cast<int2*>(w8 + L.pairs),
+        reinterpret_cast<float*>(w8 + L.hp), &hdr->status, &hdr->countN);
+    if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
+  }
+  return CKL_OK;
+}
+
+void fill_common(TcParams& p, uint8_t* w8, const Layout& L, int64_t T, int64_t d, int64_t V,
+                 int32_t K, const uint8_t* mask) {
+  Header* hdr = reinterpret_cast<Header*>(w8);
+  p.T = static_cast<int32_t>(T);
+  p.d = static_cast<int32_t>(d);
+  p.V = static_cast<int32_t>(V);
+  p.K = K;
+  p.n_vt = static_cast<int32_t>(cdiv(V, ckl::BN_V));
+  p.pairs = reinterpret_cast<const int2*>(w8 + L.pairs);
+  p.partials = reinterpret_cast<float4*>(w8 + L.partials);
+  p.mask = mask;
+  p.status = &hdr->status;
+  p.countN = &hdr->countN;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ckl_workspace_bytes(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk) {
+  if (!sizes_ok(T, d, V, K, chunk)) return 0;
+  return layout(T, V, K, chunk).total;
+}
+
+int ckl_forward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
+                const float* topk_logp, const uint8_t* mask, int64_t T, int64_t d, int64_t V,
+                int32_t K, int64_t chunk, float* loss, float* lse, void* workspace,
+                size_t workspace_bytes, void* stream, ckl_trace* trace) {
+  if (!loss || !aligned4(loss) || (T > 0 && (!lse || !aligned4(lse)))) return CKL_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DevInfo di;
+  Layout L;
+  int rc = common_prep(H, W, topk_idx, topk_logp, mask, T, d, V, K, chunk, workspace,
+                       workspace_bytes, st, trace, di, L);
+  if (rc != CKL_OK) return rc;
+  uint8_t* w8 = static_cast<uint8_t*>(workspace);
+  Header* hdr = reinterpret_cast<Header*>(w8);
+  if (T == 0) {
+    TraceScope ts(trace, st, CKL_KERNEL_OTHER);
+    ckl::zero_loss_kernel<<<1, 1, 0, st>>>(loss);
+    return cudaGetLastError() == cudaSuccess ? CKL_OK : CKL_ERR_CUDA;
+  }
+
+  TcParams p;
+  std::memset(&p, 0, sizeof(p));
+  fill_common(p, w8, L, T, d, V, K, mask);
+  p.rows = static_cast<int32_t>(T);
+  p.row0 = 0;
+  p.n_rb = static_cast<int32_t>(cdiv(T, ckl::BM));
+  p.S = choose_splits(p.n_rb, p.n_vt, di.sms);
+  p.n_units = p.n_rb * p.S;
+  if (!map2d(&p.tm[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, H, d, T, d * 2, ckl::BK, ckl::BM,
+             CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map2d(&p.tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, V, d * 2, ckl::BK, ckl::BN_V,
+             CU_TENSOR_MAP_SWIZZLE_128B))
+    return CKL_ERR_CUDA;
+  {
+    TraceScope ts(trace, st, CKL_KERNEL_FWD_GEMM);
+    const int grid = static_cast<int>(std::min<int64_t>(di.sms, p.n_units));
+    ckl::tc_kernel<ckl::MODE_FWD><<<grid, ckl::NUM_THREADS, ckl::SMEM_ALLOC, st>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
+  }
+  {
+    TraceScope ts(trace, st, CKL_KERNEL_FWD_COMBINE);
+    const unsigned grid = static_cast<unsigned>(cdiv(T, ckl::COMBINE_THREADS));
+    ckl::combine_kernel<<<grid, ckl::COMBINE_THREADS, 0, st>>>(
+        reinterpret_cast<const float4*>(w8 + L.partials), p.S,
+        reinterpret_cast<const float*>(w8 + L.hp), mask, T, lse,
+        reinterpret_cast<double*>(w8 + L.blocksums), &hdr->ticket, &hdr->countN, loss);
+    if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
+  }
+  return CKL_OK;
+}
+
+int ckl_backward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
+                 const float* topk_logp, const uint8_t* mask, int64_t T, int64_t d, int64_t V,
+                 int32_t K, int64_t chunk, const float* lse, const float* grad_loss,
+                 uint16_t* dH, float* dW, int32_t accumulate_dW, void* workspace,
+                 size_t workspace_bytes, void* stream, ckl_trace* trace) {
+  if (!dW || !aligned16(dW)) return CKL_ERR_INVALID_ARG;
+  if (T > 0 && (!lse || !aligned4(lse) || !dH || !aligned16(dH))) return CKL_ERR_INVALID_ARG;
+  if (grad_loss && !aligned4(grad_loss)) return CKL_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DevInfo di;
+  Layout L;
+  int rc = common_prep(H, W, topk_idx, topk_logp, mask, T, d, V, K, chunk, workspace,
+                       workspace_bytes, st, trace, di, L);
+  if (rc != CKL_OK) return rc;
+  if (T == 0) {
+    if (!accumulate_dW &&
+        cudaMemsetAsync(dW, 0, static_cast<size_t>(V) * d * sizeof(float), st) != cudaSuccess)
+      return CKL_ERR_CUDA;
+    return CKL_OK;
+  }
+  uint8_t* w8 = static_cast<uint8_t*>(workspace);
+  void* dz = w8 + L.dz;
+  const int bn = pick_bn(d);
+
+  for (int64_t c0 = 0; c0 < T; c0 += chunk) {
+    const int64_t rows = std::min<int64_t>(chunk, T - c0);
+    const uint16_t* Hc = H + c0 * d;
+    // ---- dZ for this chunk
+    {
+      TcParams p;
+      std::memset(&p, 0, sizeof(p));
+      fill_common(p, w8, L, T, d, V, K, mask);
+      p.rows = static_cast<int32_t>(rows);
+      p.row0 = static_cast<int32_t>(c0);
+      p.n_rb = static_cast<int32_t>(cdiv(rows, ckl::BM));
+      p.S = choose_splits(p.n_rb, p.n_vt, di.sms);
+      p.n_units = p.n_rb * p.S;
+      p.lse = lse;
+      if (!map2d(&p.tm[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Hc, d, rows, d * 2, ckl::BK,
+                 ckl::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+          !map2d(&p.tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, V, d * 2, ckl::BK, ckl::BN_V,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+          !map2d(&p.tm[2], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dz, V, rows, L.ldz * 2, 32, 32,
+                 CU_TENSOR_MAP_SWIZZLE_64B))
+        return CKL_ERR_CUDA;
+      TraceScope ts(trace, st, CKL_KERNEL_BWD_DZ);
+      const int grid = static_cast<int>(std::min<int64_t>(di.sms, p.n_units));
+      ckl::tc_kernel<ckl::MODE_DZ><<<grid, ckl::NUM_THREADS, ckl::SMEM_ALLOC, st>>>(p);
+      if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
+    }
+    // ---- dH rows of this chunk and its share of dW, one launch
+    {
+      TcParams p;
+      std::memset(&p, 0, sizeof(p));
+      fill_common(p, w8, L, T, d, V, K, mask);
+      p.rows = static_cast<int32_t>(rows);
+      p.row0 = static_cast<int32_t>(c0);
+      p.bn = bn;
+      p.n_nt = static_cast<int32_t>(cdiv(d, bn));
+      p.n_mt = static_cast<int32_t>(cdiv(V, ckl::BM));
+      p.n5 = static_cast<int32_t>(cdiv(rows, ckl::BM)) * p.n_nt;
+      p.n6 = p.n_mt * p.n_nt;
+      p.c5 = static_cast<int32_t>(cdiv(V, ckl::BK));
+      p.c6 = static_cast<int32_t>(cdiv(rows, ckl::BK));
+      p.dw_store = (c0 == 0 && !accumulate_dW) ? 1 : 0;
+      p.grad_loss = grad_loss;
+      uint16_t* dHc = dH + c0 * d;
+      if (!map2d(&p.tm[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dz, V, rows, L.ldz * 2, ckl::BK,
+                 ckl::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+          !map2d(&p.tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, V, d * 2, 64, ckl::BK,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+          !map2d(&p.tm[2], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dz, V, rows, L.ldz * 2, 64, ckl::BK,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+          !map2d(&p.tm[3], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Hc, d, rows, d * 2, 64, ckl::BK,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+          !map2d(&p.tm[4], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dHc, d, rows, d * 2, 32, 32,
+                 CU_TENSOR_MAP_SWIZZLE_64B) ||
+          !map2d(&p.tm[5], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, dW, d, V, d * 4, 32, 32,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+        return CKL_ERR_CUDA;
+      TraceScope ts(trace, st, CKL_KERNEL_BWD_DHDW);
+      const int grid = static_cast<int>(std::min<int64_t>(di.sms, p.n5 + p.n6));
+      ckl::tc_kernel<ckl::MODE_DHDW><<<grid, ckl::NUM_THREADS, ckl::SMEM_ALLOC, st>>>(p);
+      if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
+    }
+  }
+  return CKL_OK;
+}
+
+int ckl_read_device_status(const void* workspace, void* stream, int32_t* device_status) {
+  if (!workspace || !device_status) return CKL_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t w = 0;
+  if (cudaMemcpyAsync(&w, workspace, sizeof(w), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return CKL_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return CKL_ERR_CUDA;
+  *device_status = w;
+  return status_from_word(w);
+}
+
+const char* ckl_status_string(int32_t status) {
+  switch (status) {
+    case CKL_OK: return "ok";
+    case CKL_ERR_INVALID_ARG: return "invalid argument (null pointer, size or alignment)";
+    case CKL_ERR_UNSUPPORTED: return "unsupported (needs an sm_100 device and K <= 256)";
+    case CKL_ERR_WORKSPACE: return "workspace too small";
+    case CKL_ERR_CUDA: return "CUDA call or kernel launch failed";
+    case CKL_ERR_BAD_INDEX: return "teacher token id outside [0, V)";
+    case CKL_ERR_BAD_LOGP: return "teacher log-prob NaN/+inf, or a row with none finite";
+    case CKL_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out of time";
+    default: return "unknown status";
+  }
+}
+
+int32_t ckl_version(void) { return kVersion; }
+
+}  // extern "C"

@@ -1,0 +1,663 @@
+// Device kernels of the fused chunked KL-distillation loss (sm_100a).
+//
+// The method (Multiverse Computing, "Efficient Knowledge Distillation for
+// LLMs: Offline Top-K Logits and a Fused Chunked KL Loss", as summarised in
+// "LLMのための効率的な知識蒸留：オフラインTop-K LogitsおよびFused Chunked KL
+// Loss", section "2つのシステム変更"): project one chunk of hidden states to
+// logits, fold the chunk into the running loss, drop it; the backward
+// recomputes each chunk.  Here:
+//
+//   prep      per row: check the cached ids, renormalise the K teacher
+//             log-probs (p = softmax over K), sum p log p, sort (id, p) by id,
+//             count the positions that count (N).
+//   tc<FWD>   Z = H W^T on tcgen05 (TMEM accumulators, TMA-fed), never
+//             stored: the epilogue keeps a running max / sum of exp per row
+//             and gathers z at the row's teacher ids (sum_k p_k z_{idx_k}),
+//             one partial per (row, vocabulary split).
+//   combine   merges the splits: lse_t, KL_t = sum p log p - sum p z + lse,
+//             the masked mean (fixed-order sums, deterministic).
+//   tc<DZ>    per chunk: recomputes the same Z tiles (same instruction
+//             sequence, so bit-identical z), dZ = exp(z - lse) - scatter(p)
+//             for rows that count (0 otherwise), stored bf16 [chunk, V].
+//   tc<DHDW>  per chunk, one persistent launch: dH_c = s dZ_c W (A K-major,
+//             B MN-major) and dW (+)= s dZ_c^T H_c (both MN-major), s = g/N,
+//             written by TMA store / TMA reduce-add.
+#pragma once
+
+#include <cfloat>
+#include <climits>
+#include <cstdint>
+
+#include "ckl_ptx.cuh"
+
+namespace ckl {
+
+constexpr int BM = 128;           // rows per tile (TMEM lanes)
+constexpr int BK = 64;            // bf16 elements per 128-byte swizzle row
+constexpr int BN_V = 256;         // vocabulary columns per logit tile
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;        // 16 KB
+constexpr int B_BYTES = 256 * BK * 2;       // 32 KB (largest B tile)
+constexpr int ATOM_BYTES = 64 * BK * 2;     // one 64-wide MN-major atom column, 8 KB
+constexpr int EPI_WARPS = 4;
+constexpr int EPI_BUF = 4096;               // bytes per staging buffer
+constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t ACC_COLS = 256;          // TMEM columns per accumulator buffer
+constexpr int SMEM_A_OFF = 0;
+constexpr int SMEM_B_OFF = STAGES * A_BYTES;
+constexpr int SMEM_EPI_OFF = SMEM_B_OFF + STAGES * B_BYTES;
+constexpr int SMEM_BAR_OFF = SMEM_EPI_OFF + EPI_WARPS * 2 * EPI_BUF;
+constexpr int SMEM_BYTES = SMEM_BAR_OFF + 256;
+constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;  // slack to align the base to 1 KB
+static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float LN2 = 0.6931471805599453f;
+
+enum Mode { MODE_FWD = 0, MODE_DZ = 1, MODE_DHDW = 2 };
+
+struct alignas(64) TcParams {
+  CUtensorMap tm[6];
+  int32_t T, d, V, K;
+  int32_t rows;     // FWD: T; DZ / DHDW: rows of this chunk
+  int32_t row0;     // DZ / DHDW: first row of this chunk
+  int32_t n_rb;     // row blocks of 128 (FWD: over T; DZ / DHDW: over the chunk)
+  int32_t n_vt;     // vocabulary tiles of 256
+  int32_t S;        // vocabulary splits (FWD / DZ)
+  int32_t n_units;  // FWD / DZ: n_rb * S
+  int32_t bn;       // DHDW: d-tile width (64, 128, 192 or 256)
+  int32_t n_nt;     // DHDW: d tiles
+  int32_t n_mt;     // DHDW: vocabulary tiles of 128 (dW rows)
+  int32_t n5, n6;   // DHDW: dH units, dW units
+  int32_t c5, c6;   // DHDW: k-blocks per dH unit (over V), per dW unit (over rows)
+  int32_t dw_store; // DHDW: 1 = this chunk stores dW, 0 = adds into it
+  const int2* pairs;      // [T, K] (id, p as bits), sorted by id per row
+  float4* partials;       // FWD: [T, S] (max of z log2e, sum 2^(..), sum p z, 0)
+  const float* lse;       // DZ: [T]
+  const uint8_t* mask;    // [T] or null (every position counts)
+  const float* grad_loss; // DHDW: [1] or null (= 1)
+  int* status;            // device status word
+  const int* countN;      // N = number of positions that count
+};
+
+// ------------------------------------------------------------------ prep
+// One warp per row; K <= 256 (at most 8 entries per lane).
+constexpr int PREP_WARPS = 8;
+constexpr int PREP_MAXK = 256;
+
+__global__ void __launch_bounds__(PREP_WARPS * 32)
+prep_kernel(const int32_t* __restrict__ idx, const float* __restrict__ logp,
+            const uint8_t* __restrict__ mask, int64_t T, int K, int64_t V,
+            int2* __restrict__ pairs, float* __restrict__ Hp, int* status, int* countN) {
+  __shared__ int s_id[PREP_WARPS][PREP_MAXK];
+  __shared__ int s_cnt[PREP_WARPS];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * PREP_WARPS + warp;
+  int counts = 0;
+  int flags = 0;
+  if (t < T) {
+    int id[8];
+    float lp[8];
+    const int64_t base = t * K;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int k = lane + 32 * e;
+      id[e] = INT_MAX;
+      lp[e] = -INFINITY;
+      if (k < K) {
+        int v = idx[base + k];
+        float l = logp[base + k];
+        if (v < 0 || static_cast<int64_t>(v) >= V) {
+          flags |= CKL_DEV_BAD_INDEX;
+          v = INT_MAX;  // never matches a vocabulary column
+          l = -INFINITY;
+        }
+        if (isnan(l) || l == INFINITY) {
+          flags |= CKL_DEV_BAD_LOGP;
+          l = -INFINITY;
+        }
+        id[e] = v;
+        lp[e] = l;
+      }
+    }
+    float m = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) m = fmaxf(m, lp[e]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (m == -INFINITY) {
+      flags |= CKL_DEV_BAD_LOGP;  // no finite log-prob in this row
+      m = 0.f;
+    }
+    float se = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) se += (lp[e] == -INFINITY) ? 0.f : expf(lp[e] - m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) se += __shfl_xor_sync(0xffffffffu, se, o);
+    const float ell = m + logf(se);
+    float p[8];
+    float hp = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      p[e] = (lp[e] == -INFINITY) ? 0.f : expf(lp[e] - ell);
+      hp += (p[e] > 0.f) ? p[e] * (lp[e] - ell) : 0.f;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) hp += __shfl_xor_sync(0xffffffffu, hp, o);
+    // Sort by (id, original position): rank = number of entries before it.
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int k = lane + 32 * e;
+      if (k < K) s_id[warp][k] = id[e];
+    }
+    __syncwarp();
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int k = lane + 32 * e;
+      if (k < K) {
+        int rank = 0;
+        for (int j = 0; j < K; ++j) {
+          const int o = s_id[warp][j];
+          rank += (o < id[e]) || (o == id[e] && j < k);
+        }
+        pairs[base + rank] = make_int2(id[e], __float_as_int(p[e]));
+      }
+    }
+    if (lane == 0) {
+      Hp[t] = hp;
+      counts = (mask == nullptr || mask[t] != 0) ? 1 : 0;
+    }
+  }
+  if (lane == 0) s_cnt[warp] = counts;
+  flags = __reduce_or_sync(0xffffffffu, flags);
+  if (lane == 0 && flags) atomicOr(status, flags);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int c = 0;
+    for (int w = 0; w < PREP_WARPS; ++w) c += s_cnt[w];
+    if (c) atomicAdd(countN, c);
+  }
+}
+
+// ------------------------------------------------------------------ combine
+constexpr int COMBINE_THREADS = 256;
+
+__global__ void __launch_bounds__(COMBINE_THREADS)
+combine_kernel(const float4* __restrict__ partials, int S, const float* __restrict__ Hp,
+               const uint8_t* __restrict__ mask, int64_t T, float* __restrict__ lse,
+               double* block_sums, unsigned int* ticket, const int* countN, float* loss) {
+  __shared__ double s_w[COMBINE_THREADS / 32];
+  __shared__ bool s_last;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * COMBINE_THREADS + threadIdx.x;
+  float contrib = 0.f;
+  if (t < T) {
+    const float4* pr = partials + t * S;
+    float M = -INFINITY;
+    for (int s = 0; s < S; ++s) M = fmaxf(M, pr[s].x);
+    float se = 0.f, pz = 0.f;
+    for (int s = 0; s < S; ++s) {
+      const float4 q = pr[s];
+      se += q.y * exp2f(q.x - M);
+      pz += q.z;
+    }
+    const float l = (M + log2f(se)) * LN2;
+    lse[t] = l;
+    if (mask == nullptr || mask[t] != 0) contrib = Hp[t] - pz + l;
+  }
+  double v = static_cast<double>(contrib);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if ((threadIdx.x & 31) == 0) s_w[threadIdx.x >> 5] = v;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double b = 0.0;
+    for (int w = 0; w < COMBINE_THREADS / 32; ++w) b += s_w[w];
+    block_sums[blockIdx.x] = b;
+    __threadfence();
+    s_last = (atomicAdd(ticket, 1u) == gridDim.x - 1);
+  }
+  __syncthreads();
+  if (s_last && threadIdx.x == 0) {
+    __threadfence();
+    double total = 0.0;
+    const volatile double* bs = block_sums;
+    for (unsigned b = 0; b < gridDim.x; ++b) total += bs[b];
+    const int n = *reinterpret_cast<const volatile int*>(countN);
+    *loss = (n > 0) ? static_cast<float>(total / static_cast<double>(n)) : 0.f;
+  }
+}
+
+// Loss of an empty batch (T = 0).
+__global__ void zero_loss_kernel(float* loss) { *loss = 0.f; }
+
+// ------------------------------------------------------------------ tc GEMM
+
+// dW units of this CTA: a contiguous range sized so that every CTA's total
+// k-block count (its round-robin dH units plus its dW units) is near equal.
+__device__ __forceinline__ void dw_range(const TcParams& p, int cta, int G, int& b, int& e) {
+  const int64_t c6e = p.c6 + 1;  // +1: the dW epilogue is not free
+  const int64_t total = static_cast<int64_t>(p.n5) * p.c5 + static_cast<int64_t>(p.n6) * c6e;
+  const int64_t target = (total + G - 1) / G;
+  int64_t P = 0, Pc = 0, mine = 0;
+  for (int j = 0; j < G; ++j) {
+    const int64_t cnt5 = (p.n5 > j) ? (p.n5 - j + G - 1) / G : 0;
+    int64_t cap = target - cnt5 * p.c5;
+    cap = cap > 0 ? cap : 0;
+    if (j < cta) Pc += cap;
+    if (j == cta) mine = cap;
+    P += cap;
+  }
+  if (P == 0) {
+    b = static_cast<int>(static_cast<int64_t>(p.n6) * cta / G);
+    e = static_cast<int>(static_cast<int64_t>(p.n6) * (cta + 1) / G);
+  } else {
+    b = static_cast<int>(static_cast<int64_t>(p.n6) * Pc / P);
+    e = static_cast<int>(static_cast<int64_t>(p.n6) * (Pc + mine) / P);
+  }
+}
+
+// Walks this CTA's work in the order every role sees it.  One "job" is one
+// accumulator tile: FWD / DZ: (unit, vocabulary tile); DHDW: one unit.
+struct JobIter {
+  int mode, G, cta;
+  // FWD / DZ
+  int u, vt, vt_hi;
+  // DHDW
+  int phase;  // 0 = dH units, 1 = dW units, 2 = done
+  int b6, e6;
+  __device__ void vt_range(const TcParams& p, int unit, int& lo, int& hi) const {
+    const int s = unit / p.n_rb;
+    lo = static_cast<int>(static_cast<int64_t>(s) * p.n_vt / p.S);
+    hi = static_cast<int>(static_cast<int64_t>(s + 1) * p.n_vt / p.S);
+  }
+  __device__ void init(const TcParams& p, int mode_) {
+    mode = mode_;
+    G = gridDim.x;
+    cta = blockIdx.x;
+    if (mode != MODE_DHDW) {
+      u = cta;
+      vt = vt_hi = 0;
+      if (u < p.n_units) vt_range(p, u, vt, vt_hi);
+    } else {
+      dw_range(p, cta, G, b6, e6);
+      u = cta;
+      phase = 0;
+      if (u >= p.n5) {
+        phase = 1;
+        u = b6;
+        if (u >= e6) phase = 2;
+      }
+    }
+  }
+  __device__ bool valid(const TcParams& p) const {
+    return (mode != MODE_DHDW) ? (u < p.n_units) : (phase < 2);
+  }
+  __device__ void next(const TcParams& p) {
+    if (mode != MODE_DHDW) {
+      if (++vt >= vt_hi) {
+        u += G;
+        if (u < p.n_units) vt_range(p, u, vt, vt_hi);
+      }
+    } else if (phase == 0) {
+      u += G;
+      if (u >= p.n5) {
+        phase = 1;
+        u = b6;
+        if (u >= e6) phase = 2;
+      }
+    } else {
+      if (++u >= e6) phase = 2;
+    }
+  }
+  // FWD / DZ: is this the first / last tile of its unit?
+  __device__ bool first_of_unit(const TcParams& p) const {
+    int lo, hi;
+    vt_range(p, u, lo, hi);
+    return vt == lo;
+  }
+  __device__ bool last_of_unit() const { return vt + 1 == vt_hi; }
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(NUM_THREADS, 1) tc_kernel(const __grid_constant__ TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  // 1 KB-aligned base for the 128-byte swizzled tiles.
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (sbase - raw);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t bar_full = sbase + SMEM_BAR_OFF;              // [STAGES]
+  const uint32_t bar_empty = bar_full + 8 * STAGES;            // [STAGES]
+  const uint32_t bar_tfull = bar_empty + 8 * STAGES;           // [2]
+  const uint32_t bar_tempty = bar_tfull + 16;                  // [2]
+  const uint32_t bar_drain = bar_tempty + 16;                  // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + SMEM_BAR_OFF + 8 * (2 * STAGES + 5));
+
+  if (warp == 0 && lane == 0) {
+    const int n_maps = (MODE == MODE_FWD) ? 2 : (MODE == MODE_DZ) ? 3 : 6;
+#pragma unroll 1
+    for (int i = 0; i < n_maps; ++i) prefetch_tmap(&p.tm[i]);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(bar_tfull + 8 * a, 1);
+      mbar_init(bar_tempty + 8 * a, 32 * EPI_WARPS);
+    }
+    mbar_init(bar_drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0;
+      bool ok = true;
+      JobIter it;
+      it.init(p, MODE);
+      for (; ok && it.valid(p); it.next(p)) {
+        int nkb;
+        int a_x = 0, a_y = 0, b_x = 0, b_y = 0, kind = 0;
+        if (MODE != MODE_DHDW) {
+          const int rb = it.u % p.n_rb;
+          nkb = (p.d + BK - 1) / BK;
+          a_y = rb * BM;
+          b_y = it.vt * BN_V;
+        } else if (it.phase == 0) {
+          kind = 5;
+          nkb = p.c5;
+          a_y = (it.u / p.n_nt) * BM;     // chunk row block
+          b_x = (it.u % p.n_nt) * p.bn;   // d offset
+        } else {
+          kind = 6;
+          nkb = p.c6;
+          a_x = (it.u / p.n_nt) * BM;     // vocabulary row block
+          b_x = (it.u % p.n_nt) * p.bn;
+        }
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, p.status)) { ok = false; break; }
+          const uint32_t fb = bar_full + 8 * stage;
+          const uint32_t sa = sbase + SMEM_A_OFF + stage * A_BYTES;
+          const uint32_t sb = sbase + SMEM_B_OFF + stage * B_BYTES;
+          if (MODE != MODE_DHDW) {
+            mbar_arrive_expect_tx(fb, A_BYTES + B_BYTES);
+            tma_load_2d(sa, &p.tm[0], fb, kb * BK, a_y);
+            tma_load_2d(sb, &p.tm[1], fb, kb * BK, b_y);
+          } else if (kind == 5) {
+            mbar_arrive_expect_tx(fb, A_BYTES + p.bn * BK * 2);
+            tma_load_2d(sa, &p.tm[0], fb, kb * BK, a_y);
+            for (int j = 0; j < p.bn / 64; ++j)
+              tma_load_2d(sb + j * ATOM_BYTES, &p.tm[1], fb, b_x + 64 * j, kb * BK);
+          } else {
+            mbar_arrive_expect_tx(fb, A_BYTES + p.bn * BK * 2);
+            tma_load_2d(sa, &p.tm[2], fb, a_x, kb * BK);
+            tma_load_2d(sa + ATOM_BYTES, &p.tm[2], fb, a_x + 64, kb * BK);
+            for (int j = 0; j < p.bn / 64; ++j)
+              tma_load_2d(sb + j * ATOM_BYTES, &p.tm[3], fb, b_x + 64 * j, kb * BK);
+          }
+          ++issued;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // Let every load this thread started land before the CTA can exit.
+      for (int s = 0; s < STAGES; ++s) {
+        if (issued > static_cast<uint32_t>(s)) {
+          const uint32_t last = issued - 1 - ((issued - 1 - s) % STAGES);
+          mbar_wait(bar_full + 8 * s, (last / STAGES) & 1u, p.status);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      JobIter it;
+      it.init(p, MODE);
+      for (; ok && it.valid(p); it.next(p)) {
+        int nkb;
+        uint32_t idesc;
+        uint32_t a_step, b_step, a_lbo, b_lbo;
+        if (MODE != MODE_DHDW) {
+          nkb = (p.d + BK - 1) / BK;
+          idesc = idesc_bf16(BM, BN_V, 0, 0);
+          a_step = 32; b_step = 32; a_lbo = 16; b_lbo = 16;
+        } else if (it.phase == 0) {
+          nkb = p.c5;
+          idesc = idesc_bf16(BM, p.bn, 0, 1);
+          a_step = 32; b_step = 2048; a_lbo = 16; b_lbo = ATOM_BYTES;
+        } else {
+          nkb = p.c6;
+          idesc = idesc_bf16(BM, p.bn, 1, 1);
+          a_step = 2048; b_step = 2048; a_lbo = ATOM_BYTES; b_lbo = ATOM_BYTES;
+        }
+        if (!mbar_wait(bar_tempty + 8 * acc, acc_phase ^ 1u, p.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc) * ACC_COLS;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(bar_full + 8 * stage, phase, p.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = sbase + SMEM_A_OFF + stage * A_BYTES;
+          const uint32_t sb = sbase + SMEM_B_OFF + stage * B_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(sa + kk * a_step, a_lbo, 1024);
+            const uint64_t bd = sdesc_sw128(sb + kk * b_step, b_lbo, 1024);
+            umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          umma_commit(bar_empty + 8 * stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(bar_tfull + 8 * acc);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      // Every MMA this thread issued has finished before TMEM is released.
+      umma_commit(bar_drain);
+      mbar_wait(bar_drain, 0, p.status);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - 2;                 // 0..3
+    const int lg = warp & 3;                 // TMEM lane group this warp may access
+    const uint32_t lane_off = static_cast<uint32_t>(lg * 32) << 16;
+    const int row_in_tile = lg * 32 + lane;
+    const uint32_t stage_base = sbase + SMEM_EPI_OFF + ew * 2 * EPI_BUF;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    int nstore = 0;
+    bool ok = true;
+
+    // per-row state (FWD / DZ)
+    int64_t t = 0;
+    bool row_ok = false, counts = false;
+    int cur = 0;
+    int nidx = INT_MAX;
+    float np_ = 0.f;
+    float run_m = -INFINITY, run_s = 0.f, run_pz = 0.f;
+    float lse2 = 0.f;
+    float scale = 0.f;
+    if (MODE == MODE_DHDW) {
+      const int n = *p.countN;
+      const float g = (p.grad_loss != nullptr) ? *p.grad_loss : 1.f;
+      scale = (n > 0) ? g / static_cast<float>(n) : 0.f;
+    }
+
+    JobIter it;
+    it.init(p, MODE);
+    for (; ok && it.valid(p); it.next(p)) {
+      if (MODE != MODE_DHDW && it.first_of_unit(p)) {
+        const int rb = it.u % p.n_rb;
+        const int r = rb * BM + row_in_tile;  // row within T (FWD) or the chunk (DZ)
+        row_ok = r < p.rows;
+        t = static_cast<int64_t>(p.row0) + r;
+        counts = row_ok && (p.mask == nullptr || p.mask[t] != 0);
+        run_m = -INFINITY; run_s = 0.f; run_pz = 0.f;
+        nidx = INT_MAX;
+        if (MODE == MODE_DZ && row_ok) lse2 = p.lse[t] * LOG2E;
+        const bool want_ids = (MODE == MODE_FWD) ? row_ok : counts;
+        if (want_ids) {
+          const int2* pr = p.pairs + t * p.K;
+          const int v_lo = it.vt * BN_V;
+          int lo = 0, hi = p.K;
+          while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (pr[mid].x < v_lo) lo = mid + 1; else hi = mid;
+          }
+          cur = lo;
+          if (cur < p.K) { const int2 e = pr[cur]; nidx = e.x; np_ = __int_as_float(e.y); }
+        }
+      }
+      if (!mbar_wait(bar_tfull + 8 * acc, acc_phase, p.status)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t tacc = tmem_base + lane_off + static_cast<uint32_t>(acc) * ACC_COLS;
+
+      if (MODE == MODE_FWD) {
+        for (int c = 0; c < BN_V / 32; ++c) {
+          const int v0 = it.vt * BN_V + c * 32;
+          if (v0 >= p.V) break;
+          float x[32];
+          tmem_ld32(tacc + c * 32, x);
+          if (v0 + 32 > p.V) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) if (v0 + j >= p.V) x[j] = -INFINITY;
+          }
+          float cm = x[0];
+#pragma unroll
+          for (int j = 1; j < 32; ++j) cm = fmaxf(cm, x[j]);
+          const float ym = cm * LOG2E;
+          if (ym > run_m) { run_s *= ex2_approx(run_m - ym); run_m = ym; }
+          float se = 0.f;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) se += ex2_approx(fmaf(x[j], LOG2E, -run_m));
+          run_s += se;
+          while (nidx < v0 + 32) {
+            const int off = nidx - v0;
+            float val = x[0];
+#pragma unroll
+            for (int j = 1; j < 32; ++j) val = (off == j) ? x[j] : val;
+            run_pz = fmaf(np_, val, run_pz);
+            ++cur;
+            if (cur < p.K) { const int2 e = p.pairs[t * p.K + cur]; nidx = e.x; np_ = __int_as_float(e.y); }
+            else nidx = INT_MAX;
+          }
+        }
+      } else if (MODE == MODE_DZ) {
+        const int rb = it.u % p.n_rb;
+        const int y0 = rb * BM + lg * 32;  // first chunk row of this warp's 32 rows
+        for (int c = 0; c < BN_V / 32; ++c) {
+          const int v0 = it.vt * BN_V + c * 32;
+          if (v0 >= p.V) break;
+          float x[32];
+          tmem_ld32(tacc + c * 32, x);
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            x[j] = counts ? ex2_approx(fmaf(x[j], LOG2E, -lse2)) : 0.f;
+          while (nidx < v0 + 32) {
+            const int off = nidx - v0;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) x[j] -= (off == j) ? np_ : 0.f;
+            ++cur;
+            if (cur < p.K) { const int2 e = p.pairs[t * p.K + cur]; nidx = e.x; np_ = __int_as_float(e.y); }
+            else nidx = INT_MAX;
+          }
+          const uint32_t buf = stage_base + (nstore & 1) * EPI_BUF;
+          if (lane == 0) bulk_wait_read<1>();
+          __syncwarp();
+          const uint32_t rowa = buf + lane * 64;
+          const int sw = (lane >> 1) & 3;
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            st_shared_v4(rowa + ((j ^ sw) << 4), pack_bf16x2(x[8 * j], x[8 * j + 1]),
+                         pack_bf16x2(x[8 * j + 2], x[8 * j + 3]),
+                         pack_bf16x2(x[8 * j + 4], x[8 * j + 5]),
+                         pack_bf16x2(x[8 * j + 6], x[8 * j + 7]));
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&p.tm[2], buf, v0, y0);
+            bulk_commit();
+          }
+          ++nstore;
+        }
+      } else {
+        // DHDW: scale and write one accumulator tile.
+        const bool is_dh = (it.phase == 0);
+        const int nt = it.u % p.n_nt;
+        const int y0 = (it.u / p.n_nt) * BM + lg * 32;
+        for (int c = 0; c < p.bn / 32; ++c) {
+          const int x0 = nt * p.bn + c * 32;
+          if (x0 >= p.d) break;
+          float x[32];
+          tmem_ld32(tacc + c * 32, x);
+          const uint32_t buf = stage_base + (nstore & 1) * EPI_BUF;
+          if (lane == 0) bulk_wait_read<1>();
+          __syncwarp();
+          if (is_dh) {
+            const uint32_t rowa = buf + lane * 64;
+            const int sw = (lane >> 1) & 3;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              st_shared_v4(rowa + ((j ^ sw) << 4), pack_bf16x2(x[8 * j] * scale, x[8 * j + 1] * scale),
+                           pack_bf16x2(x[8 * j + 2] * scale, x[8 * j + 3] * scale),
+                           pack_bf16x2(x[8 * j + 4] * scale, x[8 * j + 5] * scale),
+                           pack_bf16x2(x[8 * j + 6] * scale, x[8 * j + 7] * scale));
+          } else {
+            const uint32_t rowa = buf + lane * 128;
+            const int sw = lane & 7;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              st_shared_v4(rowa + ((j ^ sw) << 4), __float_as_uint(x[4 * j] * scale),
+                           __float_as_uint(x[4 * j + 1] * scale),
+                           __float_as_uint(x[4 * j + 2] * scale),
+                           __float_as_uint(x[4 * j + 3] * scale));
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (is_dh) tma_store_2d(&p.tm[4], buf, x0, y0);
+            else if (p.dw_store) tma_store_2d(&p.tm[5], buf, x0, y0);
+            else tma_reduce_add_2d(&p.tm[5], buf, x0, y0);
+            bulk_commit();
+          }
+          ++nstore;
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar_tempty + 8 * acc);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+
+      if (MODE == MODE_FWD && it.last_of_unit() && row_ok) {
+        const int s = it.u / p.n_rb;
+        p.partials[t * p.S + s] = make_float4(run_m, run_s, run_pz, 0.f);
+      }
+    }
+    if (lane == 0) bulk_wait_all<0>();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+}
+
+}  // namespace ckl

@@ -1,0 +1,168 @@
+/*
+ * ckl.h -- C ABI of libckl.so, the fused chunked KL-distillation loss on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method: Multiverse Computing, "Efficient Knowledge Distillation for
+ * LLMs: Offline Top-K Logits and a Fused Chunked KL Loss".  The teacher runs
+ * once and its top-K tokens per position are cached as (token id, log-prob)
+ * pairs ("Дистилляция LLM на одной GPU: offline-кэш и chunked KL loss",
+ * section «Два приёма»).  The loss projects the student's hidden states to
+ * logits one chunk of the sequence at a time, folds the chunk into a running
+ * loss and drops it; the backward recomputes each chunk, so no [T, V] logit
+ * grid is ever held and memory grows linearly with T ("LLMのための効率的な
+ * 知識蒸留...", section "2つのシステム変更").
+ *
+ * The pages do not print the formula.  This library computes the forward KL
+ * of the renormalised teacher top-K against the full-vocabulary student
+ * softmax, averaged over the positions that count:
+ *
+ *   z_tv  = sum_j H[t,j] W[v,j]            lse_t = log sum_v exp(z_tv)
+ *   p_tk  = softmax_k(topk_logp[t,:])      (renormalised over the K entries)
+ *   KL_t  = sum_k p_tk (log p_tk - z_{t,idx_tk} + lse_t)
+ *   loss  = sum_t m_t KL_t / N,  N = sum_t m_t  (loss = 0 when N = 0)
+ *   dL/dz_tv = (g m_t / N) (exp(z_tv - lse_t) - sum_k p_tk [idx_tk = v])
+ *   dH = (dL/dz) W,  dW = (dL/dz)^T H
+ *
+ * Conventions for every call:
+ *  - Layout: every array is row-major and contiguous.  bf16 arrays are passed
+ *    as uint16_t bit patterns.  Pointers are DEVICE pointers owned by the
+ *    caller unless stated otherwise; the library allocates nothing and keeps
+ *    nothing between calls (it only caches per-device properties such as the
+ *    SM count).
+ *  - Sizes: T >= 0 tokens, d >= 8 with d % 8 == 0 (16-byte rows for the TMA
+ *    unit), V >= 1, 1 <= K <= 256, chunk >= 1.  T, d and V are below 2^31.
+ *  - Alignment: H, W, dH, dW and the workspace must be 16-byte aligned.
+ *  - Errors detectable on the host (null pointer, bad size, misalignment,
+ *    small workspace) return a status before anything is enqueued.  A
+ *    failed launch returns CKL_ERR_CUDA.  Errors that depend on the data
+ *    (a teacher id outside [0, V), a teacher row with no finite log-prob, a
+ *    NaN or +inf log-prob, a device wait that ran out of time) are recorded
+ *    in a status word inside the workspace; read it with
+ *    ckl_read_device_status.  Outputs are unspecified when it is non-zero.
+ *  - Asynchrony: calls enqueue work on `stream` (a cudaStream_t; NULL = the
+ *    legacy default stream) and return without waiting.
+ *  - Concurrency: calls that share a workspace must not overlap on the GPU.
+ */
+#ifndef CKL_H_
+#define CKL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CKL_API __attribute__((visibility("default")))
+#else
+#define CKL_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every entry point. */
+typedef enum ckl_status {
+  CKL_OK = 0,
+  CKL_ERR_INVALID_ARG = 1, /* null pointer, size out of range, misalignment */
+  CKL_ERR_UNSUPPORTED = 2, /* no sm_100 device, or K above 256 */
+  CKL_ERR_WORKSPACE = 3,   /* workspace smaller than ckl_workspace_bytes() */
+  CKL_ERR_CUDA = 4,        /* a CUDA runtime/driver call or launch failed */
+  CKL_ERR_BAD_INDEX = 5,   /* device: a teacher id outside [0, V) */
+  CKL_ERR_BAD_LOGP = 6,    /* device: NaN/+inf log-prob, or a row with none finite */
+  CKL_ERR_TIMEOUT = 7      /* device: a bounded wait inside a kernel ran out */
+} ckl_status;
+
+/* Kernel ids written by the optional launch trace. */
+enum {
+  CKL_KERNEL_PREP = 1,        /* teacher cache check, renormalisation, sort, N */
+  CKL_KERNEL_FWD_GEMM = 2,    /* logit GEMM + online log-sum-exp + teacher gather */
+  CKL_KERNEL_FWD_COMBINE = 3, /* merge vocabulary splits: lse, KL, masked mean */
+  CKL_KERNEL_BWD_DZ = 4,      /* logit recompute + dZ = softmax - scatter(p) */
+  CKL_KERNEL_BWD_DHDW = 5,    /* dH = s dZ W and dW += s dZ^T H for one chunk */
+  CKL_KERNEL_OTHER = 6
+};
+
+/*
+ * Optional per-launch trace (tracing / profiling aid).  When a non-NULL
+ * trace is passed, the library records events[2 i] before and events[2 i + 1]
+ * after its i-th kernel launch on `stream`, writes kernel_id[i], and bumps
+ * `count`, for as long as count < capacity.  The events are cudaEvent_t
+ * handles created by the caller; the library never creates or destroys them.
+ * Only the library's own kernels are traced (not memsets).
+ */
+typedef struct ckl_trace {
+  int32_t capacity;   /* in:  launch slots available */
+  int32_t count;      /* in/out: launches recorded so far */
+  void** events;      /* in:  [2 * capacity] cudaEvent_t */
+  int32_t* kernel_id; /* out: [capacity] CKL_KERNEL_* */
+} ckl_trace;
+
+/*
+ * Workspace bytes needed by ckl_forward / ckl_backward for these sizes.
+ * Linear in T: per token K*8 (sorted teacher pairs) + 4 (sum p log p) +
+ * 64*16 (vocabulary-split partials) + 8/256 bytes, plus a chunk x V bf16
+ * buffer for dZ (min(chunk, T) rows of round_up(V, 8) entries) and a
+ * 256-byte header.  Returns 0 for sizes outside the supported range.
+ */
+CKL_API size_t ckl_workspace_bytes(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk);
+
+/*
+ * Forward: the mean KL over the positions that count, and lse for EVERY row
+ * (masked rows too).
+ *   H          [T, d] bf16  student hidden states
+ *   W          [V, d] bf16  output head
+ *   topk_idx   [T, K] int32 cached teacher token ids (repeats allowed; each
+ *                           entry is its own term of the sum over k)
+ *   topk_logp  [T, K] fp32  cached teacher log-probs (any offset per row;
+ *                           renormalised over K; -inf = probability 0)
+ *   mask       [T]    uint8 non-zero = position counts; NULL = all count
+ *   chunk                   rows per backward step (sets the dZ buffer size;
+ *                           the forward holds no per-chunk logits at all)
+ *   loss       [1]    fp32  out
+ *   lse        [T]    fp32  out: log-sum-exp of each row's logits
+ *   workspace               >= ckl_workspace_bytes(T, d, V, K, chunk) bytes
+ *   stream                  cudaStream_t
+ *   trace                   optional launch trace, may be NULL
+ */
+CKL_API int ckl_forward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
+                const float* topk_logp, const uint8_t* mask, int64_t T, int64_t d, int64_t V,
+                int32_t K, int64_t chunk, float* loss, float* lse, void* workspace,
+                size_t workspace_bytes, void* stream, ckl_trace* trace);
+
+/*
+ * Backward by recomputation, one chunk of rows at a time: each chunk's
+ * logits are rebuilt from H and W, turned into the unscaled logit gradient
+ * dZ = exp(z - lse) - scatter(p) (0 on rows that do not count), stored as
+ * bf16 in the workspace (at most chunk x V), then fed to two tensor-core
+ * GEMMs: dH_c = s dZ_c W and dW (+)= s dZ_c^T H_c, with s = g / N.
+ *   lse        [T]    fp32  from ckl_forward on the same inputs
+ *   grad_loss  [1]    fp32  upstream gradient g (device); NULL = 1
+ *   dH         [T, d] bf16  out (fp32 accumulation, rounded once)
+ *   dW         [V, d] fp32  out: overwritten when accumulate_dW == 0, else
+ *                           the gradient is added to its contents
+ * Other arguments as in ckl_forward.  The workspace need not hold anything
+ * from the forward; the teacher cache is prepared again.
+ */
+CKL_API int ckl_backward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
+                 const float* topk_logp, const uint8_t* mask, int64_t T, int64_t d, int64_t V,
+                 int32_t K, int64_t chunk, const float* lse, const float* grad_loss,
+                 uint16_t* dH, float* dW, int32_t accumulate_dW, void* workspace,
+                 size_t workspace_bytes, void* stream, ckl_trace* trace);
+
+/*
+ * Reads the device status word of the last call that used `workspace`:
+ * synchronises `stream`, copies the word to *device_status (a host pointer)
+ * and returns the matching ckl_status (CKL_OK when the word is 0).
+ */
+CKL_API int ckl_read_device_status(const void* workspace, void* stream, int32_t* device_status);
+
+/* Static, human-readable text for a status code. */
+CKL_API const char* ckl_status_string(int32_t status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+CKL_API int32_t ckl_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CKL_H_ */

@@ -1,0 +1,86 @@
+"""The C ABI without a GPU: the library loads, exports what ckl.h declares,
+and rejects bad arguments on the host before touching the device."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "ckl.h")).read()
+    return sorted(set(re.findall(r"CKL_API\s+[\w\s\*]+?\b(ckl_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def ckl():
+    import chunked_kl_loss_ckl_b200 as m
+    return m
+
+
+def test_header_declares_the_entry_points():
+    assert _declared() == ["ckl_backward", "ckl_forward", "ckl_read_device_status",
+                           "ckl_status_string", "ckl_version", "ckl_workspace_bytes"]
+
+
+def test_library_exports_every_declared_symbol(ckl):
+    raw = ctypes.CDLL(ckl.LIB_PATH)
+    for name in _declared():
+        assert hasattr(raw, name), name
+
+
+def test_status_strings_and_version(ckl):
+    for code in range(8):
+        assert ckl.status_string(code) and ckl.status_string(code) != "unknown status"
+    assert ckl.status_string(99) == "unknown status"
+    assert ckl.lib.ckl_version() >= 100
+
+
+def test_workspace_is_linear_in_T(ckl):
+    d, V, K, chunk = 3072, 128256, 100, 1024
+    ws = [ckl.lib.ckl_workspace_bytes(T, d, V, K, chunk) for T in (8192, 16384, 32768, 65536)]
+    # constant second difference (up to 256-byte alignment) = a + b T
+    slope1, slope2, slope3 = ws[1] - ws[0], (ws[2] - ws[1]) / 2, (ws[3] - ws[2]) / 4
+    assert abs(slope1 - slope2) <= 2048 and abs(slope2 - slope3) <= 2048
+    # the per-token part: sorted pairs, p log p, split partials, block sums
+    assert abs(slope1 / 8192 - (K * 8 + 4 + 64 * 16 + 8 / 256)) < 1.0
+    # the dZ buffer is chunk x round_up(V, 8) bf16
+    assert ws[0] - 8192 * (K * 8 + 4 + 64 * 16) >= chunk * V * 2
+
+
+def test_workspace_rejects_bad_sizes(ckl):
+    f = ckl.lib.ckl_workspace_bytes
+    assert f(-1, 64, 100, 4, 8) == 0
+    assert f(10, 60, 100, 4, 8) == 0      # d % 8 != 0
+    assert f(10, 64, 0, 4, 8) == 0
+    assert f(10, 64, 100, 0, 8) == 0
+    assert f(10, 64, 100, 4, 0) == 0
+    assert f(0, 64, 100, 4, 8) > 0         # an empty batch is allowed
+
+
+def test_host_checks_return_before_any_device_work(ckl):
+    L = ckl.lib
+    nul = None
+    # null inputs
+    assert L.ckl_forward(nul, nul, nul, nul, nul, 4, 64, 100, 4, 8, nul, nul, nul, 0, nul,
+                         nul) == 1
+    fake = ctypes.c_void_p(4096)
+    # bad sizes with non-null pointers
+    assert L.ckl_forward(fake, fake, fake, fake, nul, 4, 60, 100, 4, 8, fake, fake, fake, 1 << 20,
+                         nul, nul) == 1
+    # misaligned H
+    assert L.ckl_forward(ctypes.c_void_p(4098), fake, fake, fake, nul, 4, 64, 100, 4, 8, fake,
+                         fake, fake, 1 << 20, nul, nul) == 1
+    # workspace too small
+    assert L.ckl_forward(fake, fake, fake, fake, nul, 4, 64, 100, 4, 8, fake, fake, fake, 16, nul,
+                         nul) == 3
+    # K above the supported maximum
+    assert L.ckl_forward(fake, fake, fake, fake, nul, 4, 64, 100, 300, 8, fake, fake, fake,
+                         1 << 30, nul, nul) == 2
+    # backward: null dW
+    assert L.ckl_backward(fake, fake, fake, fake, nul, 4, 64, 100, 4, 8, fake, nul, fake, nul, 0,
+                          fake, 1 << 20, nul, nul) == 1
+    assert L.ckl_read_device_status(nul, nul, nul) == 1
