@@ -412,3 +412,119 @@ const char* ckl_status_string(int32_t status) {
 int32_t ckl_version(void) { return kVersion; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Forward with library-owned static scratch, for callers that cannot
+// allocate device memory.  The buffer is a file-scope device array; host code
+// must never hand its name to a kernel (on the host the name is only a
+// stand-in), so each device's real address is looked up once with
+// cudaGetSymbolAddress and kept.
+namespace {
+
+static __device__ __align__(256) uint8_t g_static_scratch[CKL_STATIC_SCRATCH_BYTES];
+
+__global__ void copy_status_kernel(const int32_t* src, int32_t* dst) { *dst = *src; }
+
+// Device address of g_static_scratch on the current device, or null.
+void* static_scratch_ptr() {
+  static std::mutex mu;
+  static void* ptrs[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (ptrs[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess) return nullptr;
+    ptrs[dev] = p;
+  }
+  return ptrs[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+int ckl_forward_static_scratch(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
+                               const float* topk_logp, const uint8_t* mask, int64_t T, int64_t d,
+                               int64_t V, int32_t K, float* loss, float* lse,
+                               int32_t* device_status, void* stream) {
+  if (!sizes_ok(T, d, V, K, 1)) return CKL_ERR_INVALID_ARG;
+  if (!W || !loss || !aligned4(loss) || (T > 0 && (!H || !topk_idx || !topk_logp || !lse)))
+    return CKL_ERR_INVALID_ARG;
+  if (!aligned16(H) || !aligned16(W) || !aligned4(topk_idx) || !aligned4(topk_logp) ||
+      !aligned4(lse) || !aligned4(device_status))
+    return CKL_ERR_INVALID_ARG;
+  if (K > ckl::PREP_MAXK) return CKL_ERR_UNSUPPORTED;
+  DevInfo di;
+  if (!device_info(di)) return CKL_ERR_CUDA;
+  if (di.major != 10) return CKL_ERR_UNSUPPORTED;
+  if (!encode_fn()) return CKL_ERR_CUDA;
+
+  // Forward-only layout, sized with the split count this device will use.
+  const int64_t n_rb = cdiv(T, ckl::BM);
+  const int64_t n_vt = cdiv(V, ckl::BN_V);
+  const int S = (T > 0) ? choose_splits(n_rb, n_vt, di.sms) : 1;
+  size_t off = kHeaderBytes;
+  const size_t o_pairs = off;
+  off += align256(static_cast<size_t>(T) * K * 8);
+  const size_t o_hp = off;
+  off += align256(static_cast<size_t>(T) * 4);
+  const size_t o_part = off;
+  off += align256(static_cast<size_t>(T) * S * 16);
+  const size_t o_bs = off;
+  off += align256(static_cast<size_t>(cdiv(T, ckl::COMBINE_THREADS)) * 8);
+  if (off > CKL_STATIC_SCRATCH_BYTES) return CKL_ERR_WORKSPACE;
+
+  uint8_t* w8 = static_cast<uint8_t*>(static_scratch_ptr());
+  if (!w8) return CKL_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Header* hdr = reinterpret_cast<Header*>(w8);
+  // The buffer still holds the previous call's words: clear the header.
+  if (cudaMemsetAsync(w8, 0, kHeaderBytes, st) != cudaSuccess) return CKL_ERR_CUDA;
+  if (T == 0) {
+    ckl::zero_loss_kernel<<<1, 1, 0, st>>>(loss);
+  } else {
+    ckl::prep_kernel<<<static_cast<unsigned>(cdiv(T, ckl::PREP_WARPS)), ckl::PREP_WARPS * 32, 0,
+                       st>>>(topk_idx, topk_logp, mask, T, K, V,
+                             reinterpret_cast<int2*>(w8 + o_pairs),
+                             reinterpret_cast<float*>(w8 + o_hp), &hdr->status, &hdr->countN);
+    if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
+    TcParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.T = static_cast<int32_t>(T);
+    p.d = static_cast<int32_t>(d);
+    p.V = static_cast<int32_t>(V);
+    p.K = K;
+    p.n_vt = static_cast<int32_t>(n_vt);
+    p.pairs = reinterpret_cast<const int2*>(w8 + o_pairs);
+    p.partials = reinterpret_cast<float4*>(w8 + o_part);
+    p.mask = mask;
+    p.status = &hdr->status;
+    p.countN = &hdr->countN;
+    p.rows = static_cast<int32_t>(T);
+    p.row0 = 0;
+    p.n_rb = static_cast<int32_t>(n_rb);
+    p.S = S;
+    p.n_units = p.n_rb * S;
+    if (!map2d(&p.tm[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, H, d, T, d * 2, ckl::BK, ckl::BM,
+               CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map2d(&p.tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, V, d * 2, ckl::BK, ckl::BN_V,
+               CU_TENSOR_MAP_SWIZZLE_128B))
+      return CKL_ERR_CUDA;
+    const int grid = static_cast<int>(std::min<int64_t>(di.sms, p.n_units));
+    ckl::tc_kernel<ckl::MODE_FWD><<<grid, ckl::NUM_THREADS, ckl::SMEM_ALLOC, st>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
+    ckl::combine_kernel<<<static_cast<unsigned>(cdiv(T, ckl::COMBINE_THREADS)),
+                          ckl::COMBINE_THREADS, 0, st>>>(
+        reinterpret_cast<const float4*>(w8 + o_part), S, reinterpret_cast<const float*>(w8 + o_hp),
+        mask, T, lse, reinterpret_cast<double*>(w8 + o_bs), &hdr->ticket, &hdr->countN, loss);
+  }
+  if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
+  if (device_status) {
+    copy_status_kernel<<<1, 1, 0, st>>>(&hdr->status, device_status);
+    if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
+  }
+  return CKL_OK;
+}
+
+}  // extern "C"

@@ -161,6 +161,44 @@ CKL_API const char* ckl_status_string(int32_t status);
 /* Library version: major * 10000 + minor * 100 + patch. */
 CKL_API int32_t ckl_version(void);
 
+/*
+ * Forward without a caller-supplied workspace.
+ *
+ * The paper has no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory: a plugin or extension whose host
+ * runtime owns every device allocation and hands the plugin only its input
+ * and output pointers, or code on a latency-critical path where a device
+ * allocation (which may synchronise the device) is not allowed.  Such a
+ * caller cannot provide the workspace that ckl_forward needs.
+ *
+ * Same inputs and outputs as ckl_forward (there is no `chunk`: the forward
+ * never holds per-chunk logits).  The scratch lives in one library-owned
+ * static device buffer of CKL_STATIC_SCRATCH_BYTES, present on every GPU
+ * that loads the library until the process exits.  It must hold
+ * 256 + T*K*8 + T*4 + T*S*16 + ceil(T/256)*8 bytes (each term rounded up to
+ * 256), where S <= 64 is the number of vocabulary splits the forward picks
+ * for this GPU (37 for T = 8192 on a 148-SM B200): about 23 000 tokens at
+ * K = 100.  Larger problems return CKL_ERR_WORKSPACE before anything is
+ * enqueued.  Nothing is allocated: no cudaMalloc, no cudaFree.
+ *
+ * The first call on each device looks up the buffer's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture begins.  Every call on a device shares the one
+ * buffer, which keeps the previous call's contents (the call clears what
+ * must start at zero): calls that overlap on the GPU -- on different
+ * streams, or from different host threads -- race and give wrong results.
+ *
+ *   device_status  [1] int32, device memory, may be NULL: receives the
+ *                  device status word of this call (CKL_DEV bits: 1 = bad
+ *                  teacher id, 2 = bad log-prob, 4 = timed-out wait; 0 = ok)
+ */
+#define CKL_STATIC_SCRATCH_BYTES (32u << 20)
+CKL_API int ckl_forward_static_scratch(const uint16_t* H, const uint16_t* W,
+                                       const int32_t* topk_idx, const float* topk_logp,
+                                       const uint8_t* mask, int64_t T, int64_t d, int64_t V,
+                                       int32_t K, float* loss, float* lse, int32_t* device_status,
+                                       void* stream);
+
 #ifdef __cplusplus
 }
 #endif

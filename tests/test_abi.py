@@ -22,8 +22,9 @@ def ckl():
 
 
 def test_header_declares_the_entry_points():
-    assert _declared() == ["ckl_backward", "ckl_forward", "ckl_read_device_status",
-                           "ckl_status_string", "ckl_version", "ckl_workspace_bytes"]
+    assert _declared() == ["ckl_backward", "ckl_forward", "ckl_forward_static_scratch",
+                           "ckl_read_device_status", "ckl_status_string", "ckl_version",
+                           "ckl_workspace_bytes"]
 
 
 def test_library_exports_every_declared_symbol(ckl):
