@@ -30,11 +30,13 @@ inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255);
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 struct Layout {
-  size_t pairs, hp, partials, blocksums, dz, total;
-  int64_t ldz;  // dZ row pitch in elements
+  size_t pairs, hp, partials, blocksums, dz, hct, total;
+  int64_t npanels;  // dZ panels of 64 vocabulary columns
+  int64_t cap;      // dZ rows per panel
+  int64_t pitch_t;  // H_c^T row pitch (elements): cap rounded up to 8
 };
 
-Layout layout(int64_t T, int64_t V, int32_t K, int64_t chunk) {
+Layout layout(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk) {
   Layout L{};
   size_t off = kHeaderBytes;
   L.pairs = off;
@@ -45,9 +47,15 @@ Layout layout(int64_t T, int64_t V, int32_t K, int64_t chunk) {
   off += align256(static_cast<size_t>(T) * kMaxSplits * 16);
   L.blocksums = off;
   off += align256(static_cast<size_t>(cdiv(T, ckl::COMBINE_THREADS)) * 8);
-  L.ldz = cdiv(V, 8) * 8;
+  // dZ as 64-column panels: [ceil(V/64)][cap][64] bf16, cap = rows of the largest chunk.
+  L.npanels = cdiv(V, 64);
+  L.cap = std::min(chunk, std::max<int64_t>(T, 1));
   L.dz = off;
-  off += align256(static_cast<size_t>(std::min(chunk, std::max<int64_t>(T, 1))) * L.ldz * 2);
+  off += align256(static_cast<size_t>(L.npanels) * L.cap * 64 * 2);
+  // H_c^T for the dW GEMM: [d][pitch_t] bf16.
+  L.pitch_t = cdiv(L.cap, 8) * 8;
+  L.hct = off;
+  off += align256(static_cast<size_t>(d) * L.pitch_t * 2);
   L.total = off;
   return L;
 }
@@ -96,6 +104,34 @@ bool map2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t in
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D tiled tensor map over [d2][d1][d0] with byte pitches p1 (dim 1), p2 (dim 2).
+bool map3d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1,
+           uint64_t d2, uint64_t p1, uint64_t p2, uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {p1, p2};
+  const cuuint32_t box[3] = {b0, b1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 3-D map with a box of depth b2 along dim 2, 128-byte swizzle.
+bool map3d2(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t p1,
+            uint64_t p2, uint32_t b0, uint32_t b1, uint32_t b2) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {p1, p2};
+  const cuuint32_t box[3] = {b0, b1, b2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct DevInfo {
   int sms = 0;
   int major = 0;
@@ -117,13 +153,16 @@ bool device_info(DevInfo& out) {
   }
   if (!di.attrs_set && di.major == 10) {
     if (cudaFuncSetAttribute(ckl::tc_kernel<ckl::MODE_FWD>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, ckl::SMEM_ALLOC) !=
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             ckl::Cfg<ckl::MODE_FWD>::SMEM_ALLOC) !=
             cudaSuccess ||
         cudaFuncSetAttribute(ckl::tc_kernel<ckl::MODE_DZ>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, ckl::SMEM_ALLOC) !=
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             ckl::Cfg<ckl::MODE_DZ>::SMEM_ALLOC) !=
             cudaSuccess ||
         cudaFuncSetAttribute(ckl::tc_kernel<ckl::MODE_DHDW>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, ckl::SMEM_ALLOC) !=
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             ckl::Cfg<ckl::MODE_DHDW>::SMEM_ALLOC) !=
             cudaSuccess)
       return false;
     di.attrs_set = true;
@@ -202,7 +241,7 @@ int common_prep(const uint16_t* H, const uint16_t* W, const int32_t* idx, const 
   if (!aligned16(H) || !aligned16(W) || !aligned16(ws) || !aligned4(idx) || !aligned4(logp))
     return CKL_ERR_INVALID_ARG;
   if (K > ckl::PREP_MAXK) return CKL_ERR_UNSUPPORTED;
-  L = layout(T, V, K, chunk);
+  L = layout(T, d, V, K, chunk);
   if (ws_bytes < L.total) return CKL_ERR_WORKSPACE;
   if (!device_info(di)) return CKL_ERR_CUDA;
   if (di.major != 10) return CKL_ERR_UNSUPPORTED;
@@ -242,7 +281,7 @@ extern "C" {
 
 size_t ckl_workspace_bytes(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk) {
   if (!sizes_ok(T, d, V, K, chunk)) return 0;
-  return layout(T, V, K, chunk).total;
+  return layout(T, d, V, K, chunk).total;
 }
 
 int ckl_forward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
@@ -280,7 +319,8 @@ int ckl_forward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
   {
     TraceScope ts(trace, st, CKL_KERNEL_FWD_GEMM);
     const int grid = static_cast<int>(std::min<int64_t>(di.sms, p.n_units));
-    ckl::tc_kernel<ckl::MODE_FWD><<<grid, ckl::NUM_THREADS, ckl::SMEM_ALLOC, st>>>(p);
+    ckl::tc_kernel<ckl::MODE_FWD>
+          <<<grid, ckl::Cfg<ckl::MODE_FWD>::THREADS, ckl::Cfg<ckl::MODE_FWD>::SMEM_ALLOC, st>>>(p);
     if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
   }
   {
@@ -337,12 +377,24 @@ int ckl_backward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
                  ckl::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
           !map2d(&p.tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, V, d * 2, ckl::BK, ckl::BN_V,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
-          !map2d(&p.tm[2], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dz, V, rows, L.ldz * 2, 32, 32,
-                 CU_TENSOR_MAP_SWIZZLE_64B))
+          !map3d(&p.tm[2], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dz, 64, rows, L.npanels, 128,
+                 L.cap * 128, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
         return CKL_ERR_CUDA;
       TraceScope ts(trace, st, CKL_KERNEL_BWD_DZ);
       const int grid = static_cast<int>(std::min<int64_t>(di.sms, p.n_units));
-      ckl::tc_kernel<ckl::MODE_DZ><<<grid, ckl::NUM_THREADS, ckl::SMEM_ALLOC, st>>>(p);
+      ckl::tc_kernel<ckl::MODE_DZ>
+          <<<grid, ckl::Cfg<ckl::MODE_DZ>::THREADS, ckl::Cfg<ckl::MODE_DZ>::SMEM_ALLOC, st>>>(p);
+      if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
+    }
+    // ---- H_c^T, the K-major B operand of the dW GEMM
+    void* hct = w8 + L.hct;
+    {
+      TraceScope ts(trace, st, CKL_KERNEL_OTHER);
+      const dim3 grid(static_cast<unsigned>(cdiv(d, 32)), static_cast<unsigned>(cdiv(rows, 32)));
+      ckl::transpose_rows_kernel<<<grid, 256, 0, st>>>(Hc, static_cast<int>(rows),
+                                                       static_cast<int>(d),
+                                                       static_cast<uint16_t*>(hct),
+                                                       static_cast<int>(L.pitch_t));
       if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
     }
     // ---- dH rows of this chunk and its share of dW, one launch
@@ -362,14 +414,13 @@ int ckl_backward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
       p.dw_store = (c0 == 0 && !accumulate_dW) ? 1 : 0;
       p.grad_loss = grad_loss;
       uint16_t* dHc = dH + c0 * d;
-      if (!map2d(&p.tm[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dz, V, rows, L.ldz * 2, ckl::BK,
-                 ckl::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      if (!map3d(&p.tm[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dz, 64, rows, L.npanels, 128,
+                 L.cap * 128, ckl::BK, ckl::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
           !map2d(&p.tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, V, d * 2, 64, ckl::BK,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
-          !map2d(&p.tm[2], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dz, V, rows, L.ldz * 2, 64, ckl::BK,
-                 CU_TENSOR_MAP_SWIZZLE_128B) ||
-          !map2d(&p.tm[3], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Hc, d, rows, d * 2, 64, ckl::BK,
-                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+          !map3d2(&p.tm[2], dz, 64, rows, L.npanels, 128, L.cap * 128, 64, ckl::BK, 2) ||
+          !map2d(&p.tm[3], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hct, rows, d, L.pitch_t * 2, ckl::BK,
+                 bn, CU_TENSOR_MAP_SWIZZLE_128B) ||
           !map2d(&p.tm[4], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dHc, d, rows, d * 2, 32, 32,
                  CU_TENSOR_MAP_SWIZZLE_64B) ||
           !map2d(&p.tm[5], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, dW, d, V, d * 4, 32, 32,
@@ -377,7 +428,8 @@ int ckl_backward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
         return CKL_ERR_CUDA;
       TraceScope ts(trace, st, CKL_KERNEL_BWD_DHDW);
       const int grid = static_cast<int>(std::min<int64_t>(di.sms, p.n5 + p.n6));
-      ckl::tc_kernel<ckl::MODE_DHDW><<<grid, ckl::NUM_THREADS, ckl::SMEM_ALLOC, st>>>(p);
+      ckl::tc_kernel<ckl::MODE_DHDW>
+          <<<grid, ckl::Cfg<ckl::MODE_DHDW>::THREADS, ckl::Cfg<ckl::MODE_DHDW>::SMEM_ALLOC, st>>>(p);
       if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
     }
   }
@@ -512,7 +564,8 @@ int ckl_forward_static_scratch(const uint16_t* H, const uint16_t* W, const int32
                CU_TENSOR_MAP_SWIZZLE_128B))
       return CKL_ERR_CUDA;
     const int grid = static_cast<int>(std::min<int64_t>(di.sms, p.n_units));
-    ckl::tc_kernel<ckl::MODE_FWD><<<grid, ckl::NUM_THREADS, ckl::SMEM_ALLOC, st>>>(p);
+    ckl::tc_kernel<ckl::MODE_FWD>
+          <<<grid, ckl::Cfg<ckl::MODE_FWD>::THREADS, ckl::Cfg<ckl::MODE_FWD>::SMEM_ALLOC, st>>>(p);
     if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
     ckl::combine_kernel<<<static_cast<unsigned>(cdiv(T, ckl::COMBINE_THREADS)),
                           ckl::COMBINE_THREADS, 0, st>>>(

@@ -18,10 +18,12 @@
 //             the masked mean (fixed-order sums, deterministic).
 //   tc<DZ>    per chunk: recomputes the same Z tiles (same instruction
 //             sequence, so bit-identical z), dZ = exp(z - lse) - scatter(p)
-//             for rows that count (0 otherwise), stored bf16 [chunk, V].
+//             for rows that count (0 otherwise), stored bf16 as 64-column
+//             panels [V/64][chunk][64] so every later read of it is contiguous.
 //   tc<DHDW>  per chunk, one persistent launch: dH_c = s dZ_c W (A K-major,
-//             B MN-major) and dW (+)= s dZ_c^T H_c (both MN-major), s = g/N,
-//             written by TMA store / TMA reduce-add.
+//             B MN-major) and dW (+)= s dZ_c^T H_c (A = dZ^T MN-major, B =
+//             H_c^T K-major from a transposed copy), s = g/N, written by TMA
+//             store / TMA reduce-add.
 #pragma once
 
 #include <cfloat>
@@ -35,27 +37,34 @@ namespace ckl {
 constexpr int BM = 128;           // rows per tile (TMEM lanes)
 constexpr int BK = 64;            // bf16 elements per 128-byte swizzle row
 constexpr int BN_V = 256;         // vocabulary columns per logit tile
-constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;        // 16 KB
 constexpr int B_BYTES = 256 * BK * 2;       // 32 KB (largest B tile)
 constexpr int ATOM_BYTES = 64 * BK * 2;     // one 64-wide MN-major atom column, 8 KB
-constexpr int EPI_WARPS = 4;
-constexpr int EPI_BUF = 4096;               // bytes per staging buffer
-constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
+constexpr int EPI_BUF = 4096;               // bytes per staging buffer (2 per epilogue warp)
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COLS = 256;          // TMEM columns per accumulator buffer
-constexpr int SMEM_A_OFF = 0;
-constexpr int SMEM_B_OFF = STAGES * A_BYTES;
-constexpr int SMEM_EPI_OFF = SMEM_B_OFF + STAGES * B_BYTES;
-constexpr int SMEM_BAR_OFF = SMEM_EPI_OFF + EPI_WARPS * 2 * EPI_BUF;
-constexpr int SMEM_BYTES = SMEM_BAR_OFF + 256;
-constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;  // slack to align the base to 1 KB
-static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+
+enum Mode { MODE_FWD = 0, MODE_DZ = 1, MODE_DHDW = 2 };
+
+// Per-kernel pipeline depth and epilogue width.  The dH/dW kernel writes a
+// whole fp32 or bf16 tile per short mainloop (K = chunk rows for dW), so it
+// trades one operand stage for twice the epilogue warps: two warps per TMEM
+// lane group, each taking half of the tile's columns.
+template <int MODE>
+struct Cfg {
+  static constexpr int STAGES = (MODE == MODE_DHDW) ? 3 : 4;
+  static constexpr int EPI_WARPS = (MODE == MODE_DHDW) ? 8 : 4;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int A_OFF = 0;
+  static constexpr int B_OFF = STAGES * A_BYTES;
+  static constexpr int EPI_OFF = B_OFF + STAGES * B_BYTES;
+  static constexpr int BAR_OFF = EPI_OFF + EPI_WARPS * 2 * EPI_BUF;
+  static constexpr int SMEM_ALLOC = BAR_OFF + 256 + 1024;  // + slack to align the base to 1 KB
+  static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+};
 
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
-
-enum Mode { MODE_FWD = 0, MODE_DZ = 1, MODE_DHDW = 2 };
 
 struct alignas(64) TcParams {
   CUtensorMap tm[6];
@@ -228,6 +237,27 @@ combine_kernel(const float4* __restrict__ partials, int S, const float* __restri
   }
 }
 
+// H_c^T for the dW GEMM: Hc [rows, d] (pitch d) -> HcT [d, pitch_t] (rows
+// contiguous), 32 x 32 tiles through shared memory.
+__global__ void __launch_bounds__(256)
+transpose_rows_kernel(const uint16_t* __restrict__ Hc, int rows, int d, uint16_t* __restrict__ HcT,
+                      int pitch_t) {
+  __shared__ uint16_t tile[32][33];
+  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8 threads
+#pragma unroll
+  for (int i = 0; i < 32; i += 8) {
+    const int r = r0 + ty + i, c = c0 + tx;
+    if (r < rows && c < d) tile[ty + i][tx] = Hc[static_cast<int64_t>(r) * d + c];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < 32; i += 8) {
+    const int c = c0 + ty + i, r = r0 + tx;
+    if (r < rows && c < d) HcT[static_cast<int64_t>(c) * pitch_t + r] = tile[tx][ty + i];
+  }
+}
+
 // Loss of an empty batch (T = 0).
 __global__ void zero_loss_kernel(float* loss) { *loss = 0.f; }
 
@@ -320,7 +350,14 @@ struct JobIter {
 };
 
 template <int MODE>
-__global__ void __launch_bounds__(NUM_THREADS, 1) tc_kernel(const __grid_constant__ TcParams p) {
+__global__ void __launch_bounds__(Cfg<MODE>::THREADS, 1)
+tc_kernel(const __grid_constant__ TcParams p) {
+  constexpr int STAGES = Cfg<MODE>::STAGES;
+  constexpr int EPI_WARPS = Cfg<MODE>::EPI_WARPS;
+  constexpr int SMEM_A_OFF = Cfg<MODE>::A_OFF;
+  constexpr int SMEM_B_OFF = Cfg<MODE>::B_OFF;
+  constexpr int SMEM_EPI_OFF = Cfg<MODE>::EPI_OFF;
+  constexpr int SMEM_BAR_OFF = Cfg<MODE>::BAR_OFF;
   extern __shared__ uint8_t smem_raw[];
   // 1 KB-aligned base for the 128-byte swizzled tiles.
   const uint32_t raw = smem_u32(smem_raw);
@@ -397,16 +434,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_kernel(const __grid_constan
             tma_load_2d(sa, &p.tm[0], fb, kb * BK, a_y);
             tma_load_2d(sb, &p.tm[1], fb, kb * BK, b_y);
           } else if (kind == 5) {
+            // dZ is stored as 64-column panels: k-block kb is panel kb.
             mbar_arrive_expect_tx(fb, A_BYTES + p.bn * BK * 2);
-            tma_load_2d(sa, &p.tm[0], fb, kb * BK, a_y);
+            tma_load_3d(sa, &p.tm[0], fb, 0, a_y, kb);
             for (int j = 0; j < p.bn / 64; ++j)
               tma_load_2d(sb + j * ATOM_BYTES, &p.tm[1], fb, b_x + 64 * j, kb * BK);
           } else {
+            // A = dZ^T: one box holding the two 64-column panels of this
+            // vocabulary row block (8 KB each, one MN-major atom column each).
+            // B = H_c^T (d rows x chunk rows, chunk rows contiguous): K-major.
             mbar_arrive_expect_tx(fb, A_BYTES + p.bn * BK * 2);
-            tma_load_2d(sa, &p.tm[2], fb, a_x, kb * BK);
-            tma_load_2d(sa + ATOM_BYTES, &p.tm[2], fb, a_x + 64, kb * BK);
-            for (int j = 0; j < p.bn / 64; ++j)
-              tma_load_2d(sb + j * ATOM_BYTES, &p.tm[3], fb, b_x + 64 * j, kb * BK);
+            tma_load_3d(sa, &p.tm[2], fb, 0, kb * BK, a_x / 64);
+            tma_load_2d(sb, &p.tm[3], fb, kb * BK, b_x);
           }
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -445,8 +484,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_kernel(const __grid_constan
           a_step = 32; b_step = 2048; a_lbo = 16; b_lbo = ATOM_BYTES;
         } else {
           nkb = p.c6;
-          idesc = idesc_bf16(BM, p.bn, 1, 1);
-          a_step = 2048; b_step = 2048; a_lbo = ATOM_BYTES; b_lbo = ATOM_BYTES;
+          idesc = idesc_bf16(BM, p.bn, 1, 0);
+          a_step = 2048; b_step = 32; a_lbo = ATOM_BYTES; b_lbo = 16;
         }
         if (!mbar_wait(bar_tempty + 8 * acc, acc_phase ^ 1u, p.status)) { ok = false; break; }
         tc_fence_after();
@@ -476,8 +515,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_kernel(const __grid_constan
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int ew = warp - 2;                 // 0..3
+    const int ew = warp - 2;                 // 0 .. EPI_WARPS-1
     const int lg = warp & 3;                 // TMEM lane group this warp may access
+    const int half = ew >> 2;                // which share of the tile's columns
+    constexpr int NSHARE = EPI_WARPS / 4;
     const uint32_t lane_off = static_cast<uint32_t>(lg * 32) << 16;
     const int row_in_tile = lg * 32 + lane;
     const uint32_t stage_base = sbase + SMEM_EPI_OFF + ew * 2 * EPI_BUF;
@@ -563,9 +604,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_kernel(const __grid_constan
       } else if (MODE == MODE_DZ) {
         const int rb = it.u % p.n_rb;
         const int y0 = rb * BM + lg * 32;  // first chunk row of this warp's 32 rows
+        const int v_end = (p.V + 63) & ~63;  // dZ panels span round_up(V, 64) columns
         for (int c = 0; c < BN_V / 32; ++c) {
           const int v0 = it.vt * BN_V + c * 32;
-          if (v0 >= p.V) break;
+          if (v0 >= v_end) break;
           float x[32];
           tmem_ld32(tacc + c * 32, x);
 #pragma unroll
@@ -578,6 +620,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_kernel(const __grid_constan
             ++cur;
             if (cur < p.K) { const int2 e = p.pairs[t * p.K + cur]; nidx = e.x; np_ = __int_as_float(e.y); }
             else nidx = INT_MAX;
+          }
+          if (v0 + 32 > p.V) {
+            // the last panel's columns past V are read by the dH GEMM: write 0 there
+#pragma unroll
+            for (int j = 0; j < 32; ++j) if (v0 + j >= p.V) x[j] = 0.f;
           }
           const uint32_t buf = stage_base + (nstore & 1) * EPI_BUF;
           if (lane == 0) bulk_wait_read<1>();
@@ -593,7 +640,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_kernel(const __grid_constan
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&p.tm[2], buf, v0, y0);
+            tma_store_3d(&p.tm[2], buf, v0 & 63, y0, v0 >> 6);
             bulk_commit();
           }
           ++nstore;
@@ -603,7 +650,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_kernel(const __grid_constan
         const bool is_dh = (it.phase == 0);
         const int nt = it.u % p.n_nt;
         const int y0 = (it.u / p.n_nt) * BM + lg * 32;
-        for (int c = 0; c < p.bn / 32; ++c) {
+        const int nch = p.bn / 32 / NSHARE;  // 32-column chunks per warp
+        for (int c = half * nch; c < (half + 1) * nch; ++c) {
           const int x0 = nt * p.bn + c * 32;
           if (x0 >= p.d) break;
           float x[32];

@@ -99,9 +99,11 @@ typedef struct ckl_trace {
 /*
  * Workspace bytes needed by ckl_forward / ckl_backward for these sizes.
  * Linear in T: per token K*8 (sorted teacher pairs) + 4 (sum p log p) +
- * 64*16 (vocabulary-split partials) + 8/256 bytes, plus a chunk x V bf16
- * buffer for dZ (min(chunk, T) rows of round_up(V, 8) entries) and a
- * 256-byte header.  Returns 0 for sizes outside the supported range.
+ * 64*16 (vocabulary-split partials) + 8/256 bytes, plus, independent of T
+ * once T >= chunk, a chunk x V bf16 buffer for dZ (min(chunk, T) rows of
+ * round_up(V, 64) entries), a transposed copy of one chunk of H
+ * (d x round_up(min(chunk, T), 8) bf16) and a 256-byte header.  Returns 0
+ * for sizes outside the supported range.
  */
 CKL_API size_t ckl_workspace_bytes(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk);
 
