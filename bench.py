@@ -46,6 +46,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--memory-sweep", action="store_true",
+                    help="measure workspace and peak device memory vs T at the 256K shape")
     return ap.parse_args(argv)
 
 
@@ -63,6 +65,31 @@ def workload_desc(c):
     return (f"{c['name']}: T={c['T']} d={c['d']} V={c['V']} K={c['K']} chunk={c['chunk']}, "
             f"{masked} positions masked, synthetic (seeded N(0,1) H, N(0,0.02) W, Zipf(1.1) "
             f"teacher ids, sorted N(0,2) teacher log-probs)")
+
+
+def kernel_source_hash() -> str:
+    """Hash of the CUDA sources; ncu traffic figures are valid only for it."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "chunked_kl_loss_ckl_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of ``kernel`` from profiles/traffic.json, or None
+    when absent or taken on other kernel sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f)
+    if t.get("source_hash") != kernel_source_hash():
+        return None
+    e = t.get("kernels", {}).get(workload, {}).get(kernel)
+    return None if e is None else float(e["dram_bytes_per_launch"])
 
 
 def flops_per_token(c):
@@ -162,8 +189,11 @@ def cpu_oracle_sample(c, target_s: float, rows: int | None = None):
         return time.perf_counter() - t0
 
     if rows is None:
-        t_probe = run(16)
-        rows = int(min(2048, max(16, 16 * target_s / max(t_probe, 1e-3))))
+        # fixed cost (widening W to fp64) + per-row cost, from two probes
+        t16, t48 = run(16), run(48)
+        per_row = max((t48 - t16) / 32.0, 1e-4)
+        fixed = max(t16 - 16 * per_row, 0.0)
+        rows = int(min(4096, max(16, (target_s - fixed) / per_row)))
     dt = run(rows)
     return rows / dt, rows, dt, threads
 
@@ -264,7 +294,9 @@ def bench_ours(args):
                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                     "peak_source": f"{peak_src} bf16_tflops_sustained",
                     "avg_launch_ms": round(dom_avg_ms, 4), "launches": per[dom][0],
-                    "traffic": None}
+                    "traffic": profiled_traffic(dom, args.config),
+                    "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + "
+                                    "dram__bytes_write.sum)"}
     kernels = {k: {"launches": v[0], "total_ms": round(v[1], 3),
                    "share": round(v[1] / sum(x[1] for x in per.values()), 4)}
                for k, v in sorted(per.items())}
@@ -382,10 +414,58 @@ def bench_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def memory_sweep(args):
+    """Workspace and peak device memory of forward + backward vs T at the
+    256K shape (d=4096, V=128256, K=100, chunk=4096, 1 % of each 32K
+    sequence masked).  Inputs are seeded device tensors of the workload's
+    shapes; memory does not depend on their values."""
+    import torch
+    import chunked_kl_loss_ckl_b200 as ckl
+    d, V, K, chunk = 4096, 128256, 100, 4096
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(args.seed)
+    W = (torch.randn(V, d, generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    rows = []
+    for T in (8192, 16384, 32768, 65536, 131072, 262144):
+        H = torch.randn(T, d, generator=g, device=dev).to(torch.bfloat16)
+        idx = torch.randint(0, V, (T, K), generator=g, device=dev, dtype=torch.int32)
+        logp = torch.log_softmax(2.0 * torch.randn(T, K, generator=g, device=dev), dim=1)
+        mask = torch.ones(T, dtype=torch.uint8, device=dev)
+        mask.view(-1, min(T, 32768))[:, -328:] = 0
+        torch.cuda.synchronize()
+        base = torch.cuda.memory_allocated(dev)
+        torch.cuda.reset_peak_memory_stats(dev)
+        ws = ckl.new_workspace(T, d, V, K, chunk, dev)
+        loss, lse = ckl.forward(H, W, idx, logp, mask, chunk, workspace=ws)
+        dH, dW = ckl.backward(H, W, idx, logp, mask, lse, chunk=chunk, workspace=ws)
+        torch.cuda.synchronize()
+        peak = torch.cuda.max_memory_allocated(dev) - base
+        outputs = lse.numel() * 4 + 4 + dH.numel() * 2 + dW.numel() * 4
+        rows.append({"T": T, "workspace_bytes": ws.numel(),
+                     "peak_minus_inputs_bytes": int(peak),
+                     "peak_minus_inputs_and_outputs_bytes": int(peak - outputs),
+                     "loss": float(loss.item())})
+        del H, idx, logp, mask, ws, loss, lse, dH, dW
+        torch.cuda.empty_cache()
+    Ts = np.array([r["T"] for r in rows], float)
+    fit = {}
+    for key in ("workspace_bytes", "peak_minus_inputs_and_outputs_bytes"):
+        y = np.array([r[key] for r in rows], float)
+        A = np.stack([np.ones_like(Ts), Ts], 1)
+        (a, b), *_ = np.linalg.lstsq(A, y, rcond=None)
+        resid = float(np.max(np.abs(A @ np.array([a, b]) - y) / y))
+        fit[key] = {"a_bytes": a, "b_bytes_per_token": b, "max_rel_residual": resid}
+    print(json.dumps({"memory_vs_T": rows, "linear_fit": fit,
+                      "shape": {"d": d, "V": V, "K": K, "chunk": chunk}}), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    if args.memory_sweep:
+        memory_sweep(args)
+        return
     if args.impl == "reference":
         bench_reference(args)
     else:

@@ -46,14 +46,15 @@ constexpr uint32_t ACC_COLS = 256;          // TMEM columns per accumulator buff
 
 enum Mode { MODE_FWD = 0, MODE_DZ = 1, MODE_DHDW = 2 };
 
-// Per-kernel pipeline depth and epilogue width.  The dH/dW kernel writes a
-// whole fp32 or bf16 tile per short mainloop (K = chunk rows for dW), so it
-// trades one operand stage for twice the epilogue warps: two warps per TMEM
-// lane group, each taking half of the tile's columns.
+// Pipeline depth and epilogue width.  Four 48 KB operand stages fill the
+// shared memory beside the epilogue staging.  The epilogue code also runs
+// with eight warps (two per TMEM lane group, each taking half of a tile's
+// columns), which measured slower for every kernel here because it costs one
+// operand stage: the epilogue is not the bottleneck.
 template <int MODE>
 struct Cfg {
-  static constexpr int STAGES = (MODE == MODE_DHDW) ? 3 : 4;
-  static constexpr int EPI_WARPS = (MODE == MODE_DHDW) ? 8 : 4;
+  static constexpr int STAGES = 4;
+  static constexpr int EPI_WARPS = 4;
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static constexpr int A_OFF = 0;
   static constexpr int B_OFF = STAGES * A_BYTES;
