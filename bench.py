@@ -243,8 +243,11 @@ def bench_ours(args):
     if rc != 0:
         raise SystemExit(f"device status {rc} ({word}) after warm-up")
 
-    n_launch = 3 + 1 + 2 * ((T + chunk - 1) // chunk)
-    trace = ckl.Trace(capacity=args.steps * n_launch + 8)
+    # forward: prep, logits GEMM, combine; backward: prep + per chunk
+    # (dZ GEMM, H_c transpose, dH/dW GEMM); the capacity leaves headroom and
+    # a full trace is treated as an error below.
+    n_launch = 3 + 1 + 3 * ((T + chunk - 1) // chunk)
+    trace = ckl.Trace(capacity=args.steps * (n_launch + 4) + 16)
     uuid = None
     try:
         uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
@@ -272,6 +275,8 @@ def bench_ours(args):
     value = tokens / (ms_step / 1e3)
     tflops = flops_per_token(c) * tokens / (ms_step / 1e3) / 1e12
 
+    if trace.count >= trace.capacity:
+        raise SystemExit("launch trace overflowed: per-kernel times would be incomplete")
     # per-kernel times from the library's own launch events
     per = {}
     for name, ms in trace.durations():
