@@ -132,11 +132,64 @@ bool map3d2(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Every GEMM runs on CTA pairs sharing one cta_group::2 MMA (each CTA
+// stages half of the B operand); one scheduling slot = one pair.
+constexpr bool kPair = true;
+constexpr int kSlotCTAs = kPair ? 2 : 1;
+constexpr int64_t kMB = kPair ? 2 * ckl::BM : ckl::BM;  // rows of one job's M extent
+
 struct DevInfo {
   int sms = 0;
   int major = 0;
   bool attrs_set = false;
+  int slots[3] = {0, 0, 0};  // co-resident CTA pairs per GEMM mode
 };
+
+template <int MODE>
+cudaLaunchConfig_t tc_config(int slots, cudaStream_t st, cudaLaunchAttribute* attr) {
+  using C = ckl::Cfg<MODE, kPair>;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(slots * kSlotCTAs));
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_ALLOC;
+  cfg.stream = st;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kSlotCTAs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
+template <int MODE>
+bool setup_mode(DevInfo& di) {
+  using C = ckl::Cfg<MODE, kPair>;
+  if (cudaFuncSetAttribute(ckl::tc_kernel<MODE, kPair>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) !=
+      cudaSuccess)
+    return false;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = tc_config<MODE>(di.sms / kSlotCTAs, nullptr, attr);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, ckl::tc_kernel<MODE, kPair>, &cfg) != cudaSuccess ||
+      n <= 0) {
+    cudaGetLastError();
+    n = di.sms / kSlotCTAs;
+  }
+  di.slots[MODE] = std::min(n, di.sms / kSlotCTAs);
+  return true;
+}
+
+// Launches one persistent GEMM on min(co-resident slots, units) CTA pairs.
+template <int MODE>
+int launch_tc(const TcParams& p, int64_t units, const DevInfo& di, cudaStream_t st) {
+  const int slots = static_cast<int>(std::min<int64_t>(di.slots[MODE], units));
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = tc_config<MODE>(slots, st, attr);
+  return cudaLaunchKernelEx(&cfg, ckl::tc_kernel<MODE, kPair>, p) == cudaSuccess ? CKL_OK
+                                                                                 : CKL_ERR_CUDA;
+}
 
 bool device_info(DevInfo& out) {
   static std::mutex mu;
@@ -152,18 +205,8 @@ bool device_info(DevInfo& out) {
       return false;
   }
   if (!di.attrs_set && di.major == 10) {
-    if (cudaFuncSetAttribute(ckl::tc_kernel<ckl::MODE_FWD>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             ckl::Cfg<ckl::MODE_FWD>::SMEM_ALLOC) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(ckl::tc_kernel<ckl::MODE_DZ>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             ckl::Cfg<ckl::MODE_DZ>::SMEM_ALLOC) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(ckl::tc_kernel<ckl::MODE_DHDW>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             ckl::Cfg<ckl::MODE_DHDW>::SMEM_ALLOC) !=
-            cudaSuccess)
+    if (!setup_mode<ckl::MODE_FWD>(di) || !setup_mode<ckl::MODE_DZ>(di) ||
+        !setup_mode<ckl::MODE_DHDW>(di))
       return false;
     di.attrs_set = true;
   }
@@ -214,6 +257,7 @@ int pick_bn(int64_t d) {
   int best = 256;
   int64_t best_waste = cdiv(d, 256) * 256 - d;
   for (int bn : {192, 128, 64}) {
+    if (kPair && bn % 128 != 0) continue;  // each CTA of a pair stages bn/2 columns
     const int64_t w = cdiv(d, bn) * bn - d;
     if (w < best_waste) {
       best_waste = w;
@@ -308,20 +352,17 @@ int ckl_forward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
   fill_common(p, w8, L, T, d, V, K, mask);
   p.rows = static_cast<int32_t>(T);
   p.row0 = 0;
-  p.n_rb = static_cast<int32_t>(cdiv(T, ckl::BM));
-  p.S = choose_splits(p.n_rb, p.n_vt, di.sms);
+  p.n_rb = static_cast<int32_t>(cdiv(T, kMB));
+  p.S = choose_splits(p.n_rb, p.n_vt, di.slots[ckl::MODE_FWD]);
   p.n_units = p.n_rb * p.S;
   if (!map2d(&p.tm[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, H, d, T, d * 2, ckl::BK, ckl::BM,
              CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !map2d(&p.tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, V, d * 2, ckl::BK, ckl::BN_V,
-             CU_TENSOR_MAP_SWIZZLE_128B))
+      !map2d(&p.tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, V, d * 2, ckl::BK,
+             ckl::BN_V / kSlotCTAs, CU_TENSOR_MAP_SWIZZLE_128B))
     return CKL_ERR_CUDA;
   {
     TraceScope ts(trace, st, CKL_KERNEL_FWD_GEMM);
-    const int grid = static_cast<int>(std::min<int64_t>(di.sms, p.n_units));
-    ckl::tc_kernel<ckl::MODE_FWD>
-          <<<grid, ckl::Cfg<ckl::MODE_FWD>::THREADS, ckl::Cfg<ckl::MODE_FWD>::SMEM_ALLOC, st>>>(p);
-    if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
+    if (launch_tc<ckl::MODE_FWD>(p, p.n_units, di, st) != CKL_OK) return CKL_ERR_CUDA;
   }
   {
     TraceScope ts(trace, st, CKL_KERNEL_FWD_COMBINE);
@@ -369,22 +410,19 @@ int ckl_backward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
       fill_common(p, w8, L, T, d, V, K, mask);
       p.rows = static_cast<int32_t>(rows);
       p.row0 = static_cast<int32_t>(c0);
-      p.n_rb = static_cast<int32_t>(cdiv(rows, ckl::BM));
-      p.S = choose_splits(p.n_rb, p.n_vt, di.sms);
+      p.n_rb = static_cast<int32_t>(cdiv(rows, kMB));
+      p.S = choose_splits(p.n_rb, p.n_vt, di.slots[ckl::MODE_DZ]);
       p.n_units = p.n_rb * p.S;
       p.lse = lse;
       if (!map2d(&p.tm[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Hc, d, rows, d * 2, ckl::BK,
                  ckl::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-          !map2d(&p.tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, V, d * 2, ckl::BK, ckl::BN_V,
-                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+          !map2d(&p.tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, V, d * 2, ckl::BK,
+                 ckl::BN_V / kSlotCTAs, CU_TENSOR_MAP_SWIZZLE_128B) ||
           !map3d(&p.tm[2], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dz, 64, rows, L.npanels, 128,
                  L.cap * 128, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
         return CKL_ERR_CUDA;
       TraceScope ts(trace, st, CKL_KERNEL_BWD_DZ);
-      const int grid = static_cast<int>(std::min<int64_t>(di.sms, p.n_units));
-      ckl::tc_kernel<ckl::MODE_DZ>
-          <<<grid, ckl::Cfg<ckl::MODE_DZ>::THREADS, ckl::Cfg<ckl::MODE_DZ>::SMEM_ALLOC, st>>>(p);
-      if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
+      if (launch_tc<ckl::MODE_DZ>(p, p.n_units, di, st) != CKL_OK) return CKL_ERR_CUDA;
     }
     // ---- H_c^T, the K-major B operand of the dW GEMM
     void* hct = w8 + L.hct;
@@ -406,8 +444,8 @@ int ckl_backward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
       p.row0 = static_cast<int32_t>(c0);
       p.bn = bn;
       p.n_nt = static_cast<int32_t>(cdiv(d, bn));
-      p.n_mt = static_cast<int32_t>(cdiv(V, ckl::BM));
-      p.n5 = static_cast<int32_t>(cdiv(rows, ckl::BM)) * p.n_nt;
+      p.n_mt = static_cast<int32_t>(cdiv(V, kMB));
+      p.n5 = static_cast<int32_t>(cdiv(rows, kMB)) * p.n_nt;
       p.n6 = p.n_mt * p.n_nt;
       p.c5 = static_cast<int32_t>(cdiv(V, ckl::BK));
       p.c6 = static_cast<int32_t>(cdiv(rows, ckl::BK));
@@ -420,17 +458,14 @@ int ckl_backward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
           !map3d2(&p.tm[2], dz, 64, rows, L.npanels, 128, L.cap * 128, 64, ckl::BK, 2) ||
           !map2d(&p.tm[3], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hct, rows, d, L.pitch_t * 2, ckl::BK,
-                 bn, CU_TENSOR_MAP_SWIZZLE_128B) ||
+                 bn / kSlotCTAs, CU_TENSOR_MAP_SWIZZLE_128B) ||
           !map2d(&p.tm[4], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dHc, d, rows, d * 2, 32, 32,
                  CU_TENSOR_MAP_SWIZZLE_64B) ||
           !map2d(&p.tm[5], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, dW, d, V, d * 4, 32, 32,
                  CU_TENSOR_MAP_SWIZZLE_128B))
         return CKL_ERR_CUDA;
       TraceScope ts(trace, st, CKL_KERNEL_BWD_DHDW);
-      const int grid = static_cast<int>(std::min<int64_t>(di.sms, p.n5 + p.n6));
-      ckl::tc_kernel<ckl::MODE_DHDW>
-          <<<grid, ckl::Cfg<ckl::MODE_DHDW>::THREADS, ckl::Cfg<ckl::MODE_DHDW>::SMEM_ALLOC, st>>>(p);
-      if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
+      if (launch_tc<ckl::MODE_DHDW>(p, p.n5 + p.n6, di, st) != CKL_OK) return CKL_ERR_CUDA;
     }
   }
   return CKL_OK;
@@ -513,9 +548,9 @@ int ckl_forward_static_scratch(const uint16_t* H, const uint16_t* W, const int32
   if (!encode_fn()) return CKL_ERR_CUDA;
 
   // Forward-only layout, sized with the split count this device will use.
-  const int64_t n_rb = cdiv(T, ckl::BM);
+  const int64_t n_rb = cdiv(T, kMB);
   const int64_t n_vt = cdiv(V, ckl::BN_V);
-  const int S = (T > 0) ? choose_splits(n_rb, n_vt, di.sms) : 1;
+  const int S = (T > 0) ? choose_splits(n_rb, n_vt, di.slots[ckl::MODE_FWD]) : 1;
   size_t off = kHeaderBytes;
   const size_t o_pairs = off;
   off += align256(static_cast<size_t>(T) * K * 8);
@@ -560,13 +595,10 @@ int ckl_forward_static_scratch(const uint16_t* H, const uint16_t* W, const int32
     p.n_units = p.n_rb * S;
     if (!map2d(&p.tm[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, H, d, T, d * 2, ckl::BK, ckl::BM,
                CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !map2d(&p.tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, V, d * 2, ckl::BK, ckl::BN_V,
-               CU_TENSOR_MAP_SWIZZLE_128B))
+        !map2d(&p.tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, V, d * 2, ckl::BK,
+               ckl::BN_V / kSlotCTAs, CU_TENSOR_MAP_SWIZZLE_128B))
       return CKL_ERR_CUDA;
-    const int grid = static_cast<int>(std::min<int64_t>(di.sms, p.n_units));
-    ckl::tc_kernel<ckl::MODE_FWD>
-          <<<grid, ckl::Cfg<ckl::MODE_FWD>::THREADS, ckl::Cfg<ckl::MODE_FWD>::SMEM_ALLOC, st>>>(p);
-    if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
+    if (launch_tc<ckl::MODE_FWD>(p, p.n_units, di, st) != CKL_OK) return CKL_ERR_CUDA;
     ckl::combine_kernel<<<static_cast<unsigned>(cdiv(T, ckl::COMBINE_THREADS)),
                           ckl::COMBINE_THREADS, 0, st>>>(
         reinterpret_cast<const float4*>(w8 + o_part), S, reinterpret_cast<const float*>(w8 + o_hp),

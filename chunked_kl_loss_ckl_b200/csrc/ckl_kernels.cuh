@@ -46,19 +46,23 @@ constexpr uint32_t ACC_COLS = 256;          // TMEM columns per accumulator buff
 
 enum Mode { MODE_FWD = 0, MODE_DZ = 1, MODE_DHDW = 2 };
 
-// Pipeline depth and epilogue width.  Four 48 KB operand stages fill the
-// shared memory beside the epilogue staging.  The epilogue code also runs
-// with eight warps (two per TMEM lane group, each taking half of a tile's
-// columns), which measured slower for every kernel here because it costs one
-// operand stage: the epilogue is not the bottleneck.
-template <int MODE>
+// Pipeline depth and epilogue width.  A single CTA holds a 128 x 256 tile:
+// four 48 KB operand stages fill the shared memory beside the epilogue
+// staging.  A CTA pair (PAIR) shares one 256-row MMA: each CTA stages its own
+// 128 rows of A and half of B, 32 KB per stage, so six stages fit.  The
+// epilogue code also runs with eight warps (two per TMEM lane group, each
+// taking half of a tile's columns); that measured slower here because it
+// costs an operand stage: the epilogue is not the bottleneck.
+template <int MODE, bool PAIR>
 struct Cfg {
-  static constexpr int STAGES = 4;
+  static constexpr int STAGES = PAIR ? 6 : 4;
   static constexpr int EPI_WARPS = 4;
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int B_STAGE = PAIR ? B_BYTES / 2 : B_BYTES;
+  static constexpr int MB = PAIR ? 2 * BM : BM;  // rows of one job's M extent
   static constexpr int A_OFF = 0;
   static constexpr int B_OFF = STAGES * A_BYTES;
-  static constexpr int EPI_OFF = B_OFF + STAGES * B_BYTES;
+  static constexpr int EPI_OFF = B_OFF + STAGES * B_STAGE;
   static constexpr int BAR_OFF = EPI_OFF + EPI_WARPS * 2 * EPI_BUF;
   static constexpr int SMEM_ALLOC = BAR_OFF + 256 + 1024;  // + slack to align the base to 1 KB
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
@@ -291,7 +295,7 @@ __device__ __forceinline__ void dw_range(const TcParams& p, int cta, int G, int&
 // Walks this CTA's work in the order every role sees it.  One "job" is one
 // accumulator tile: FWD / DZ: (unit, vocabulary tile); DHDW: one unit.
 struct JobIter {
-  int mode, G, cta;
+  int mode, G, cta;  // G scheduling slots (CTAs, or CTA pairs); this slot
   // FWD / DZ
   int u, vt, vt_hi;
   // DHDW
@@ -302,10 +306,10 @@ struct JobIter {
     lo = static_cast<int>(static_cast<int64_t>(s) * p.n_vt / p.S);
     hi = static_cast<int>(static_cast<int64_t>(s + 1) * p.n_vt / p.S);
   }
-  __device__ void init(const TcParams& p, int mode_) {
+  __device__ void init(const TcParams& p, int mode_, int per_slot) {
     mode = mode_;
-    G = gridDim.x;
-    cta = blockIdx.x;
+    G = gridDim.x / per_slot;
+    cta = blockIdx.x / per_slot;
     if (mode != MODE_DHDW) {
       u = cta;
       vt = vt_hi = 0;
@@ -350,50 +354,59 @@ struct JobIter {
   __device__ bool last_of_unit() const { return vt + 1 == vt_hi; }
 };
 
-template <int MODE>
-__global__ void __launch_bounds__(Cfg<MODE>::THREADS, 1)
+template <int MODE, bool PAIR>
+__global__ void __launch_bounds__(Cfg<MODE, PAIR>::THREADS, 1)
 tc_kernel(const __grid_constant__ TcParams p) {
-  constexpr int STAGES = Cfg<MODE>::STAGES;
-  constexpr int EPI_WARPS = Cfg<MODE>::EPI_WARPS;
-  constexpr int SMEM_A_OFF = Cfg<MODE>::A_OFF;
-  constexpr int SMEM_B_OFF = Cfg<MODE>::B_OFF;
-  constexpr int SMEM_EPI_OFF = Cfg<MODE>::EPI_OFF;
-  constexpr int SMEM_BAR_OFF = Cfg<MODE>::BAR_OFF;
+  using C = Cfg<MODE, PAIR>;
+  constexpr int STAGES = C::STAGES;
+  constexpr int EPI_WARPS = C::EPI_WARPS;
+  constexpr int B_STAGE = C::B_STAGE;
+  constexpr int MB = C::MB;
+  constexpr uint32_t MMA_M = PAIR ? 2 * BM : BM;
   extern __shared__ uint8_t smem_raw[];
-  // 1 KB-aligned base for the 128-byte swizzled tiles.
+  // 1 KB-aligned base for the 128-byte swizzled tiles.  Both CTAs of a pair
+  // get the same layout, so every offset names the same slot in either CTA.
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (sbase - raw);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t bar_full = sbase + SMEM_BAR_OFF;              // [STAGES]
-  const uint32_t bar_empty = bar_full + 8 * STAGES;            // [STAGES]
-  const uint32_t bar_tfull = bar_empty + 8 * STAGES;           // [2]
-  const uint32_t bar_tempty = bar_tfull + 16;                  // [2]
-  const uint32_t bar_drain = bar_tempty + 16;                  // [1]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + SMEM_BAR_OFF + 8 * (2 * STAGES + 5));
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;  // 0 = the pair's leader
+  const bool leader = (rank == 0);
+  const uint32_t bar_full = sbase + C::BAR_OFF;               // [STAGES] (leader's count both)
+  const uint32_t bar_empty = bar_full + 8 * STAGES;           // [STAGES]
+  const uint32_t bar_tfull = bar_empty + 8 * STAGES;          // [2]
+  const uint32_t bar_tempty = bar_tfull + 16;                 // [2] (leader's count both)
+  const uint32_t bar_drain = bar_tempty + 16;                 // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::BAR_OFF + 8 * (2 * STAGES + 5));
 
   if (warp == 0 && lane == 0) {
     const int n_maps = (MODE == MODE_FWD) ? 2 : (MODE == MODE_DZ) ? 3 : 6;
 #pragma unroll 1
     for (int i = 0; i < n_maps; ++i) prefetch_tmap(&p.tm[i]);
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_full + 8 * s, PAIR ? 2 : 1);
       mbar_init(bar_empty + 8 * s, 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(bar_tfull + 8 * a, 1);
-      mbar_init(bar_tempty + 8 * a, 32 * EPI_WARPS);
+      mbar_init(bar_tempty + 8 * a, (PAIR ? 2 : 1) * 32 * EPI_WARPS);
     }
     mbar_init(bar_drain, 1);
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if (PAIR) cluster_sync();  // the peer may signal the leader's barriers from here on
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
 
@@ -405,87 +418,115 @@ tc_kernel(const __grid_constant__ TcParams p) {
       uint32_t issued = 0;
       bool ok = true;
       JobIter it;
-      it.init(p, MODE);
+      it.init(p, MODE, PAIR ? 2 : 1);
       for (; ok && it.valid(p); it.next(p)) {
         int nkb;
         int a_x = 0, a_y = 0, b_x = 0, b_y = 0, kind = 0;
+        const int half_n = PAIR ? p.bn / 2 : p.bn;  // B rows / columns this CTA stages
         if (MODE != MODE_DHDW) {
           const int rb = it.u % p.n_rb;
           nkb = (p.d + BK - 1) / BK;
-          a_y = rb * BM;
-          b_y = it.vt * BN_V;
+          a_y = rb * MB + static_cast<int>(rank) * BM;
+          b_y = it.vt * BN_V + static_cast<int>(rank) * (BN_V / (PAIR ? 2 : 1));
         } else if (it.phase == 0) {
           kind = 5;
           nkb = p.c5;
-          a_y = (it.u / p.n_nt) * BM;     // chunk row block
-          b_x = (it.u % p.n_nt) * p.bn;   // d offset
+          a_y = (it.u / p.n_nt) * MB + static_cast<int>(rank) * BM;      // chunk rows
+          b_x = (it.u % p.n_nt) * p.bn + static_cast<int>(rank) * half_n;  // d offset
         } else {
           kind = 6;
           nkb = p.c6;
-          a_x = (it.u / p.n_nt) * BM;     // vocabulary row block
-          b_x = (it.u % p.n_nt) * p.bn;
+          a_x = (it.u / p.n_nt) * MB + static_cast<int>(rank) * BM;      // vocabulary rows
+          b_x = (it.u % p.n_nt) * p.bn + static_cast<int>(rank) * half_n;
         }
+        const uint32_t bytes = (MODE != MODE_DHDW) ? A_BYTES + B_STAGE : A_BYTES + half_n * BK * 2;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, p.status)) { ok = false; break; }
-          const uint32_t fb = bar_full + 8 * stage;
-          const uint32_t sa = sbase + SMEM_A_OFF + stage * A_BYTES;
-          const uint32_t sb = sbase + SMEM_B_OFF + stage * B_BYTES;
+          uint32_t fb = bar_full + 8 * stage;
+          if (PAIR) {
+            // The leader's barrier counts both CTAs' bytes; the peer arrives on it.
+            if (leader) mbar_arrive_expect_tx(fb, 2 * bytes);
+            fb = mapa_shared(fb, 0);
+            if (!leader) mbar_arrive_cluster(fb);
+          } else {
+            mbar_arrive_expect_tx(fb, bytes);
+          }
+          const uint32_t sa = sbase + C::A_OFF + stage * A_BYTES;
+          const uint32_t sb = sbase + C::B_OFF + stage * B_STAGE;
           if (MODE != MODE_DHDW) {
-            mbar_arrive_expect_tx(fb, A_BYTES + B_BYTES);
-            tma_load_2d(sa, &p.tm[0], fb, kb * BK, a_y);
-            tma_load_2d(sb, &p.tm[1], fb, kb * BK, b_y);
+            if (PAIR) {
+              tma_load_2d_pair(sa, &p.tm[0], fb, kb * BK, a_y);
+              tma_load_2d_pair(sb, &p.tm[1], fb, kb * BK, b_y);
+            } else {
+              tma_load_2d(sa, &p.tm[0], fb, kb * BK, a_y);
+              tma_load_2d(sb, &p.tm[1], fb, kb * BK, b_y);
+            }
           } else if (kind == 5) {
-            // dZ is stored as 64-column panels: k-block kb is panel kb.
-            mbar_arrive_expect_tx(fb, A_BYTES + p.bn * BK * 2);
-            tma_load_3d(sa, &p.tm[0], fb, 0, a_y, kb);
-            for (int j = 0; j < p.bn / 64; ++j)
-              tma_load_2d(sb + j * ATOM_BYTES, &p.tm[1], fb, b_x + 64 * j, kb * BK);
+            // dZ is stored as 64-column panels: k-block kb is panel kb.  W is
+            // MN-major here: one 64-column atom per box.
+            if (PAIR) {
+              tma_load_3d_pair(sa, &p.tm[0], fb, 0, a_y, kb);
+              for (int j = 0; j < half_n / 64; ++j)
+                tma_load_2d_pair(sb + j * ATOM_BYTES, &p.tm[1], fb, b_x + 64 * j, kb * BK);
+            } else {
+              tma_load_3d(sa, &p.tm[0], fb, 0, a_y, kb);
+              for (int j = 0; j < half_n / 64; ++j)
+                tma_load_2d(sb + j * ATOM_BYTES, &p.tm[1], fb, b_x + 64 * j, kb * BK);
+            }
           } else {
             // A = dZ^T: one box holding the two 64-column panels of this
             // vocabulary row block (8 KB each, one MN-major atom column each).
             // B = H_c^T (d rows x chunk rows, chunk rows contiguous): K-major.
-            mbar_arrive_expect_tx(fb, A_BYTES + p.bn * BK * 2);
-            tma_load_3d(sa, &p.tm[2], fb, 0, kb * BK, a_x / 64);
-            tma_load_2d(sb, &p.tm[3], fb, kb * BK, b_x);
+            if (PAIR) {
+              tma_load_3d_pair(sa, &p.tm[2], fb, 0, kb * BK, a_x / 64);
+              tma_load_2d_pair(sb, &p.tm[3], fb, kb * BK, b_x);
+            } else {
+              tma_load_3d(sa, &p.tm[2], fb, 0, kb * BK, a_x / 64);
+              tma_load_2d(sb, &p.tm[3], fb, kb * BK, b_x);
+            }
           }
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
-      // Let every load this thread started land before the CTA can exit.
-      for (int s = 0; s < STAGES; ++s) {
-        if (issued > static_cast<uint32_t>(s)) {
-          const uint32_t last = issued - 1 - ((issued - 1 - s) % STAGES);
-          mbar_wait(bar_full + 8 * s, (last / STAGES) & 1u, p.status);
+      // Let every load this thread started land before the CTA can exit.  A
+      // pair's loads all count on the leader's barriers, so the leader waits.
+      if (leader) {
+        for (int s = 0; s < STAGES; ++s) {
+          if (issued > static_cast<uint32_t>(s)) {
+            const uint32_t last = issued - 1 - ((issued - 1 - s) % STAGES);
+            mbar_wait(bar_full + 8 * s, (last / STAGES) & 1u, p.status);
+          }
         }
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // (the leader's; a pair's peer only holds its TMEM)
+    if (lane == 0 && leader) {
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
       JobIter it;
-      it.init(p, MODE);
+      it.init(p, MODE, PAIR ? 2 : 1);
       for (; ok && it.valid(p); it.next(p)) {
         int nkb;
         uint32_t idesc;
         uint32_t a_step, b_step, a_lbo, b_lbo;
         if (MODE != MODE_DHDW) {
           nkb = (p.d + BK - 1) / BK;
-          idesc = idesc_bf16(BM, BN_V, 0, 0);
+          idesc = idesc_bf16(MMA_M, BN_V, 0, 0);
           a_step = 32; b_step = 32; a_lbo = 16; b_lbo = 16;
         } else if (it.phase == 0) {
           nkb = p.c5;
-          idesc = idesc_bf16(BM, p.bn, 0, 1);
+          idesc = idesc_bf16(MMA_M, p.bn, 0, 1);
           a_step = 32; b_step = 2048; a_lbo = 16; b_lbo = ATOM_BYTES;
         } else {
           nkb = p.c6;
-          idesc = idesc_bf16(BM, p.bn, 1, 0);
+          idesc = idesc_bf16(MMA_M, p.bn, 1, 0);
           a_step = 2048; b_step = 32; a_lbo = ATOM_BYTES; b_lbo = 16;
         }
         if (!mbar_wait(bar_tempty + 8 * acc, acc_phase ^ 1u, p.status)) { ok = false; break; }
@@ -494,23 +535,27 @@ tc_kernel(const __grid_constant__ TcParams p) {
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(bar_full + 8 * stage, phase, p.status)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sa = sbase + SMEM_A_OFF + stage * A_BYTES;
-          const uint32_t sb = sbase + SMEM_B_OFF + stage * B_BYTES;
+          const uint32_t sa = sbase + C::A_OFF + stage * A_BYTES;
+          const uint32_t sb = sbase + C::B_OFF + stage * B_STAGE;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t ad = sdesc_sw128(sa + kk * a_step, a_lbo, 1024);
             const uint64_t bd = sdesc_sw128(sb + kk * b_step, b_lbo, 1024);
-            umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            if (PAIR) umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            else umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
-          umma_commit(bar_empty + 8 * stage);
+          if (PAIR) umma_commit_pair(bar_empty + 8 * stage, 3);
+          else umma_commit(bar_empty + 8 * stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        umma_commit(bar_tfull + 8 * acc);
+        if (PAIR) umma_commit_pair(bar_tfull + 8 * acc, 3);
+        else umma_commit(bar_tfull + 8 * acc);
         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
       }
       // Every MMA this thread issued has finished before TMEM is released.
-      umma_commit(bar_drain);
+      if (PAIR) umma_commit_pair(bar_drain, 1);
+      else umma_commit(bar_drain);
       mbar_wait(bar_drain, 0, p.status);
     }
     __syncwarp();
@@ -521,8 +566,10 @@ tc_kernel(const __grid_constant__ TcParams p) {
     const int half = ew >> 2;                // which share of the tile's columns
     constexpr int NSHARE = EPI_WARPS / 4;
     const uint32_t lane_off = static_cast<uint32_t>(lg * 32) << 16;
-    const int row_in_tile = lg * 32 + lane;
-    const uint32_t stage_base = sbase + SMEM_EPI_OFF + ew * 2 * EPI_BUF;
+    const int row_in_tile = static_cast<int>(rank) * BM + lg * 32 + lane;  // within MB
+    const int row0_warp = static_cast<int>(rank) * BM + lg * 32;
+    const uint32_t stage_base = sbase + C::EPI_OFF + ew * 2 * EPI_BUF;
+    const uint32_t tempty_leader = PAIR ? mapa_shared(bar_tempty, 0) : bar_tempty;
     int acc = 0;
     uint32_t acc_phase = 0;
     int nstore = 0;
@@ -544,11 +591,11 @@ tc_kernel(const __grid_constant__ TcParams p) {
     }
 
     JobIter it;
-    it.init(p, MODE);
+    it.init(p, MODE, PAIR ? 2 : 1);
     for (; ok && it.valid(p); it.next(p)) {
       if (MODE != MODE_DHDW && it.first_of_unit(p)) {
         const int rb = it.u % p.n_rb;
-        const int r = rb * BM + row_in_tile;  // row within T (FWD) or the chunk (DZ)
+        const int r = rb * MB + row_in_tile;  // row within T (FWD) or the chunk (DZ)
         row_ok = r < p.rows;
         t = static_cast<int64_t>(p.row0) + r;
         counts = row_ok && (p.mask == nullptr || p.mask[t] != 0);
@@ -604,7 +651,7 @@ tc_kernel(const __grid_constant__ TcParams p) {
         }
       } else if (MODE == MODE_DZ) {
         const int rb = it.u % p.n_rb;
-        const int y0 = rb * BM + lg * 32;  // first chunk row of this warp's 32 rows
+        const int y0 = rb * MB + row0_warp;  // first chunk row of this warp's 32 rows
         const int v_end = (p.V + 63) & ~63;  // dZ panels span round_up(V, 64) columns
         for (int c = 0; c < BN_V / 32; ++c) {
           const int v0 = it.vt * BN_V + c * 32;
@@ -647,10 +694,10 @@ tc_kernel(const __grid_constant__ TcParams p) {
           ++nstore;
         }
       } else {
-        // DHDW: scale and write one accumulator tile.
+        // DHDW: scale and write one accumulator tile (this CTA's rows, all columns).
         const bool is_dh = (it.phase == 0);
         const int nt = it.u % p.n_nt;
-        const int y0 = (it.u / p.n_nt) * BM + lg * 32;
+        const int y0 = (it.u / p.n_nt) * MB + row0_warp;
         const int nch = p.bn / 32 / NSHARE;  // 32-column chunks per warp
         for (int c = half * nch; c < (half + 1) * nch; ++c) {
           const int x0 = nt * p.bn + c * 32;
@@ -691,7 +738,8 @@ tc_kernel(const __grid_constant__ TcParams p) {
         }
       }
       tc_fence_before();
-      mbar_arrive(bar_tempty + 8 * acc);
+      if (PAIR) mbar_arrive_cluster(tempty_leader + 8 * acc);
+      else mbar_arrive(bar_tempty + 8 * acc);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
 
       if (MODE == MODE_FWD && it.last_of_unit() && row_ok) {
@@ -705,8 +753,12 @@ tc_kernel(const __grid_constant__ TcParams p) {
 
   tc_fence_before();
   __syncthreads();
+  if (PAIR) cluster_sync();  // neither CTA frees TMEM or exits while the pair's MMAs run
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+  if (warp == 1) {
+    if (PAIR) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else tmem_dealloc(tmem_base, TMEM_COLS);
+  }
 }
 
 }  // namespace ckl
