@@ -48,6 +48,9 @@ def parse_args(argv=None):
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--memory-sweep", action="store_true",
                     help="measure workspace and peak device memory vs T at the 256K shape")
+    ap.add_argument("--compare", action="store_true",
+                    help="peak memory and time vs T: dense / forward-chunked PyTorch losses "
+                         "against the fused library, at the 32K shape")
     return ap.parse_args(argv)
 
 
@@ -464,12 +467,119 @@ def memory_sweep(args):
                       "shape": {"d": d, "V": V, "K": K, "chunk": chunk}}), flush=True)
 
 
+# ----------------------------------------------------------------- comparators
+# The two non-fused ways of computing the same loss that the source pages
+# measure beside the fused one ("Tối ưu hóa chi phí chưng cất tri thức ...",
+# section "Hai thay đổi hệ thống"; their numbers in "LLMのための効率的な知識蒸留
+# ...", section "ロングコンテキストへのスケーリング").  Plain PyTorch with autograd;
+# used only by --compare and by the test that checks they agree with the
+# library.
+
+def _kl_rows_torch(Hc, W, idx, logp):
+    """Per-row KL of the renormalised teacher top-K against the student's
+    full-vocabulary softmax, for one block of rows (bf16 logits, fp32 math)."""
+    import torch
+    logq = torch.log_softmax((Hc @ W.T).float(), dim=1)
+    logp_n = torch.log_softmax(logp, dim=1)
+    g = logq.gather(1, idx.long())
+    return (logp_n.exp() * (logp_n - g)).sum(1)
+
+
+def dense_kl_torch(H, W, idx, logp, mask):
+    """The textbook dense loss: the whole [T, V] logit grid at once."""
+    m = mask.float()
+    return (_kl_rows_torch(H, W, idx, logp) * m).sum() / m.sum().clamp(min=1.0)
+
+
+def forward_chunked_kl_torch(H, W, idx, logp, mask, chunk):
+    """The loss computed chunk by chunk; autograd still keeps every chunk's
+    logits for the backward."""
+    m = mask.float()
+    total = 0.0
+    for c0 in range(0, H.shape[0], chunk):
+        c1 = min(H.shape[0], c0 + chunk)
+        total = total + (_kl_rows_torch(H[c0:c1], W, idx[c0:c1], logp[c0:c1]) * m[c0:c1]).sum()
+    return total / m.sum().clamp(min=1.0)
+
+
+def compare(args):
+    import torch
+    import chunked_kl_loss_ckl_b200 as ckl
+    d, V, K, chunk = 4096, 128256, 100, 2048
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(args.seed)
+    W0 = (torch.randn(V, d, generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    out = []
+    for T in (8192, 16384, 32768, 65536, 131072, 262144):
+        H0 = torch.randn(T, d, generator=g, device=dev).to(torch.bfloat16)
+        idx = torch.randint(0, V, (T, K), generator=g, device=dev, dtype=torch.int32)
+        logp = torch.log_softmax(2.0 * torch.randn(T, K, generator=g, device=dev), dim=1)
+        mask = torch.ones(T, dtype=torch.uint8, device=dev)
+        row = {"T": T}
+        for name in ("dense", "forward_chunked", "fused_library"):
+            if name != "fused_library" and T > 65536:
+                row[name] = "not run (needs more than the 180 GB of one B200)"
+                continue
+            H = H0.detach().clone().requires_grad_(name != "fused_library")
+            W = W0.detach().clone().requires_grad_(name != "fused_library")
+            torch.cuda.synchronize()
+            torch.cuda.empty_cache()
+            base = torch.cuda.memory_allocated(dev)
+            torch.cuda.reset_peak_memory_stats(dev)
+            try:
+                times = []
+                for rep in range(3):
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    if name == "fused_library":
+                        ws = ckl.new_workspace(T, d, V, K, chunk, dev)
+                        loss, lse = ckl.forward(H, W, idx, logp, mask, chunk, workspace=ws)
+                        dH, dW = ckl.backward(H, W, idx, logp, mask, lse, chunk=chunk,
+                                              workspace=ws)
+                        del ws, lse, dH, dW
+                    else:
+                        H.grad = None
+                        W.grad = None
+                        loss = (dense_kl_torch(H, W, idx, logp, mask) if name == "dense" else
+                                forward_chunked_kl_torch(H, W, idx, logp, mask, chunk))
+                        loss.backward()
+                    e1.record()
+                    torch.cuda.synchronize()
+                    times.append(e0.elapsed_time(e1))
+                peak = torch.cuda.max_memory_allocated(dev) - base
+                # peak above the inputs: everything the method itself holds,
+                # its outputs (lse, dH, dW or the two gradients) included
+                row[name] = {"peak_gib_over_inputs": round(peak / 2 ** 30, 2),
+                             "ms": round(float(np.median(times[1:])), 2),
+                             "loss": float(loss.item())}
+            except torch.OutOfMemoryError:
+                row[name] = "out of memory"
+            # `loss` keeps the autograd graph, and with it H, W and their
+            # gradients, alive: drop it before the next method's baseline
+            loss = None
+            H.grad = None
+            W.grad = None
+            del H, W, loss
+            torch.cuda.synchronize()
+            torch.cuda.empty_cache()
+        print(json.dumps(row), flush=True)
+        out.append(row)
+        del H0, idx, logp, mask
+        torch.cuda.empty_cache()
+    print(json.dumps({"compare": out, "shape": {"d": d, "V": V, "K": K, "chunk": chunk}}),
+          flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.memory_sweep:
         memory_sweep(args)
+        return
+    if args.compare:
+        compare(args)
         return
     if args.impl == "reference":
         bench_reference(args)

@@ -168,3 +168,24 @@ def test_autograd_function(gpu_lib):
     assert np.linalg.norm(gH - ref["dH"]) / np.linalg.norm(ref["dH"]) < 1e-2
     gW = W32.grad.cpu().numpy()
     assert np.linalg.norm(gW - ref["dW"]) / np.linalg.norm(ref["dW"]) < 1e-2
+
+
+def test_comparator_losses_agree_with_the_library(gpu_lib):
+    # The dense and forward-chunked PyTorch losses that bench.py --compare
+    # measures compute the same loss and gradients as the fused library.
+    import bench
+
+    c = make_inputs(400, 256, 3000, 16, seed=16, w_std=0.1, mask=("bernoulli", 0.1))
+    H, W, idx, logp, m = to_device(c)
+    out = run_library(gpu_lib, c, chunk=128)
+    for fn in (lambda h, w: bench.dense_kl_torch(h, w, idx, logp, m),
+               lambda h, w: bench.forward_chunked_kl_torch(h, w, idx, logp, m, 128)):
+        h = H.detach().clone().requires_grad_(True)
+        w = W.detach().clone().requires_grad_(True)
+        loss = fn(h, w)
+        loss.backward()
+        assert abs(loss.item() - out["loss"]) <= 1e-3 * out["loss"]
+        gh = h.grad.float().cpu().numpy()
+        gw = w.grad.float().cpu().numpy()
+        assert np.linalg.norm(gh - out["dH"]) / np.linalg.norm(out["dH"]) < 2e-2
+        assert np.linalg.norm(gw - out["dW"]) / np.linalg.norm(out["dW"]) < 2e-2
