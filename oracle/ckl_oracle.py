@@ -65,6 +65,7 @@ __all__ = [
     "chunked",
     "rows_subset",
     "dw_rows_from_subset",
+    "topk_cache",
 ]
 
 
@@ -266,3 +267,27 @@ def dw_rows_from_subset(H_bits, G: np.ndarray, rows, vrows) -> np.ndarray:
     vrows = np.asarray(vrows, dtype=np.int64)
     Hs = widen_bf16(H_bits[rows])
     return G[:, vrows].T @ Hs
+
+
+def topk_cache(logits_bits: np.ndarray, K: int):
+    """The teacher's offline cache: per row, the K most likely tokens.
+
+    "Дистилляция LLM на одной GPU: offline-кэш и chunked KL loss", section
+    «Два приёма»: the teacher runs once and the 100 most likely tokens per
+    position are kept.  Given the teacher's logits (bf16 bits, [T, V]),
+    returns ids [T, K] ordered by descending logit (equal logits: smaller id
+    first) and their log-probabilities under the full-vocabulary softmax,
+    z_v - log sum_u exp z_u, in fp64.
+    """
+    z = widen_bf16(logits_bits)
+    T, V = z.shape
+    if K < 1 or K > V:
+        raise ValueError("need 1 <= K <= V")
+    ids = np.empty((T, K), dtype=np.int64)
+    cols = np.arange(V)
+    for t in range(T):
+        order = np.lexsort((cols, -z[t]))   # primary: -z, then id
+        ids[t] = order[:K]
+    lse = logsumexp_rows(z)
+    logp = np.take_along_axis(z, ids, axis=1) - lse[:, None]
+    return ids.astype(np.int32), logp

@@ -290,3 +290,31 @@ def test_rows_subset_and_dw_from_subset_match_dense():
     vrows = np.array([0, 3, 69, 40])
     dw = oracle.dw_rows_from_subset(c["H"], sub["G"], rows, vrows)
     np.testing.assert_allclose(dw, out["dW"][vrows], rtol=1e-12, atol=1e-16)
+
+
+# --- the offline top-K cache producer ------------------------------------------
+
+def test_topk_cache_matches_torch_topk_and_log_softmax():
+    # Distinct logits: the selection is torch.topk's, the log-probs are
+    # torch.log_softmax's at those ids.
+    rng = np.random.default_rng(21)
+    T, V, K = 7, 300, 10
+    # distinct bf16 values: every pattern with exponent field 121..130, both signs
+    pos = np.arange(121 * 128, 131 * 128, dtype=np.uint16)
+    pool = np.concatenate([pos, pos | np.uint16(0x8000)])
+    bits = rng.choice(pool, T * V, replace=False).astype(np.uint16).reshape(T, V)
+    zb = oracle.widen_bf16(bits)
+    assert len(np.unique(zb)) == T * V  # exactly representable, no ties
+    ids, logp = oracle.topk_cache(bits, K)
+    zt = torch.tensor(zb)
+    want_ids = torch.topk(zt, K, dim=1).indices.numpy()
+    assert np.array_equal(ids, want_ids)
+    want = torch.log_softmax(zt, dim=1).gather(1, torch.tensor(want_ids)).numpy()
+    np.testing.assert_allclose(logp, want, rtol=0, atol=1e-12)
+
+
+def test_topk_cache_breaks_ties_by_smaller_id():
+    bits = f32_to_bf16_bits(np.array([[1.0, 3.0, 3.0, 2.0, 3.0, 0.5]], np.float32))
+    ids, logp = oracle.topk_cache(bits, 4)
+    assert ids.tolist() == [[1, 2, 4, 3]]
+    assert logp[0, 0] == logp[0, 1] == logp[0, 2]
