@@ -48,6 +48,8 @@ def parse_args(argv=None):
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--memory-sweep", action="store_true",
                     help="measure workspace and peak device memory vs T at the 256K shape")
+    ap.add_argument("--topk", action="store_true",
+                    help="time the teacher top-K cache producer (T=8192, V=128256, K=100)")
     ap.add_argument("--compare", action="store_true",
                     help="peak memory and time vs T: dense / forward-chunked PyTorch losses "
                          "against the fused library, at the 32K shape")
@@ -571,6 +573,35 @@ def compare(args):
           flush=True)
 
 
+def bench_topk(args):
+    """The teacher top-K cache producer: one pass over [T, V] bf16 logits,
+    HBM-bound; achieved GB/s = (T V 2 + T K 8) bytes / kernel time."""
+    import torch
+    import chunked_kl_loss_ckl_b200 as ckl
+    T, V, K = 8192, 128256, 100
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(args.seed)
+    logits = (2.0 * torch.randn(T, V, generator=g, device=dev)).to(torch.bfloat16)
+    for _ in range(args.warmup):
+        ckl.topk_cache(logits, K)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        idx, logp, st = ckl.topk_cache(logits, K)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    peaks, src = load_peaks()
+    nbytes = T * V * 2 + T * K * 8
+    gbs = nbytes / (ms / 1e3) / 1e9
+    print(json.dumps({"kernel": "topk_cache", "T": T, "V": V, "K": K, "ms": round(ms, 4),
+                      "rows_per_s": round(T / (ms / 1e3), 1), "achieved_gbs": round(gbs, 1),
+                      "peak_gbs": peaks.get("hbm_gbs"), "frac": round(gbs / peaks.get("hbm_gbs"), 4),
+                      "peak_source": src, "status": int(st.item())}), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.warmup < 3:
@@ -580,6 +611,9 @@ def main(argv=None):
         return
     if args.compare:
         compare(args)
+        return
+    if args.topk:
+        bench_topk(args)
         return
     if args.impl == "reference":
         bench_reference(args)

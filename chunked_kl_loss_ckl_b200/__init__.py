@@ -22,6 +22,7 @@ import torch
 __all__ = [
     "LIB_PATH", "CklError", "Trace", "KERNEL_NAMES", "lib", "workspace_bytes", "new_workspace",
     "forward", "backward", "read_device_status", "status_string", "chunked_kl_loss",
+    "topk_cache",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libckl.so")
@@ -30,8 +31,10 @@ CKL_OK = 0
 STATUS_NAMES = {
     0: "CKL_OK", 1: "CKL_ERR_INVALID_ARG", 2: "CKL_ERR_UNSUPPORTED", 3: "CKL_ERR_WORKSPACE",
     4: "CKL_ERR_CUDA", 5: "CKL_ERR_BAD_INDEX", 6: "CKL_ERR_BAD_LOGP", 7: "CKL_ERR_TIMEOUT",
+    8: "CKL_ERR_TOPK_TIES",
 }
-KERNEL_NAMES = {1: "prep", 2: "fwd_gemm", 3: "fwd_combine", 4: "bwd_dz", 5: "bwd_dhdw", 6: "other"}
+KERNEL_NAMES = {1: "prep", 2: "fwd_gemm", 3: "fwd_combine", 4: "bwd_dz", 5: "bwd_dhdw", 6: "other",
+                7: "topk"}
 
 
 class CklError(RuntimeError):
@@ -60,6 +63,8 @@ def _load() -> ctypes.CDLL:
     L.ckl_backward.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i64, vp, vp, vp, vp, i32,
                                vp, sz, vp, tr]
     L.ckl_backward.restype = ctypes.c_int
+    L.ckl_topk_cache.argtypes = [vp, i64, i64, i32, vp, vp, vp, vp]
+    L.ckl_topk_cache.restype = ctypes.c_int
     L.ckl_read_device_status.argtypes = [vp, vp, ctypes.POINTER(i32)]
     L.ckl_read_device_status.restype = ctypes.c_int
     L.ckl_status_string.argtypes = [i32]
@@ -190,6 +195,30 @@ def backward(H, W, idx, logp, mask, lse, grad_loss=None, chunk: int = 1024, dW=N
     if rc != CKL_OK:
         raise CklError(rc, "ckl_backward")
     return dH, dW
+
+
+def topk_cache(logits, K: int, stream=None, status=None):
+    """The teacher's offline cache from its logits ([T, V] bf16 on the GPU).
+
+    Returns (ids [T, K] int32, log-probs [T, K] fp32, status [1] int32): per
+    row the K most likely tokens by descending logit (equal logits: smaller
+    id first) and their log-probabilities under the full softmax.  A non-zero
+    status (bit 8) marks a row with more ties at its K-th logit than the
+    kernel's sort holds.
+    """
+    if not logits.is_cuda or logits.dim() != 2 or not logits.is_contiguous():
+        raise ValueError("logits must be a contiguous 2-D CUDA tensor")
+    if logits.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
+        raise TypeError("logits must be bf16 (or its bits as int16/uint16)")
+    T, V = logits.shape
+    idx = torch.empty(T, K, dtype=torch.int32, device=logits.device)
+    logp = torch.empty(T, K, dtype=torch.float32, device=logits.device)
+    st = status if status is not None else torch.zeros(1, dtype=torch.int32, device=logits.device)
+    rc = lib.ckl_topk_cache(_ptr(logits), T, V, K, _ptr(idx), _ptr(logp), _ptr(st),
+                            _stream_handle(stream))
+    if rc != CKL_OK:
+        raise CklError(rc, "ckl_topk_cache")
+    return idx, logp, st
 
 
 def read_device_status(workspace, stream=None):

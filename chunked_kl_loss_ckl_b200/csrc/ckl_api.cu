@@ -10,6 +10,7 @@
 
 #include "../../include/ckl.h"
 #include "ckl_kernels.cuh"
+#include "ckl_topk.cuh"
 
 namespace {
 
@@ -471,6 +472,31 @@ int ckl_backward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
   return CKL_OK;
 }
 
+int ckl_topk_cache(const uint16_t* teacher_logits, int64_t T, int64_t V, int32_t K,
+                   int32_t* topk_idx, float* topk_logp, int32_t* device_status, void* stream) {
+  const int64_t lim = (int64_t(1) << 31) - 1;
+  if (T < 0 || T >= lim || V < 1 || V >= lim || K < 1 || K > V) return CKL_ERR_INVALID_ARG;
+  if (K > ckl::TK_CAP) return CKL_ERR_UNSUPPORTED;
+  if (T > 0 && (!teacher_logits || !topk_idx || !topk_logp)) return CKL_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(teacher_logits) & 1u) || !aligned4(topk_idx) ||
+      !aligned4(topk_logp) || !aligned4(device_status))
+    return CKL_ERR_INVALID_ARG;
+  if (T * V >= (int64_t(1) << 62) / 2) return CKL_ERR_INVALID_ARG;
+  DevInfo di;
+  if (!device_info(di)) return CKL_ERR_CUDA;
+  if (di.major != 10) return CKL_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (device_status && cudaMemsetAsync(device_status, 0, sizeof(int32_t), st) != cudaSuccess)
+    return CKL_ERR_CUDA;
+  if (T == 0) return CKL_OK;
+  const int vec8 = (V % 8 == 0 && aligned16(teacher_logits)) ? 1 : 0;
+  const int grid = static_cast<int>(std::min<int64_t>(T, static_cast<int64_t>(di.sms) * 2));
+  ckl::topk_cache_kernel<<<grid, ckl::TK_THREADS, 0, st>>>(teacher_logits, T, static_cast<int>(V),
+                                                           K, vec8, topk_idx, topk_logp,
+                                                           device_status);
+  return cudaGetLastError() == cudaSuccess ? CKL_OK : CKL_ERR_CUDA;
+}
+
 int ckl_read_device_status(const void* workspace, void* stream, int32_t* device_status) {
   if (!workspace || !device_status) return CKL_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -492,6 +518,7 @@ const char* ckl_status_string(int32_t status) {
     case CKL_ERR_BAD_INDEX: return "teacher token id outside [0, V)";
     case CKL_ERR_BAD_LOGP: return "teacher log-prob NaN/+inf, or a row with none finite";
     case CKL_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out of time";
+    case CKL_ERR_TOPK_TIES: return "too many teacher logits tie at a row's K-th value";
     default: return "unknown status";
   }
 }

@@ -1,0 +1,246 @@
+// The offline teacher cache: per row of teacher logits, the K most likely
+// tokens and their log-probabilities.
+//
+// "Дистилляция LLM на одной GPU: offline-кэш и chunked KL loss", section
+// «Два приёма»: the teacher runs once, the 100 most likely tokens of every
+// position are kept, and training reads that cache.  This is the step that
+// writes it, given the teacher's logits.
+//
+// One CTA per row (persistent over rows), three passes over the row (the
+// first from HBM, the others mostly from L2):
+//   1. the largest key (packed 16-bit maxima, two keys per instruction);
+//   2. the row's sum of exp(z - max) (log-sum-exp = max + log of it), and a
+//      histogram of the 256 keys just below the largest (one bucket per bf16
+//      value, two binades) whose block scan finds the K-th largest key; only
+//      if fewer than K elements fall there does the window slide down, 4096
+//      keys at a time, in further passes;
+//   3. every element at or above that key is gathered, and a bitonic sort of
+//      (key, -id) in shared memory puts them in order: descending logit,
+//      equal logits by smaller id.
+// Keys are the bf16 bit patterns mapped to an order-preserving 16-bit code
+// (-0 counts as +0), so every comparison is exact.
+#pragma once
+
+#include <cstdint>
+
+#include "ckl_ptx.cuh"
+
+#define CKL_DEV_TOPK_TIES 8  // more elements tie at the K-th logit than the sort holds
+
+namespace ckl {
+
+constexpr int TK_THREADS = 512;
+constexpr int TK_WIN = 4096;  // keys per histogram window
+constexpr int TK_WIN0 = 256;  // keys in the first window (two binades of bf16)
+constexpr int TK_CAP = 2048;  // elements the final sort holds (K plus the ties at the K-th)
+
+__device__ __forceinline__ uint32_t bf16_key(uint32_t b) {
+  if (b == 0x8000u) b = 0u;  // -0 == +0
+  return (b & 0x8000u) ? (~b & 0xFFFFu) : (b | 0x8000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+  const uint32_t b = (k & 0x8000u) ? (k & 0x7FFFu) : (~k & 0xFFFFu);
+  return __uint_as_float(b << 16);
+}
+
+// Order-preserving keys of two packed bf16 values (each half as bf16_key).
+__device__ __forceinline__ uint32_t bf16_key2(uint32_t w) {
+  w &= ~__vcmpeq2(w, 0x80008000u);                 // -0 -> +0
+  const uint32_t neg = ((w & 0x80008000u) >> 15) * 0x7FFFu;
+  return w ^ (0x80008000u | neg);
+}
+
+constexpr int TK_UNROLL = 2;  // independent 16-byte loads in flight per thread
+
+// Largest key of the row.
+__device__ __forceinline__ uint32_t tk_row_max(const uint16_t* z, int V, bool vec8) {
+  uint32_t m2 = 0;
+  if (vec8) {
+    const uint4* z4 = reinterpret_cast<const uint4*>(z);
+    const int n8 = V / 8;
+    for (int base = threadIdx.x; base < n8; base += TK_THREADS * TK_UNROLL) {
+      uint4 v[TK_UNROLL];
+#pragma unroll
+      for (int u = 0; u < TK_UNROLL; ++u) {
+        const int i = base + u * TK_THREADS;
+        v[u] = (i < n8) ? z4[i] : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < TK_UNROLL; ++u)
+        m2 = __vmaxu2(m2, __vmaxu2(__vmaxu2(bf16_key2(v[u].x), bf16_key2(v[u].y)),
+                                   __vmaxu2(bf16_key2(v[u].z), bf16_key2(v[u].w))));
+    }
+  } else {
+    for (int i = threadIdx.x; i < V; i += TK_THREADS) m2 = __vmaxu2(m2, bf16_key(z[i]));
+  }
+  return max(m2 & 0xFFFFu, m2 >> 16);
+}
+
+// Calls f(key, id) for every element of the row, eight bf16 per 16-byte load
+// when the row allows it.
+template <typename F>
+__device__ __forceinline__ void tk_for_row(const uint16_t* z, int V, bool vec8, F&& f) {
+  if (vec8) {
+    const uint4* z4 = reinterpret_cast<const uint4*>(z);
+    const int n8 = V / 8;
+    for (int base = threadIdx.x; base < n8; base += TK_THREADS * TK_UNROLL) {
+      uint4 v[TK_UNROLL];
+#pragma unroll
+      for (int u = 0; u < TK_UNROLL; ++u) {
+        const int i = base + u * TK_THREADS;
+        if (i < n8) v[u] = z4[i];
+      }
+#pragma unroll
+      for (int u = 0; u < TK_UNROLL; ++u) {
+        const int i = base + u * TK_THREADS;
+        if (i < n8) {
+          const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            f(bf16_key(w[j] & 0xFFFFu), 8 * i + 2 * j);
+            f(bf16_key(w[j] >> 16), 8 * i + 2 * j + 1);
+          }
+        }
+      }
+    }
+  } else {
+    for (int i = threadIdx.x; i < V; i += TK_THREADS) f(bf16_key(z[i]), i);
+  }
+}
+
+__global__ void __launch_bounds__(TK_THREADS, 2)
+topk_cache_kernel(const uint16_t* __restrict__ logits, int64_t T, int V, int K, int vec8,
+                  int32_t* __restrict__ idx_out, float* __restrict__ logp_out, int* status) {
+  __shared__ uint32_t hist[TK_WIN];
+  __shared__ unsigned long long cand[TK_CAP];
+  __shared__ float s_s[TK_THREADS / 32];
+  __shared__ uint32_t s_k[TK_THREADS / 32];
+  __shared__ uint32_t s_part[TK_THREADS / 32];
+  __shared__ uint32_t s_thr, s_ncand, s_found, s_total;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  for (int64_t row = blockIdx.x; row < T; row += gridDim.x) {
+    const uint16_t* z = logits + row * static_cast<int64_t>(V);
+
+    // ---- pass 1: the largest key
+    uint32_t kmax = tk_row_max(z, V, vec8 != 0);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    if (lane == 0) s_k[warp] = kmax;
+    for (int j = tid; j < TK_WIN; j += TK_THREADS) hist[j] = 0;
+    if (tid == 0) { s_found = 0; s_thr = 0; }
+    __syncthreads();
+    kmax = 0;
+    for (int w = 0; w < TK_THREADS / 32; ++w) kmax = max(kmax, s_k[w]);
+    const float zmax = key_value(kmax);  // the row's largest logit
+
+    // ---- pass 2: sum of exp against the maximum, and the first window's
+    // histogram; further windows (4096 keys each) only when needed
+    uint32_t above = 0;         // elements with a key above the window
+    int top = static_cast<int>(kmax);
+    float lse = 0.f;
+    for (int win = 0;; ++win) {
+      const int lo = top - (win == 0 ? TK_WIN0 : TK_WIN) + 1;
+      if (win == 0) {
+        float s = 0.f;
+        tk_for_row(z, V, vec8 != 0, [&](uint32_t k, int) {
+          s += ex2_approx((key_value(k) - zmax) * LOG2E);
+          const int kk = static_cast<int>(k);
+          if (kk >= lo) atomicAdd(&hist[top - kk], 1u);
+        });
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0) s_s[warp] = s;
+      } else {
+        for (int j = tid; j < TK_WIN; j += TK_THREADS) hist[j] = 0;
+        __syncthreads();
+        tk_for_row(z, V, vec8 != 0, [&](uint32_t k, int) {
+          const int kk = static_cast<int>(k);
+          if (kk <= top && kk >= lo) atomicAdd(&hist[top - kk], 1u);
+        });
+      }
+      __syncthreads();
+      if (win == 0) {
+        float S = 0.f;
+        for (int w = 0; w < TK_THREADS / 32; ++w) S += s_s[w];
+        lse = zmax + logf(S);
+      }
+      // block scan over the window: thread tid owns buckets [8 tid, 8 tid + 8)
+      uint32_t own = 0;
+#pragma unroll
+      for (int j = 0; j < TK_WIN / TK_THREADS; ++j) own += hist[tid * (TK_WIN / TK_THREADS) + j];
+      uint32_t incl = own;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (lane == 31) s_part[warp] = incl;
+      __syncthreads();
+      uint32_t before = 0;
+      for (int w = 0; w < warp; ++w) before += s_part[w];
+      before += incl - own;  // elements in buckets before this thread's (higher keys)
+      if (tid == TK_THREADS - 1) s_total = before + own;
+      if (above + before < static_cast<uint32_t>(K) &&
+          above + before + own >= static_cast<uint32_t>(K)) {
+        uint32_t c = above + before;
+        for (int j = 0; j < TK_WIN / TK_THREADS; ++j) {
+          c += hist[tid * (TK_WIN / TK_THREADS) + j];
+          if (c >= static_cast<uint32_t>(K)) {
+            s_thr = static_cast<uint32_t>(top - (tid * (TK_WIN / TK_THREADS) + j));
+            s_found = 1;
+            break;
+          }
+        }
+      }
+      __syncthreads();
+      if (s_found || lo <= 0) break;
+      above += s_total;
+      top = lo - 1;
+      __syncthreads();
+    }
+    const uint32_t thr = s_thr;
+
+    // ---- pass 3: gather every element at or above the threshold key
+    if (tid == 0) s_ncand = 0;
+    __syncthreads();
+    tk_for_row(z, V, vec8 != 0, [&](uint32_t k, int i) {
+      if (k >= thr) {
+        const uint32_t slot = atomicAdd(&s_ncand, 1u);
+        if (slot < TK_CAP)
+          cand[slot] = (static_cast<unsigned long long>(k) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(i));
+      }
+    });
+    __syncthreads();
+    const uint32_t n = min(s_ncand, static_cast<uint32_t>(TK_CAP));
+    if (tid == 0 && s_ncand > static_cast<uint32_t>(TK_CAP) && status != nullptr)
+      atomicOr(status, CKL_DEV_TOPK_TIES);
+    uint32_t P = 1;
+    while (P < n) P <<= 1;
+    for (uint32_t i = n + tid; i < P; i += TK_THREADS) cand[i] = 0ull;
+    __syncthreads();
+    // bitonic sort, descending
+    for (uint32_t k = 2; k <= P; k <<= 1) {
+      for (uint32_t j = k >> 1; j > 0; j >>= 1) {
+        for (uint32_t i = tid; i < P; i += TK_THREADS) {
+          const uint32_t ixj = i ^ j;
+          if (ixj > i) {
+            const unsigned long long a = cand[i], b = cand[ixj];
+            const bool up = (i & k) == 0;
+            if (up ? (a < b) : (a > b)) { cand[i] = b; cand[ixj] = a; }
+          }
+        }
+        __syncthreads();
+      }
+    }
+    for (int k = tid; k < K; k += TK_THREADS) {
+      const unsigned long long e = cand[k];
+      const uint32_t key = static_cast<uint32_t>(e >> 32);
+      idx_out[row * K + k] = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(e));
+      logp_out[row * K + k] = key_value(key) - lse;
+    }
+    __syncthreads();
+  }
+}
+
+}  // namespace ckl

@@ -68,7 +68,8 @@ typedef enum ckl_status {
   CKL_ERR_CUDA = 4,        /* a CUDA runtime/driver call or launch failed */
   CKL_ERR_BAD_INDEX = 5,   /* device: a teacher id outside [0, V) */
   CKL_ERR_BAD_LOGP = 6,    /* device: NaN/+inf log-prob, or a row with none finite */
-  CKL_ERR_TIMEOUT = 7      /* device: a bounded wait inside a kernel ran out */
+  CKL_ERR_TIMEOUT = 7,     /* device: a bounded wait inside a kernel ran out */
+  CKL_ERR_TOPK_TIES = 8    /* device: too many logits tie at a row's K-th value */
 } ckl_status;
 
 /* Kernel ids written by the optional launch trace. */
@@ -78,7 +79,8 @@ enum {
   CKL_KERNEL_FWD_COMBINE = 3, /* merge vocabulary splits: lse, KL, masked mean */
   CKL_KERNEL_BWD_DZ = 4,      /* logit recompute + dZ = softmax - scatter(p) */
   CKL_KERNEL_BWD_DHDW = 5,    /* dH = s dZ W and dW += s dZ^T H for one chunk */
-  CKL_KERNEL_OTHER = 6
+  CKL_KERNEL_OTHER = 6,
+  CKL_KERNEL_TOPK = 7         /* teacher top-K cache producer */
 };
 
 /*
@@ -156,6 +158,28 @@ CKL_API int ckl_backward(const uint16_t* H, const uint16_t* W, const int32_t* to
  * and returns the matching ckl_status (CKL_OK when the word is 0).
  */
 CKL_API int ckl_read_device_status(const void* workspace, void* stream, int32_t* device_status);
+
+/*
+ * The offline teacher cache ("Дистилляция LLM на одной GPU: offline-кэш и
+ * chunked KL loss", section «Два приёма»: the teacher runs once and its 100
+ * most likely tokens per position are kept).  From the teacher's logits,
+ * writes per row the K most likely token ids, ordered by descending logit
+ * (equal logits: smaller id first), and their log-probabilities under the
+ * full-vocabulary softmax, z_v - log sum_u exp z_u.
+ *   teacher_logits [T, V] bf16  device, row-major, finite values
+ *   topk_idx       [T, K] int32 out
+ *   topk_logp      [T, K] fp32  out
+ *   device_status  [1]    int32 device memory or NULL: zeroed, then
+ *                               bit 8 is set when a row has more than
+ *                               2048 elements at or above its K-th largest
+ *                               logit (ties at that value; the row's output
+ *                               is then unspecified)
+ * Requires 1 <= K <= min(V, 2048).  Needs no workspace.  Enqueued on
+ * `stream`.  ckl_status_string(CKL_ERR_TOPK_TIES) names the device error.
+ */
+CKL_API int ckl_topk_cache(const uint16_t* teacher_logits, int64_t T, int64_t V, int32_t K,
+                           int32_t* topk_idx, float* topk_logp, int32_t* device_status,
+                           void* stream);
 
 /* Static, human-readable text for a status code. */
 CKL_API const char* ckl_status_string(int32_t status);

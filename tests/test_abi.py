@@ -23,8 +23,8 @@ def ckl():
 
 def test_header_declares_the_entry_points():
     assert _declared() == ["ckl_backward", "ckl_forward", "ckl_forward_static_scratch",
-                           "ckl_read_device_status", "ckl_status_string", "ckl_version",
-                           "ckl_workspace_bytes"]
+                           "ckl_read_device_status", "ckl_status_string", "ckl_topk_cache",
+                           "ckl_version", "ckl_workspace_bytes"]
 
 
 def test_library_exports_every_declared_symbol(ckl):
@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol(ckl):
 
 
 def test_status_strings_and_version(ckl):
-    for code in range(8):
+    for code in range(9):
         assert ckl.status_string(code) and ckl.status_string(code) != "unknown status"
     assert ckl.status_string(99) == "unknown status"
     assert ckl.lib.ckl_version() >= 100
@@ -85,3 +85,7 @@ def test_host_checks_return_before_any_device_work(ckl):
     assert L.ckl_backward(fake, fake, fake, fake, nul, 4, 64, 100, 4, 8, fake, nul, fake, nul, 0,
                           fake, 1 << 20, nul, nul) == 1
     assert L.ckl_read_device_status(nul, nul, nul) == 1
+    # top-K cache: K must be in [1, min(V, 2048)]
+    assert L.ckl_topk_cache(fake, 4, 100, 0, fake, fake, nul, nul) == 1
+    assert L.ckl_topk_cache(fake, 4, 100, 101, fake, fake, nul, nul) == 1
+    assert L.ckl_topk_cache(fake, 4, 5000, 3000, fake, fake, nul, nul) == 2

@@ -1,0 +1,94 @@
+"""GPU parity of the teacher top-K cache producer against the oracle.
+
+The ids must match exactly (the selection compares bf16 values, exact in any
+precision; equal logits go to the smaller id); the log-probabilities within
+1e-4 absolute (fp32 log-sum-exp over the row).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from ckl_synth import f32_to_bf16_bits
+
+pytestmark = pytest.mark.gpu
+
+LOGP_ATOL = 1e-4
+LOGP_RTOL = 1e-6   # log-probs of logits far from 1 carry fp32 relative error
+
+
+def _run(ckl, bits, K):
+    x = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda()
+    idx, logp, st = ckl.topk_cache(x, K)
+    torch.cuda.synchronize()
+    return idx.cpu().numpy(), logp.cpu().numpy().astype(np.float64), int(st.item())
+
+
+def _check(ckl, bits, K, rows=None):
+    idx, logp, st = _run(ckl, bits, K)
+    assert st == 0
+    sel = slice(None) if rows is None else rows
+    ref_idx, ref_logp = oracle.topk_cache(bits[sel], K)
+    assert np.array_equal(idx[sel], ref_idx)
+    assert (np.abs(logp[sel] - ref_logp) <= LOGP_ATOL + LOGP_RTOL * np.abs(ref_logp)).all()
+    return idx, logp
+
+
+def test_teacher_sized_rows(gpu_lib):
+    rng = np.random.default_rng(1)
+    bits = f32_to_bf16_bits(rng.normal(0, 2, (48, 128256)).astype(np.float32))
+    _check(gpu_lib, bits, 100)
+
+
+def test_unaligned_rows_and_heavy_ties(gpu_lib):
+    # V not a multiple of 8 (scalar loads); logits on a 0.25 grid tie often
+    rng = np.random.default_rng(2)
+    z = np.round(rng.normal(0, 2, (33, 1001)) * 4) / 4
+    _check(gpu_lib, f32_to_bf16_bits(z.astype(np.float32)), 16)
+
+
+@pytest.mark.parametrize("K", [1, 300])
+def test_k_one_and_k_equals_v(gpu_lib, K):
+    rng = np.random.default_rng(3)
+    _check(gpu_lib, f32_to_bf16_bits(rng.normal(0, 1, (17, 300)).astype(np.float32)), K)
+
+
+def test_signed_zeros_and_wide_value_range(gpu_lib):
+    # -0 and +0 are equal logits (ties by id); values spread over many binades
+    # so the histogram window has to slide below the largest key
+    rng = np.random.default_rng(4)
+    z = rng.normal(0, 1, (9, 5000)).astype(np.float32)
+    z[0, :50] = -0.0
+    z[0, 50:100] = 0.0
+    z[0, 100:] = -rng.uniform(1, 2, 4900)
+    z[1] = np.exp(rng.uniform(-80, 80, 5000)).astype(np.float32) * rng.choice([-1, 1], 5000)
+    _check(gpu_lib, f32_to_bf16_bits(z), 80)
+
+
+def test_too_many_ties_is_reported_and_other_rows_are_right(gpu_lib):
+    rng = np.random.default_rng(5)
+    z = rng.normal(0, 1, (4, 10000)).astype(np.float32)
+    z[2] = 1.5                                    # 10 000 equal logits
+    bits = f32_to_bf16_bits(z)
+    idx, logp, st = _run(gpu_lib, bits, 10)
+    assert st & 8
+    rows = np.array([0, 1, 3])
+    ref_idx, ref_logp = oracle.topk_cache(bits[rows], 10)
+    assert np.array_equal(idx[rows], ref_idx)
+    assert np.abs(logp[rows] - ref_logp).max() <= LOGP_ATOL
+
+
+def test_cache_feeds_the_loss(gpu_lib):
+    # The producer's output is a valid teacher cache for the fused loss.
+    from ckl_synth import make_inputs
+    from gpu_util import assert_parity, run_library
+
+    rng = np.random.default_rng(6)
+    c = make_inputs(200, 64, 2000, 20, seed=17, w_std=0.3)
+    teacher = f32_to_bf16_bits(rng.normal(0, 2, (200, 2000)).astype(np.float32))
+    idx, logp, st = _run(gpu_lib, teacher, 20)
+    assert st == 0
+    c = dict(c, idx=idx.astype(np.int32), logp=logp.astype(np.float32))
+    ref = oracle.dense(c["H"], c["W"], c["idx"], c["logp"], None)
+    assert_parity(run_library(gpu_lib, c, chunk=64), ref, "top-K cache -> loss")
