@@ -420,7 +420,7 @@ int ckl_backward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
           !map2d(&p.tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, V, d * 2, ckl::BK,
                  ckl::BN_V / kSlotCTAs, CU_TENSOR_MAP_SWIZZLE_128B) ||
           !map3d(&p.tm[2], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dz, 64, rows, L.npanels, 128,
-                 L.cap * 128, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+                 L.cap * 128, 32, ckl::BM, CU_TENSOR_MAP_SWIZZLE_64B))
         return CKL_ERR_CUDA;
       TraceScope ts(trace, st, CKL_KERNEL_BWD_DZ);
       if (launch_tc<ckl::MODE_DZ>(p, p.n_units, di, st) != CKL_OK) return CKL_ERR_CUDA;
@@ -460,9 +460,9 @@ int ckl_backward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
           !map3d2(&p.tm[2], dz, 64, rows, L.npanels, 128, L.cap * 128, 64, ckl::BK, 2) ||
           !map2d(&p.tm[3], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hct, rows, d, L.pitch_t * 2, ckl::BK,
                  bn / kSlotCTAs, CU_TENSOR_MAP_SWIZZLE_128B) ||
-          !map2d(&p.tm[4], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dHc, d, rows, d * 2, 32, 32,
+          !map2d(&p.tm[4], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dHc, d, rows, d * 2, 32, ckl::BM,
                  CU_TENSOR_MAP_SWIZZLE_64B) ||
-          !map2d(&p.tm[5], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, dW, d, V, d * 4, 32, 32,
+          !map2d(&p.tm[5], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, dW, d, V, d * 4, 32, ckl::BM,
                  CU_TENSOR_MAP_SWIZZLE_128B))
         return CKL_ERR_CUDA;
       TraceScope ts(trace, st, CKL_KERNEL_BWD_DHDW);

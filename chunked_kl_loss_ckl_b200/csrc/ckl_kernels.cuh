@@ -40,7 +40,7 @@ constexpr int BN_V = 256;         // vocabulary columns per logit tile
 constexpr int A_BYTES = BM * BK * 2;        // 16 KB
 constexpr int B_BYTES = 256 * BK * 2;       // 32 KB (largest B tile)
 constexpr int ATOM_BYTES = 64 * BK * 2;     // one 64-wide MN-major atom column, 8 KB
-constexpr int EPI_BUF = 4096;               // bytes per staging buffer (2 per epilogue warp)
+constexpr int EPI_STAGE = BM * 128;         // one 128-row x 128-byte staging tile, 16 KB
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COLS = 256;          // TMEM columns per accumulator buffer
 
@@ -49,10 +49,10 @@ enum Mode { MODE_FWD = 0, MODE_DZ = 1, MODE_DHDW = 2 };
 // Pipeline depth and epilogue width.  A single CTA holds a 128 x 256 tile:
 // four 48 KB operand stages fill the shared memory beside the epilogue
 // staging.  A CTA pair (PAIR) shares one 256-row MMA: each CTA stages its own
-// 128 rows of A and half of B, 32 KB per stage, so six stages fit.  The
-// epilogue code also runs with eight warps (two per TMEM lane group, each
-// taking half of a tile's columns); that measured slower here because it
-// costs an operand stage: the epilogue is not the bottleneck.
+// 128 rows of A and half of B, 32 KB per stage, so six stages fit.  Four
+// epilogue warps, one per TMEM lane group (eight, splitting the columns,
+// measured slower: the extra staging costs an operand stage, and the
+// epilogue is not the bottleneck).
 template <int MODE, bool PAIR>
 struct Cfg {
   static constexpr int STAGES = PAIR ? 6 : 4;
@@ -63,9 +63,10 @@ struct Cfg {
   static constexpr int A_OFF = 0;
   static constexpr int B_OFF = STAGES * A_BYTES;
   static constexpr int EPI_OFF = B_OFF + STAGES * B_STAGE;
-  static constexpr int BAR_OFF = EPI_OFF + EPI_WARPS * 2 * EPI_BUF;
+  static constexpr int BAR_OFF = EPI_OFF + 2 * EPI_STAGE;  // two staging tiles
   static constexpr int SMEM_ALLOC = BAR_OFF + 256 + 1024;  // + slack to align the base to 1 KB
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+  static_assert(8 * (2 * STAGES + 9) + 4 <= 256, "barrier area");
 };
 
 constexpr float LOG2E = 1.4426950408889634f;
@@ -378,7 +379,9 @@ tc_kernel(const __grid_constant__ TcParams p) {
   const uint32_t bar_tfull = bar_empty + 8 * STAGES;          // [2]
   const uint32_t bar_tempty = bar_tfull + 16;                 // [2] (leader's count both)
   const uint32_t bar_drain = bar_tempty + 16;                 // [1]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::BAR_OFF + 8 * (2 * STAGES + 5));
+  const uint32_t bar_staged = bar_drain + 8;                  // [2] staging tile written
+  const uint32_t bar_sfree = bar_staged + 16;                 // [2] staging tile read out
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::BAR_OFF + 8 * (2 * STAGES + 9));
 
   if (warp == 0 && lane == 0) {
     const int n_maps = (MODE == MODE_FWD) ? 2 : (MODE == MODE_DZ) ? 3 : 6;
@@ -393,6 +396,10 @@ tc_kernel(const __grid_constant__ TcParams p) {
       mbar_init(bar_tempty + 8 * a, (PAIR ? 2 : 1) * 32 * EPI_WARPS);
     }
     mbar_init(bar_drain, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_staged + 8 * b, EPI_WARPS);
+      mbar_init(bar_sfree + 8 * b, 1);
+    }
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -563,17 +570,58 @@ tc_kernel(const __grid_constant__ TcParams p) {
     // ------------------------------------------------------------ epilogue
     const int ew = warp - 2;                 // 0 .. EPI_WARPS-1
     const int lg = warp & 3;                 // TMEM lane group this warp may access
-    const int half = ew >> 2;                // which share of the tile's columns
-    constexpr int NSHARE = EPI_WARPS / 4;
+    static_assert(EPI_WARPS == 4, "one warp per TMEM lane group");
     const uint32_t lane_off = static_cast<uint32_t>(lg * 32) << 16;
     const int row_in_tile = static_cast<int>(rank) * BM + lg * 32 + lane;  // within MB
-    const int row0_warp = static_cast<int>(rank) * BM + lg * 32;
-    const uint32_t stage_base = sbase + C::EPI_OFF + ew * 2 * EPI_BUF;
+    const int row0_cta = static_cast<int>(rank) * BM;  // this CTA's rows within MB
+    // Stores go through two alternating 128-row staging tiles: every warp
+    // writes its 32 rows, and one thread stores the whole tile with a single
+    // TMA call once all four warps have arrived (4x fewer TMA operations than
+    // a store per warp; the TMA unit is shared with the operand loads).
+    const uint32_t stage_base = sbase + C::EPI_OFF;
+    const uint32_t srow = static_cast<uint32_t>(lg * 32 + lane);  // staging row of this thread
+    const bool issuer = (ew == 0 && lane == 0);
     const uint32_t tempty_leader = PAIR ? mapa_shared(bar_tempty, 0) : bar_tempty;
     int acc = 0;
     uint32_t acc_phase = 0;
     int nstore = 0;
     bool ok = true;
+    // Wait until staging tile nstore & 1 has been read out by its previous store.
+    auto stage_begin = [&]() -> bool {
+      bool good = true;
+      if (lane == 0 && nstore >= 2)
+        good = mbar_wait(bar_sfree + 8 * (nstore & 1), static_cast<uint32_t>((nstore >> 1) - 1) & 1u,
+                         p.status);
+      __syncwarp();
+      return __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
+    };
+    // Publish this warp's rows; the issuer stores the tile once all warps have
+    // (kind 0: dZ panel, 1: dH, 2: dW store, 3: dW add) and then frees the
+    // tile of the store before.
+    auto stage_end = [&](int kind, int x, int y, int z) -> bool {
+      fence_proxy_async_smem();
+      __syncwarp();
+      const uint32_t sb = static_cast<uint32_t>(nstore & 1);
+      if (lane == 0) mbar_arrive(bar_staged + 8 * sb);
+      bool good = true;
+      if (issuer) {
+        good = mbar_wait(bar_staged + 8 * sb, static_cast<uint32_t>(nstore >> 1) & 1u, p.status);
+        if (good) {
+          const uint32_t buf = stage_base + sb * EPI_STAGE;
+          if (kind == 0) tma_store_3d(&p.tm[2], buf, x, y, z);
+          else if (kind == 1) tma_store_2d(&p.tm[4], buf, x, y);
+          else if (kind == 2) tma_store_2d(&p.tm[5], buf, x, y);
+          else tma_reduce_add_2d(&p.tm[5], buf, x, y);
+          bulk_commit();
+          if (nstore >= 1) {
+            bulk_wait_read<1>();
+            mbar_arrive(bar_sfree + 8 * (sb ^ 1u));
+          }
+        }
+      }
+      ++nstore;
+      return __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
+    };
 
     // per-row state (FWD / DZ)
     int64_t t = 0;
@@ -651,7 +699,7 @@ tc_kernel(const __grid_constant__ TcParams p) {
         }
       } else if (MODE == MODE_DZ) {
         const int rb = it.u % p.n_rb;
-        const int y0 = rb * MB + row0_warp;  // first chunk row of this warp's 32 rows
+        const int y0 = rb * MB + row0_cta;  // first chunk row of this CTA's 128
         const int v_end = (p.V + 63) & ~63;  // dZ panels span round_up(V, 64) columns
         for (int c = 0; c < BN_V / 32; ++c) {
           const int v0 = it.vt * BN_V + c * 32;
@@ -674,10 +722,9 @@ tc_kernel(const __grid_constant__ TcParams p) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) if (v0 + j >= p.V) x[j] = 0.f;
           }
-          const uint32_t buf = stage_base + (nstore & 1) * EPI_BUF;
-          if (lane == 0) bulk_wait_read<1>();
-          __syncwarp();
-          const uint32_t rowa = buf + lane * 64;
+          if (!stage_begin()) { ok = false; break; }
+          // 64-byte rows, 64-byte swizzle: 16-byte unit j of row r at unit j ^ ((r >> 1) & 3)
+          const uint32_t rowa = stage_base + (nstore & 1) * EPI_STAGE + srow * 64;
           const int sw = (lane >> 1) & 3;
 #pragma unroll
           for (int j = 0; j < 4; ++j)
@@ -685,30 +732,22 @@ tc_kernel(const __grid_constant__ TcParams p) {
                          pack_bf16x2(x[8 * j + 2], x[8 * j + 3]),
                          pack_bf16x2(x[8 * j + 4], x[8 * j + 5]),
                          pack_bf16x2(x[8 * j + 6], x[8 * j + 7]));
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_3d(&p.tm[2], buf, v0 & 63, y0, v0 >> 6);
-            bulk_commit();
-          }
-          ++nstore;
+          if (!stage_end(0, v0 & 63, y0, v0 >> 6)) { ok = false; break; }
         }
       } else {
         // DHDW: scale and write one accumulator tile (this CTA's rows, all columns).
         const bool is_dh = (it.phase == 0);
         const int nt = it.u % p.n_nt;
-        const int y0 = (it.u / p.n_nt) * MB + row0_warp;
-        const int nch = p.bn / 32 / NSHARE;  // 32-column chunks per warp
-        for (int c = half * nch; c < (half + 1) * nch; ++c) {
+        const int y0 = (it.u / p.n_nt) * MB + row0_cta;
+        for (int c = 0; c < p.bn / 32; ++c) {
           const int x0 = nt * p.bn + c * 32;
           if (x0 >= p.d) break;
           float x[32];
           tmem_ld32(tacc + c * 32, x);
-          const uint32_t buf = stage_base + (nstore & 1) * EPI_BUF;
-          if (lane == 0) bulk_wait_read<1>();
-          __syncwarp();
+          if (!stage_begin()) { ok = false; break; }
+          const uint32_t buf = stage_base + (nstore & 1) * EPI_STAGE;
           if (is_dh) {
-            const uint32_t rowa = buf + lane * 64;
+            const uint32_t rowa = buf + srow * 64;
             const int sw = (lane >> 1) & 3;
 #pragma unroll
             for (int j = 0; j < 4; ++j)
@@ -717,7 +756,8 @@ tc_kernel(const __grid_constant__ TcParams p) {
                            pack_bf16x2(x[8 * j + 4] * scale, x[8 * j + 5] * scale),
                            pack_bf16x2(x[8 * j + 6] * scale, x[8 * j + 7] * scale));
           } else {
-            const uint32_t rowa = buf + lane * 128;
+            // 128-byte rows, 128-byte swizzle: unit j of row r at unit j ^ (r & 7)
+            const uint32_t rowa = buf + srow * 128;
             const int sw = lane & 7;
 #pragma unroll
             for (int j = 0; j < 8; ++j)
@@ -726,15 +766,7 @@ tc_kernel(const __grid_constant__ TcParams p) {
                            __float_as_uint(x[4 * j + 2] * scale),
                            __float_as_uint(x[4 * j + 3] * scale));
           }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            if (is_dh) tma_store_2d(&p.tm[4], buf, x0, y0);
-            else if (p.dw_store) tma_store_2d(&p.tm[5], buf, x0, y0);
-            else tma_reduce_add_2d(&p.tm[5], buf, x0, y0);
-            bulk_commit();
-          }
-          ++nstore;
+          if (!stage_end(is_dh ? 1 : (p.dw_store ? 2 : 3), x0, y0, 0)) { ok = false; break; }
         }
       }
       tc_fence_before();
