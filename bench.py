@@ -44,6 +44,8 @@ def parse_args(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-single-pass", action="store_true",
+                    help="skip timing the single-pass entry point (ckl_forward_backward)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--memory-sweep", action="store_true",
@@ -314,6 +316,61 @@ def bench_ours(args):
     if rc != 0:
         raise SystemExit(f"device status {rc} ({word}) after the timed steps")
 
+    # ------------------------------------------------------------ single pass
+    # ckl_forward_backward on the same inputs: each chunk's logits computed
+    # once (6 d V FLOP per token executed), reported beside the headline.
+    single = None
+    if not args.no_single_pass:
+        ws_sp = torch.empty(ckl.single_pass_workspace_bytes(T, d, V, K, chunk), dtype=torch.uint8,
+                            device=dev)
+
+        def sp_step(trace=None):
+            ckl.forward_backward(H, W, idx, logp, mask, chunk=chunk, dW=dW, accumulate_dW=False,
+                                 workspace=ws_sp, trace=trace, out_loss=loss, out_lse=lse,
+                                 out_dH=dH)
+
+        for _ in range(args.warmup):
+            sp_step()
+        torch.cuda.synchronize()
+        rc, word = ckl.read_device_status(ws_sp)
+        if rc != 0:
+            raise SystemExit(f"device status {rc} ({word}) in the single pass")
+        sp_trace = ckl.Trace(capacity=args.steps * (3 + 4 * chunks + 4) + 16)
+        if ws_n > 1:
+            torch.distributed.barrier()
+        g0 = torch.cuda.Event(enable_timing=True)
+        g1 = torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(args.steps):
+            sp_step(sp_trace)
+        g1.record(stream)
+        torch.cuda.synchronize()
+        if sp_trace.count >= sp_trace.capacity:
+            raise SystemExit("single-pass launch trace overflowed")
+        ms_sp = max_over_ranks(g0.elapsed_time(g1) / args.steps, ws_n, dev)
+        sp_per = {}
+        for name, ms in sp_trace.durations():
+            a = sp_per.setdefault(name, [0, 0.0])
+            a[0] += 1
+            a[1] += ms
+        sp_total = sum(x[1] for x in sp_per.values())
+        single = {
+            "value": round(tokens / (ms_sp / 1e3), 1), "unit": "tokens/s",
+            "ms_per_step": round(ms_sp, 4),
+            "executed_tflops": round(6.0 * d * V * tokens / (ms_sp / 1e3) / 1e12, 1),
+            "tflops_8dV_convention": round(flops_per_token(c) * tokens / (ms_sp / 1e3) / 1e12, 1),
+            "executed_flop_per_token": "6 d V (logits once, dH, dW)",
+            "gpu_launches": sp_trace.count,
+            "kernels": {k: {"launches": v[0], "total_ms": round(v[1], 3),
+                            "share": round(v[1] / sp_total, 4)}
+                        for k, v in sorted(sp_per.items())},
+            "workspace_bytes": ws_sp.numel(),
+        }
+        rc, word = ckl.read_device_status(ws_sp)
+        if rc != 0:
+            raise SystemExit(f"device status {rc} ({word}) after the single-pass steps")
+        del ws_sp
+
     # ------------------------------------------------------------ end to end
     e2e = None
     if not args.no_e2e:
@@ -383,6 +440,7 @@ def bench_ours(args):
         "peak_source": peak_src,
         "flop_convention": "8 d V per token (fwd logits, bwd recompute, dH, dW)",
         "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+        "single_pass": single,
         "gpu_launches": gpu_launches, "clocks": clocks,
         "workspace_bytes": ws.numel(),
         "peak_mem_bytes": int(torch.cuda.max_memory_allocated(dev)),

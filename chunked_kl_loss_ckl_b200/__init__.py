@@ -22,7 +22,7 @@ import torch
 __all__ = [
     "LIB_PATH", "CklError", "Trace", "KERNEL_NAMES", "lib", "workspace_bytes", "new_workspace",
     "forward", "backward", "read_device_status", "status_string", "chunked_kl_loss",
-    "topk_cache",
+    "topk_cache", "single_pass_workspace_bytes", "forward_backward",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libckl.so")
@@ -34,7 +34,7 @@ STATUS_NAMES = {
     8: "CKL_ERR_TOPK_TIES",
 }
 KERNEL_NAMES = {1: "prep", 2: "fwd_gemm", 3: "fwd_combine", 4: "bwd_dz", 5: "bwd_dhdw", 6: "other",
-                7: "topk"}
+                7: "topk", 8: "sp_gemm", 9: "sp_rows"}
 
 
 class CklError(RuntimeError):
@@ -54,6 +54,10 @@ def _load() -> ctypes.CDLL:
         raise ImportError(f"{LIB_PATH} is missing: build it with "
                           "`python -m chunked_kl_loss_ckl_b200._build` (nvcc, sm_100a)")
     L = ctypes.CDLL(LIB_PATH)
+    for name in ("ckl_forward", "ckl_backward", "ckl_forward_backward", "ckl_topk_cache"):
+        if not hasattr(L, name):
+            raise ImportError(f"{LIB_PATH} lacks {name}: it is older than its sources; rebuild "
+                              "with `python -m chunked_kl_loss_ckl_b200._build --force`")
     vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
     tr = ctypes.POINTER(_Trace)
     L.ckl_workspace_bytes.argtypes = [i64, i64, i64, i32, i64]
@@ -63,6 +67,11 @@ def _load() -> ctypes.CDLL:
     L.ckl_backward.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i64, vp, vp, vp, vp, i32,
                                vp, sz, vp, tr]
     L.ckl_backward.restype = ctypes.c_int
+    L.ckl_single_pass_workspace_bytes.argtypes = [i64, i64, i64, i32, i64]
+    L.ckl_single_pass_workspace_bytes.restype = sz
+    L.ckl_forward_backward.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i64, vp, vp, vp, vp,
+                                       vp, i32, vp, sz, vp, tr]
+    L.ckl_forward_backward.restype = ctypes.c_int
     L.ckl_topk_cache.argtypes = [vp, i64, i64, i32, vp, vp, vp, vp]
     L.ckl_topk_cache.restype = ctypes.c_int
     L.ckl_read_device_status.argtypes = [vp, vp, ctypes.POINTER(i32)]
@@ -195,6 +204,42 @@ def backward(H, W, idx, logp, mask, lse, grad_loss=None, chunk: int = 1024, dW=N
     if rc != CKL_OK:
         raise CklError(rc, "ckl_backward")
     return dH, dW
+
+
+def single_pass_workspace_bytes(T: int, d: int, V: int, K: int, chunk: int) -> int:
+    n = lib.ckl_single_pass_workspace_bytes(T, d, V, K, chunk)
+    if n == 0:
+        raise CklError(1, "ckl_single_pass_workspace_bytes")
+    return int(n)
+
+
+def forward_backward(H, W, idx, logp, mask=None, grad_loss=None, chunk: int = 1024, dW=None,
+                     accumulate_dW: bool = False, workspace=None, stream=None,
+                     trace: Trace | None = None, out_loss=None, out_lse=None, out_dH=None):
+    """Single pass: loss, lse, dH and dW with each chunk's logits computed once.
+
+    Returns (loss, lse, dH, dW).  The upstream gradient g (``grad_loss``, a
+    CUDA float32 [1] tensor; None = 1) must be known before the call.
+    """
+    T, d, V, K = _check_inputs(H, W, idx, logp, mask)
+    if workspace is None:
+        n = single_pass_workspace_bytes(T, d, V, K, chunk)
+        workspace = torch.empty(n, dtype=torch.uint8, device=H.device)
+    loss = out_loss if out_loss is not None else torch.empty(1, dtype=torch.float32, device=H.device)
+    lse = out_lse if out_lse is not None else torch.empty(T, dtype=torch.float32, device=H.device)
+    dH = out_dH if out_dH is not None else torch.empty(T, d, dtype=torch.bfloat16, device=H.device)
+    if dW is None:
+        dW = torch.empty(V, d, dtype=torch.float32, device=H.device)
+        accumulate_dW = False
+    if grad_loss is not None and (grad_loss.dtype != torch.float32 or not grad_loss.is_cuda):
+        raise TypeError("grad_loss must be a CUDA float32 tensor")
+    rc = lib.ckl_forward_backward(_ptr(H), _ptr(W), _ptr(idx), _ptr(logp), _ptr(mask), T, d, V, K,
+                                  chunk, _ptr(grad_loss), _ptr(loss), _ptr(lse), _ptr(dH),
+                                  _ptr(dW), int(bool(accumulate_dW)), _ptr(workspace),
+                                  workspace.numel(), _stream_handle(stream), _trace_ptr(trace))
+    if rc != CKL_OK:
+        raise CklError(rc, "ckl_forward_backward")
+    return loss, lse, dH, dW
 
 
 def topk_cache(logits, K: int, stream=None, status=None):

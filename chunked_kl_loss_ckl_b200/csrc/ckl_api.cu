@@ -31,13 +31,15 @@ inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255);
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 struct Layout {
-  size_t pairs, hp, partials, blocksums, dz, hct, total;
+  size_t pairs, hp, partials, blocksums, dz, hct, z, rowloss, total;
   int64_t npanels;  // dZ panels of 64 vocabulary columns
   int64_t cap;      // dZ rows per panel
   int64_t pitch_t;  // H_c^T row pitch (elements): cap rounded up to 8
+  int64_t zpitch;   // single pass: fp32 logit row pitch (elements), V rounded up to 4
 };
 
-Layout layout(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk) {
+// single_pass adds the chunk's fp32 logits [cap][zpitch] and the rows' loss terms [T].
+Layout layout(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk, bool single_pass) {
   Layout L{};
   size_t off = kHeaderBytes;
   L.pairs = off;
@@ -57,6 +59,13 @@ Layout layout(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk) {
   L.pitch_t = cdiv(L.cap, 8) * 8;
   L.hct = off;
   off += align256(static_cast<size_t>(d) * L.pitch_t * 2);
+  L.zpitch = cdiv(V, 4) * 4;
+  if (single_pass) {
+    L.z = off;
+    off += align256(static_cast<size_t>(L.cap) * L.zpitch * 4);
+    L.rowloss = off;
+    off += align256(static_cast<size_t>(T) * 4);
+  }
   L.total = off;
   return L;
 }
@@ -143,7 +152,7 @@ struct DevInfo {
   int sms = 0;
   int major = 0;
   bool attrs_set = false;
-  int slots[3] = {0, 0, 0};  // co-resident CTA pairs per GEMM mode
+  int slots[4] = {0, 0, 0, 0};  // co-resident CTA pairs per GEMM mode
 };
 
 template <int MODE>
@@ -207,7 +216,7 @@ bool device_info(DevInfo& out) {
   }
   if (!di.attrs_set && di.major == 10) {
     if (!setup_mode<ckl::MODE_FWD>(di) || !setup_mode<ckl::MODE_DZ>(di) ||
-        !setup_mode<ckl::MODE_DHDW>(di))
+        !setup_mode<ckl::MODE_DHDW>(di) || !setup_mode<ckl::MODE_FWDZ>(di))
       return false;
     di.attrs_set = true;
   }
@@ -279,14 +288,14 @@ int status_from_word(int32_t w) {
 int common_prep(const uint16_t* H, const uint16_t* W, const int32_t* idx, const float* logp,
                 const uint8_t* mask, int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk,
                 void* ws, size_t ws_bytes, cudaStream_t st, ckl_trace* trace, DevInfo& di,
-                Layout& L) {
+                Layout& L, bool single_pass = false) {
   if (!sizes_ok(T, d, V, K, chunk)) return CKL_ERR_INVALID_ARG;
   // H, topk_idx and topk_logp may be NULL only for an empty batch.
   if (!W || !ws || (T > 0 && (!H || !idx || !logp))) return CKL_ERR_INVALID_ARG;
   if (!aligned16(H) || !aligned16(W) || !aligned16(ws) || !aligned4(idx) || !aligned4(logp))
     return CKL_ERR_INVALID_ARG;
   if (K > ckl::PREP_MAXK) return CKL_ERR_UNSUPPORTED;
-  L = layout(T, d, V, K, chunk);
+  L = layout(T, d, V, K, chunk, single_pass);
   if (ws_bytes < L.total) return CKL_ERR_WORKSPACE;
   if (!device_info(di)) return CKL_ERR_CUDA;
   if (di.major != 10) return CKL_ERR_UNSUPPORTED;
@@ -320,13 +329,63 @@ void fill_common(TcParams& p, uint8_t* w8, const Layout& L, int64_t T, int64_t d
   p.countN = &hdr->countN;
 }
 
+// The dH rows of one chunk and its share of dW, from the chunk's dZ panels:
+// H_c^T (the K-major B operand of the dW GEMM), then one merged GEMM launch.
+int dhdw_chunk(const uint16_t* H, const uint16_t* W, const uint8_t* mask, int64_t T, int64_t d,
+               int64_t V, int32_t K, int64_t c0, int64_t rows, const float* grad_loss,
+               uint16_t* dH, float* dW, int32_t accumulate_dW, uint8_t* w8, const Layout& L,
+               const DevInfo& di, cudaStream_t st, ckl_trace* trace) {
+  const uint16_t* Hc = H + c0 * d;
+  void* dz = w8 + L.dz;
+  void* hct = w8 + L.hct;
+  const int bn = pick_bn(d);
+  {
+    TraceScope ts(trace, st, CKL_KERNEL_OTHER);
+    const dim3 grid(static_cast<unsigned>(cdiv(d, 32)), static_cast<unsigned>(cdiv(rows, 32)));
+    ckl::transpose_rows_kernel<<<grid, 256, 0, st>>>(Hc, static_cast<int>(rows),
+                                                     static_cast<int>(d),
+                                                     static_cast<uint16_t*>(hct),
+                                                     static_cast<int>(L.pitch_t));
+    if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
+  }
+  TcParams p;
+  std::memset(&p, 0, sizeof(p));
+  fill_common(p, w8, L, T, d, V, K, mask);
+  p.rows = static_cast<int32_t>(rows);
+  p.row0 = static_cast<int32_t>(c0);
+  p.bn = bn;
+  p.n_nt = static_cast<int32_t>(cdiv(d, bn));
+  p.n_mt = static_cast<int32_t>(cdiv(V, kMB));
+  p.n5 = static_cast<int32_t>(cdiv(rows, kMB)) * p.n_nt;
+  p.n6 = p.n_mt * p.n_nt;
+  p.c5 = static_cast<int32_t>(cdiv(V, ckl::BK));
+  p.c6 = static_cast<int32_t>(cdiv(rows, ckl::BK));
+  p.dw_store = (c0 == 0 && !accumulate_dW) ? 1 : 0;
+  p.grad_loss = grad_loss;
+  uint16_t* dHc = dH + c0 * d;
+  if (!map3d(&p.tm[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dz, 64, rows, L.npanels, 128,
+             L.cap * 128, ckl::BK, ckl::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map2d(&p.tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, V, d * 2, 64, ckl::BK,
+             CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map3d2(&p.tm[2], dz, 64, rows, L.npanels, 128, L.cap * 128, 64, ckl::BK, 2) ||
+      !map2d(&p.tm[3], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hct, rows, d, L.pitch_t * 2, ckl::BK,
+             bn / kSlotCTAs, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map2d(&p.tm[4], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dHc, d, rows, d * 2, 32, ckl::BM,
+             CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !map2d(&p.tm[5], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, dW, d, V, d * 4, 32, ckl::BM,
+             CU_TENSOR_MAP_SWIZZLE_128B))
+    return CKL_ERR_CUDA;
+  TraceScope ts(trace, st, CKL_KERNEL_BWD_DHDW);
+  return launch_tc<ckl::MODE_DHDW>(p, p.n5 + p.n6, di, st);
+}
+
 }  // namespace
 
 extern "C" {
 
 size_t ckl_workspace_bytes(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk) {
   if (!sizes_ok(T, d, V, K, chunk)) return 0;
-  return layout(T, d, V, K, chunk).total;
+  return layout(T, d, V, K, chunk, false).total;
 }
 
 int ckl_forward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
@@ -399,7 +458,6 @@ int ckl_backward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
   }
   uint8_t* w8 = static_cast<uint8_t*>(workspace);
   void* dz = w8 + L.dz;
-  const int bn = pick_bn(d);
 
   for (int64_t c0 = 0; c0 < T; c0 += chunk) {
     const int64_t rows = std::min<int64_t>(chunk, T - c0);
@@ -425,49 +483,87 @@ int ckl_backward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
       TraceScope ts(trace, st, CKL_KERNEL_BWD_DZ);
       if (launch_tc<ckl::MODE_DZ>(p, p.n_units, di, st) != CKL_OK) return CKL_ERR_CUDA;
     }
-    // ---- H_c^T, the K-major B operand of the dW GEMM
-    void* hct = w8 + L.hct;
+    rc = dhdw_chunk(H, W, mask, T, d, V, K, c0, rows, grad_loss, dH, dW, accumulate_dW, w8, L,
+                    di, st, trace);
+    if (rc != CKL_OK) return rc;
+  }
+  return CKL_OK;
+}
+
+size_t ckl_single_pass_workspace_bytes(int64_t T, int64_t d, int64_t V, int32_t K,
+                                       int64_t chunk) {
+  if (!sizes_ok(T, d, V, K, chunk)) return 0;
+  return layout(T, d, V, K, chunk, true).total;
+}
+
+int ckl_forward_backward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
+                         const float* topk_logp, const uint8_t* mask, int64_t T, int64_t d,
+                         int64_t V, int32_t K, int64_t chunk, const float* grad_loss, float* loss,
+                         float* lse, uint16_t* dH, float* dW, int32_t accumulate_dW,
+                         void* workspace, size_t workspace_bytes, void* stream,
+                         ckl_trace* trace) {
+  if (!loss || !aligned4(loss) || !dW || !aligned16(dW)) return CKL_ERR_INVALID_ARG;
+  if (T > 0 && (!lse || !aligned4(lse) || !dH || !aligned16(dH))) return CKL_ERR_INVALID_ARG;
+  if (grad_loss && !aligned4(grad_loss)) return CKL_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DevInfo di;
+  Layout L;
+  int rc = common_prep(H, W, topk_idx, topk_logp, mask, T, d, V, K, chunk, workspace,
+                       workspace_bytes, st, trace, di, L, true);
+  if (rc != CKL_OK) return rc;
+  if (T == 0) {
+    if (!accumulate_dW &&
+        cudaMemsetAsync(dW, 0, static_cast<size_t>(V) * d * sizeof(float), st) != cudaSuccess)
+      return CKL_ERR_CUDA;
+    TraceScope ts(trace, st, CKL_KERNEL_OTHER);
+    ckl::zero_loss_kernel<<<1, 1, 0, st>>>(loss);
+    return cudaGetLastError() == cudaSuccess ? CKL_OK : CKL_ERR_CUDA;
+  }
+  uint8_t* w8 = static_cast<uint8_t*>(workspace);
+  Header* hdr = reinterpret_cast<Header*>(w8);
+  float* z = reinterpret_cast<float*>(w8 + L.z);
+  float* rowloss = reinterpret_cast<float*>(w8 + L.rowloss);
+  for (int64_t c0 = 0; c0 < T; c0 += chunk) {
+    const int64_t rows = std::min<int64_t>(chunk, T - c0);
+    const uint16_t* Hc = H + c0 * d;
+    // ---- logits of this chunk, once: online log-sum-exp + gather partials and fp32 z
+    TcParams p;
+    std::memset(&p, 0, sizeof(p));
+    fill_common(p, w8, L, T, d, V, K, mask);
+    p.rows = static_cast<int32_t>(rows);
+    p.row0 = static_cast<int32_t>(c0);
+    p.n_rb = static_cast<int32_t>(cdiv(rows, kMB));
+    p.S = choose_splits(p.n_rb, p.n_vt, di.slots[ckl::MODE_FWDZ]);
+    p.n_units = p.n_rb * p.S;
+    if (!map2d(&p.tm[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Hc, d, rows, d * 2, ckl::BK, ckl::BM,
+               CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map2d(&p.tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, V, d * 2, ckl::BK,
+               ckl::BN_V / kSlotCTAs, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map2d(&p.tm[2], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, z, V, rows, L.zpitch * 4, 32, ckl::BM,
+               CU_TENSOR_MAP_SWIZZLE_128B))
+      return CKL_ERR_CUDA;
     {
-      TraceScope ts(trace, st, CKL_KERNEL_OTHER);
-      const dim3 grid(static_cast<unsigned>(cdiv(d, 32)), static_cast<unsigned>(cdiv(rows, 32)));
-      ckl::transpose_rows_kernel<<<grid, 256, 0, st>>>(Hc, static_cast<int>(rows),
-                                                       static_cast<int>(d),
-                                                       static_cast<uint16_t*>(hct),
-                                                       static_cast<int>(L.pitch_t));
+      TraceScope ts(trace, st, CKL_KERNEL_SP_GEMM);
+      if (launch_tc<ckl::MODE_FWDZ>(p, p.n_units, di, st) != CKL_OK) return CKL_ERR_CUDA;
+    }
+    // ---- lse, the rows' loss terms and dZ from the stored logits
+    {
+      TraceScope ts(trace, st, CKL_KERNEL_SP_ROWS);
+      ckl::zrow_kernel<<<static_cast<unsigned>(rows), ckl::ZROW_THREADS, 0, st>>>(
+          z, L.zpitch, reinterpret_cast<const float4*>(w8 + L.partials), p.S,
+          reinterpret_cast<const float*>(w8 + L.hp), mask,
+          reinterpret_cast<const int2*>(w8 + L.pairs), K, static_cast<int>(V), c0, L.cap, lse,
+          rowloss, reinterpret_cast<uint16_t*>(w8 + L.dz));
       if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
     }
-    // ---- dH rows of this chunk and its share of dW, one launch
-    {
-      TcParams p;
-      std::memset(&p, 0, sizeof(p));
-      fill_common(p, w8, L, T, d, V, K, mask);
-      p.rows = static_cast<int32_t>(rows);
-      p.row0 = static_cast<int32_t>(c0);
-      p.bn = bn;
-      p.n_nt = static_cast<int32_t>(cdiv(d, bn));
-      p.n_mt = static_cast<int32_t>(cdiv(V, kMB));
-      p.n5 = static_cast<int32_t>(cdiv(rows, kMB)) * p.n_nt;
-      p.n6 = p.n_mt * p.n_nt;
-      p.c5 = static_cast<int32_t>(cdiv(V, ckl::BK));
-      p.c6 = static_cast<int32_t>(cdiv(rows, ckl::BK));
-      p.dw_store = (c0 == 0 && !accumulate_dW) ? 1 : 0;
-      p.grad_loss = grad_loss;
-      uint16_t* dHc = dH + c0 * d;
-      if (!map3d(&p.tm[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dz, 64, rows, L.npanels, 128,
-                 L.cap * 128, ckl::BK, ckl::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-          !map2d(&p.tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, V, d * 2, 64, ckl::BK,
-                 CU_TENSOR_MAP_SWIZZLE_128B) ||
-          !map3d2(&p.tm[2], dz, 64, rows, L.npanels, 128, L.cap * 128, 64, ckl::BK, 2) ||
-          !map2d(&p.tm[3], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hct, rows, d, L.pitch_t * 2, ckl::BK,
-                 bn / kSlotCTAs, CU_TENSOR_MAP_SWIZZLE_128B) ||
-          !map2d(&p.tm[4], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dHc, d, rows, d * 2, 32, ckl::BM,
-                 CU_TENSOR_MAP_SWIZZLE_64B) ||
-          !map2d(&p.tm[5], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, dW, d, V, d * 4, 32, ckl::BM,
-                 CU_TENSOR_MAP_SWIZZLE_128B))
-        return CKL_ERR_CUDA;
-      TraceScope ts(trace, st, CKL_KERNEL_BWD_DHDW);
-      if (launch_tc<ckl::MODE_DHDW>(p, p.n5 + p.n6, di, st) != CKL_OK) return CKL_ERR_CUDA;
-    }
+    rc = dhdw_chunk(H, W, mask, T, d, V, K, c0, rows, grad_loss, dH, dW, accumulate_dW, w8, L,
+                    di, st, trace);
+    if (rc != CKL_OK) return rc;
+  }
+  {
+    TraceScope ts(trace, st, CKL_KERNEL_FWD_COMBINE);
+    ckl::rowsum_loss_kernel<<<1, ckl::ROWSUM_THREADS, 0, st>>>(rowloss, T, &hdr->countN, loss);
+    if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
   }
   return CKL_OK;
 }

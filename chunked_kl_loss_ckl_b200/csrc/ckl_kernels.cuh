@@ -44,7 +44,10 @@ constexpr int EPI_STAGE = BM * 128;         // one 128-row x 128-byte staging ti
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COLS = 256;          // TMEM columns per accumulator buffer
 
-enum Mode { MODE_FWD = 0, MODE_DZ = 1, MODE_DHDW = 2 };
+// FWD: logits + online log-sum-exp + teacher gather; DZ: logit recompute +
+// dZ; DHDW: dH and dW of one chunk; FWDZ: FWD over one chunk that also
+// stores the fp32 logits (the single-pass schedule).
+enum Mode { MODE_FWD = 0, MODE_DZ = 1, MODE_DHDW = 2, MODE_FWDZ = 3 };
 
 // Pipeline depth and epilogue width.  A single CTA holds a 128 x 256 tile:
 // four 48 KB operand stages fill the shared memory beside the epilogue
@@ -267,6 +270,95 @@ transpose_rows_kernel(const uint16_t* __restrict__ Hc, int rows, int d, uint16_t
 // Loss of an empty batch (T = 0).
 __global__ void zero_loss_kernel(float* loss) { *loss = 0.f; }
 
+// ------------------------------------------------------------------ single pass
+// One chunk row per CTA, after the FWDZ GEMM: merge the row's vocabulary
+// splits into lse_t and its loss term m_t (Hp_t - pz_t + lse_t), then turn the
+// stored fp32 logits into dZ_t = m_t (exp(z - lse_t) - scatter p_t) as bf16 in
+// the 64-column panel layout the dH/dW GEMM reads (columns V .. round_up(V, 64)
+// are written 0).  Same arithmetic as the recompute path's dZ epilogue.
+constexpr int ZROW_THREADS = 512;
+
+__global__ void __launch_bounds__(ZROW_THREADS)
+zrow_kernel(const float* __restrict__ Z, int64_t zpitch, const float4* __restrict__ partials,
+            int S, const float* __restrict__ Hp, const uint8_t* __restrict__ mask,
+            const int2* __restrict__ pairs, int K, int V, int64_t row0, int64_t cap,
+            float* __restrict__ lse, float* __restrict__ rowloss, uint16_t* __restrict__ dz) {
+  __shared__ float s_lse2;
+  __shared__ int s_counts;
+  const int r = blockIdx.x;
+  const int64_t t = row0 + r;
+  if (threadIdx.x == 0) {
+    const float4* pr = partials + t * S;
+    float M = -INFINITY;
+    for (int s = 0; s < S; ++s) M = fmaxf(M, pr[s].x);
+    float se = 0.f, pz = 0.f;
+    for (int s = 0; s < S; ++s) {
+      const float4 q = pr[s];
+      se += q.y * exp2f(q.x - M);
+      pz += q.z;
+    }
+    const float l = (M + log2f(se)) * LN2;
+    const int counts = (mask == nullptr || mask[t] != 0) ? 1 : 0;
+    lse[t] = l;
+    rowloss[t] = counts ? Hp[t] - pz + l : 0.f;
+    s_lse2 = l * LOG2E;
+    s_counts = counts;
+  }
+  __syncthreads();
+  const float lse2 = s_lse2;
+  const bool counts = s_counts != 0;
+  const float* zr = Z + static_cast<int64_t>(r) * zpitch;
+  const int vend = (V + 63) & ~63;
+  // softmax part, four columns per thread and step
+  for (int v = 4 * threadIdx.x; v < vend; v += 4 * ZROW_THREADS) {
+    float q[4] = {0.f, 0.f, 0.f, 0.f};
+    if (counts && v < V) {
+      const float4 z = *reinterpret_cast<const float4*>(zr + v);
+      const float zz[4] = {z.x, z.y, z.z, z.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) q[j] = (v + j < V) ? ex2_approx(fmaf(zz[j], LOG2E, -lse2)) : 0.f;
+    }
+    uint2 o;
+    o.x = pack_bf16x2(q[0], q[1]);
+    o.y = pack_bf16x2(q[2], q[3]);
+    *reinterpret_cast<uint2*>(dz + ((static_cast<int64_t>(v >> 6) * cap + r) << 6) + (v & 63)) = o;
+  }
+  __syncthreads();
+  // teacher entries: the first of each run of equal ids rewrites its column
+  // (q minus every p of the run, subtracted in sorted order)
+  if (counts) {
+    const int2* pr = pairs + t * K;
+    for (int k = threadIdx.x; k < K; k += ZROW_THREADS) {
+      const int id = pr[k].x;
+      if (id < 0 || id >= V || (k > 0 && pr[k - 1].x == id)) continue;
+      float x = ex2_approx(fmaf(zr[id], LOG2E, -lse2));
+      for (int j = k; j < K && pr[j].x == id; ++j) x -= __int_as_float(pr[j].y);
+      const uint32_t b = pack_bf16x2(x, 0.f);
+      dz[((static_cast<int64_t>(id >> 6) * cap + r) << 6) + (id & 63)] = static_cast<uint16_t>(b & 0xFFFFu);
+    }
+  }
+}
+
+// loss = (sum of the rows' terms, in a fixed order, in fp64) / N.
+constexpr int ROWSUM_THREADS = 1024;
+
+__global__ void __launch_bounds__(ROWSUM_THREADS)
+rowsum_loss_kernel(const float* __restrict__ rowloss, int64_t T, const int* countN, float* loss) {
+  __shared__ double s[ROWSUM_THREADS];
+  double v = 0.0;
+  for (int64_t t = threadIdx.x; t < T; t += ROWSUM_THREADS) v += static_cast<double>(rowloss[t]);
+  s[threadIdx.x] = v;
+  __syncthreads();
+  for (int h = ROWSUM_THREADS / 2; h > 0; h >>= 1) {
+    if (threadIdx.x < h) s[threadIdx.x] += s[threadIdx.x + h];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const int n = *countN;
+    *loss = (n > 0) ? static_cast<float>(s[0] / static_cast<double>(n)) : 0.f;
+  }
+}
+
 // ------------------------------------------------------------------ tc GEMM
 
 // dW units of this CTA: a contiguous range sized so that every CTA's total
@@ -384,7 +476,7 @@ tc_kernel(const __grid_constant__ TcParams p) {
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::BAR_OFF + 8 * (2 * STAGES + 9));
 
   if (warp == 0 && lane == 0) {
-    const int n_maps = (MODE == MODE_FWD) ? 2 : (MODE == MODE_DZ) ? 3 : 6;
+    const int n_maps = (MODE == MODE_FWD) ? 2 : (MODE == MODE_DHDW) ? 6 : 3;
 #pragma unroll 1
     for (int i = 0; i < n_maps; ++i) prefetch_tmap(&p.tm[i]);
     for (int s = 0; s < STAGES; ++s) {
@@ -596,7 +688,7 @@ tc_kernel(const __grid_constant__ TcParams p) {
       return __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
     };
     // Publish this warp's rows; the issuer stores the tile once all warps have
-    // (kind 0: dZ panel, 1: dH, 2: dW store, 3: dW add) and then frees the
+    // (kind 0: dZ panel, 1: dH, 2: dW store, 3: dW add, 4: logits) and then frees the
     // tile of the store before.
     auto stage_end = [&](int kind, int x, int y, int z) -> bool {
       fence_proxy_async_smem();
@@ -611,7 +703,8 @@ tc_kernel(const __grid_constant__ TcParams p) {
           if (kind == 0) tma_store_3d(&p.tm[2], buf, x, y, z);
           else if (kind == 1) tma_store_2d(&p.tm[4], buf, x, y);
           else if (kind == 2) tma_store_2d(&p.tm[5], buf, x, y);
-          else tma_reduce_add_2d(&p.tm[5], buf, x, y);
+          else if (kind == 3) tma_reduce_add_2d(&p.tm[5], buf, x, y);
+          else tma_store_2d(&p.tm[2], buf, x, y);
           bulk_commit();
           if (nstore >= 1) {
             bulk_wait_read<1>();
@@ -650,7 +743,7 @@ tc_kernel(const __grid_constant__ TcParams p) {
         run_m = -INFINITY; run_s = 0.f; run_pz = 0.f;
         nidx = INT_MAX;
         if (MODE == MODE_DZ && row_ok) lse2 = p.lse[t] * LOG2E;
-        const bool want_ids = (MODE == MODE_FWD) ? row_ok : counts;
+        const bool want_ids = (MODE == MODE_DZ) ? counts : row_ok;
         if (want_ids) {
           const int2* pr = p.pairs + t * p.K;
           const int v_lo = it.vt * BN_V;
@@ -667,12 +760,25 @@ tc_kernel(const __grid_constant__ TcParams p) {
       tc_fence_after();
       const uint32_t tacc = tmem_base + lane_off + static_cast<uint32_t>(acc) * ACC_COLS;
 
-      if (MODE == MODE_FWD) {
+      if (MODE == MODE_FWD || MODE == MODE_FWDZ) {
+        const int zy0 = (it.u % p.n_rb) * MB + row0_cta;  // FWDZ: first chunk row of this CTA
         for (int c = 0; c < BN_V / 32; ++c) {
           const int v0 = it.vt * BN_V + c * 32;
           if (v0 >= p.V) break;
           float x[32];
           tmem_ld32(tacc + c * 32, x);
+          if (MODE == MODE_FWDZ) {
+            // the fp32 logits of this 128 x 32 block (columns past V are clipped by the store)
+            if (!stage_begin()) { ok = false; break; }
+            const uint32_t rowa = stage_base + (nstore & 1) * EPI_STAGE + srow * 128;
+            const int sw = lane & 7;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              st_shared_v4(rowa + ((j ^ sw) << 4), __float_as_uint(x[4 * j]),
+                           __float_as_uint(x[4 * j + 1]), __float_as_uint(x[4 * j + 2]),
+                           __float_as_uint(x[4 * j + 3]));
+            if (!stage_end(4, v0, zy0, 0)) { ok = false; break; }
+          }
           if (v0 + 32 > p.V) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) if (v0 + j >= p.V) x[j] = -INFINITY;
@@ -774,7 +880,7 @@ tc_kernel(const __grid_constant__ TcParams p) {
       else mbar_arrive(bar_tempty + 8 * acc);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
 
-      if (MODE == MODE_FWD && it.last_of_unit() && row_ok) {
+      if ((MODE == MODE_FWD || MODE == MODE_FWDZ) && it.last_of_unit() && row_ok) {
         const int s = it.u / p.n_rb;
         p.partials[t * p.S + s] = make_float4(run_m, run_s, run_pz, 0.f);
       }

@@ -80,7 +80,9 @@ enum {
   CKL_KERNEL_BWD_DZ = 4,      /* logit recompute + dZ = softmax - scatter(p) */
   CKL_KERNEL_BWD_DHDW = 5,    /* dH = s dZ W and dW += s dZ^T H for one chunk */
   CKL_KERNEL_OTHER = 6,
-  CKL_KERNEL_TOPK = 7         /* teacher top-K cache producer */
+  CKL_KERNEL_TOPK = 7,        /* teacher top-K cache producer */
+  CKL_KERNEL_SP_GEMM = 8,     /* single pass: one chunk's logit GEMM, stores fp32 z too */
+  CKL_KERNEL_SP_ROWS = 9      /* single pass: lse, loss terms and dZ from the stored z */
 };
 
 /*
@@ -151,6 +153,36 @@ CKL_API int ckl_backward(const uint16_t* H, const uint16_t* W, const int32_t* to
                  int32_t K, int64_t chunk, const float* lse, const float* grad_loss,
                  uint16_t* dH, float* dW, int32_t accumulate_dW, void* workspace,
                  size_t workspace_bytes, void* stream, ckl_trace* trace);
+
+/*
+ * Single-pass forward + backward (the loss is the only consumer of the
+ * logits, and g is known before the forward runs).
+ *
+ * The pages measure the fused method's backward projection as its extra cost
+ * at 8K context ("Tối ưu hóa chi phí chưng cất tri thức ...", section "Điều
+ * này thay đổi những gì trong thực tế"; "LLMのための効率的な知識蒸留", table
+ * in "パフォーマンスとメモリのベンチマーク": fused chunked slower than
+ * forward-chunked).  This entry point drops the recompute: per chunk of rows
+ * it runs the logit GEMM once, storing the chunk's fp32 logits (chunk x V)
+ * beside the online log-sum-exp, turns them into dZ once lse is known, and
+ * feeds dZ to the same dH / dW GEMMs as ckl_backward.  6 d V FLOP per token
+ * instead of 8 d V, for chunk x V x 4 more workspace bytes.  Results equal
+ * ckl_forward followed by ckl_backward up to rounding (lse may differ in the
+ * last bits: the vocabulary is split differently per chunk).
+ *   grad_loss  [1]    fp32  upstream gradient g (device); NULL = 1
+ *   loss, lse               as in ckl_forward
+ *   dH, dW, accumulate_dW   as in ckl_backward
+ *   workspace               >= ckl_single_pass_workspace_bytes(...) bytes
+ * Other arguments as in ckl_forward.
+ */
+CKL_API size_t ckl_single_pass_workspace_bytes(int64_t T, int64_t d, int64_t V, int32_t K,
+                                               int64_t chunk);
+CKL_API int ckl_forward_backward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
+                                 const float* topk_logp, const uint8_t* mask, int64_t T,
+                                 int64_t d, int64_t V, int32_t K, int64_t chunk,
+                                 const float* grad_loss, float* loss, float* lse, uint16_t* dH,
+                                 float* dW, int32_t accumulate_dW, void* workspace,
+                                 size_t workspace_bytes, void* stream, ckl_trace* trace);
 
 /*
  * Reads the device status word of the last call that used `workspace`:

@@ -22,9 +22,10 @@ def ckl():
 
 
 def test_header_declares_the_entry_points():
-    assert _declared() == ["ckl_backward", "ckl_forward", "ckl_forward_static_scratch",
-                           "ckl_read_device_status", "ckl_status_string", "ckl_topk_cache",
-                           "ckl_version", "ckl_workspace_bytes"]
+    assert _declared() == ["ckl_backward", "ckl_forward", "ckl_forward_backward",
+                           "ckl_forward_static_scratch", "ckl_read_device_status",
+                           "ckl_single_pass_workspace_bytes", "ckl_status_string",
+                           "ckl_topk_cache", "ckl_version", "ckl_workspace_bytes"]
 
 
 def test_library_exports_every_declared_symbol(ckl):
@@ -50,6 +51,17 @@ def test_workspace_is_linear_in_T(ckl):
     assert abs(slope1 / 8192 - (K * 8 + 4 + 64 * 16 + 8 / 256)) < 1.0
     # the dZ buffer is chunk x round_up(V, 8) bf16
     assert ws[0] - 8192 * (K * 8 + 4 + 64 * 16) >= chunk * V * 2
+
+
+def test_single_pass_workspace_adds_the_chunk_logits(ckl):
+    d, V, K, chunk = 3072, 128256, 100, 1024
+    for T in (100, 8192, 32768):
+        base = ckl.lib.ckl_workspace_bytes(T, d, V, K, chunk)
+        sp = ckl.lib.ckl_single_pass_workspace_bytes(T, d, V, K, chunk)
+        rows = min(chunk, T)
+        extra = rows * ((V + 3) // 4 * 4) * 4 + T * 4  # fp32 logits + per-row loss terms
+        assert extra <= sp - base <= extra + 512
+    assert ckl.lib.ckl_single_pass_workspace_bytes(10, 60, 100, 4, 8) == 0
 
 
 def test_workspace_rejects_bad_sizes(ckl):
@@ -84,6 +96,15 @@ def test_host_checks_return_before_any_device_work(ckl):
     # backward: null dW
     assert L.ckl_backward(fake, fake, fake, fake, nul, 4, 64, 100, 4, 8, fake, nul, fake, nul, 0,
                           fake, 1 << 20, nul, nul) == 1
+    # single pass: null dW, null loss, and the larger workspace it needs
+    assert L.ckl_forward_backward(fake, fake, fake, fake, nul, 4, 64, 100, 4, 8, nul, fake, fake,
+                                  fake, nul, 0, fake, 1 << 20, nul, nul) == 1
+    assert L.ckl_forward_backward(fake, fake, fake, fake, nul, 4, 64, 100, 4, 8, nul, nul, fake,
+                                  fake, fake, 0, fake, 1 << 20, nul, nul) == 1
+    small = L.ckl_workspace_bytes(4, 64, 100, 4, 8)
+    assert small < L.ckl_single_pass_workspace_bytes(4, 64, 100, 4, 8)
+    assert L.ckl_forward_backward(fake, fake, fake, fake, nul, 4, 64, 100, 4, 8, nul, fake, fake,
+                                  fake, fake, 0, fake, small, nul, nul) == 3
     assert L.ckl_read_device_status(nul, nul, nul) == 1
     # top-K cache: K must be in [1, min(V, 2048)]
     assert L.ckl_topk_cache(fake, 4, 100, 0, fake, fake, nul, nul) == 1

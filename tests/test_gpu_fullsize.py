@@ -42,16 +42,22 @@ def _sample_rows(c, n=10, seed=123):
     return np.array(sorted(rows))
 
 
-def _run(ckl, c, mask, rows, vrows=None):
-    """One forward + backward at full size; returns only what the checks use
-    (the full outputs are gigabytes)."""
+def _run(ckl, c, mask, rows, vrows=None, single_pass=False):
+    """One forward + backward at full size (two calls, or the single-pass
+    call); returns only what the checks use (the full outputs are gigabytes)."""
     H, W, idx, logp, m = to_device(c, mask)
     T, d, V, K, chunk = c["T"], c["d"], c["V"], c["K"], c["chunk"]
-    ws = ckl.new_workspace(T, d, V, K, chunk)
-    loss, lse = ckl.forward(H, W, idx, logp, m, chunk, workspace=ws)
-    st_f = ckl.read_device_status(ws)
-    dH, dW = ckl.backward(H, W, idx, logp, m, lse, chunk=chunk, workspace=ws)
-    st_b = ckl.read_device_status(ws)
+    if single_pass:
+        ws = torch.empty(ckl.single_pass_workspace_bytes(T, d, V, K, chunk), dtype=torch.uint8,
+                         device="cuda")
+        loss, lse, dH, dW = ckl.forward_backward(H, W, idx, logp, m, chunk=chunk, workspace=ws)
+        st_f = st_b = ckl.read_device_status(ws)
+    else:
+        ws = ckl.new_workspace(T, d, V, K, chunk)
+        loss, lse = ckl.forward(H, W, idx, logp, m, chunk, workspace=ws)
+        st_f = ckl.read_device_status(ws)
+        dH, dW = ckl.backward(H, W, idx, logp, m, lse, chunk=chunk, workspace=ws)
+        st_b = ckl.read_device_status(ws)
     r = torch.from_numpy(rows).cuda()
     out = dict(loss=float(loss.item()), lse=lse[r].double().cpu().numpy(),
                dH=dH[r].double().cpu().numpy(), status=(st_f[0], st_b[0]),
@@ -66,13 +72,16 @@ def _run(ckl, c, mask, rows, vrows=None):
     return out
 
 
-@pytest.mark.parametrize("name", ["8k", "32k", "oss", "256k"])
-def test_full_size_workload(gpu_lib, name):
+@pytest.mark.parametrize("name,single_pass", [("8k", False), ("32k", False), ("oss", False),
+                                              ("256k", False), ("8k", True), ("oss", True)])
+def test_full_size_workload(gpu_lib, name, single_pass):
     c = _config(name)
     T, V = c["T"], c["V"]
+    if single_pass:
+        name += " single pass"
     # --- run A: the workload as given
     rows = _sample_rows(c)
-    a = _run(gpu_lib, c, "config", rows)
+    a = _run(gpu_lib, c, "config", rows, single_pass=single_pass)
     assert a["status"] == (0, 0)
     assert np.isfinite(a["loss"]) and a["loss"] > 0
     N = T if c["mask"] is None else int((c["mask"] != 0).sum())
@@ -91,7 +100,7 @@ def test_full_size_workload(gpu_lib, name):
     vset = set(range(64)) | set(int(v) for v in c["idx"][rows_b].ravel()) | {V - 1}
     vset |= set(int(v) for v in np.random.default_rng(11).choice(V, 1024, replace=False))
     vrows = np.array(sorted(vset))
-    b = _run(gpu_lib, c, mask, rows_b, vrows)
+    b = _run(gpu_lib, c, mask, rows_b, vrows, single_pass=single_pass)
     assert b["status"] == (0, 0)
     ref_b = oracle.rows_subset(c["H"], c["W"], c["idx"], c["logp"], rows_b, N=len(rows_b),
                                mask=mask)
