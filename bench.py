@@ -250,10 +250,12 @@ def bench_ours(args):
     if rc != 0:
         raise SystemExit(f"device status {rc} ({word}) after warm-up")
 
-    # forward: prep, logits GEMM, combine; backward: prep + per chunk
-    # (dZ GEMM, H_c transpose, dH/dW GEMM); the capacity leaves headroom and
-    # a full trace is treated as an error below.
-    n_launch = 3 + 1 + 3 * ((T + chunk - 1) // chunk)
+    # forward: prep, logits GEMM, combine; backward: prep + per row chunk an
+    # H_c transpose, per vocabulary slab a dZ GEMM and a dH/dW GEMM, and a dH
+    # conversion when sliced; the capacity leaves headroom and a full trace is
+    # treated as an error below.
+    Cr, Sv, n_slabs = ckl.backward_plan(T, d, V, K, chunk)
+    n_launch = 3 + 1 + -(-T // Cr) * (1 + 2 * n_slabs + (1 if n_slabs > 1 else 0))
     trace = ckl.Trace(capacity=args.steps * (n_launch + 4) + 16)
     uuid = None
     try:
@@ -292,10 +294,13 @@ def bench_ours(args):
         a[1] += ms
     gpu_launches = trace.count
     peaks, peak_src = load_peaks()
-    # algorithmic FLOPs per launch of each tensor-core kernel
+    # algorithmic FLOPs per launch of each tensor-core kernel: its FLOPs per
+    # step (forward logits 2 T V d; recompute 2 T V d; dH + dW 4 T V d) over
+    # its launches per step (the backward's blocking sets the count)
     chunks = (T + chunk - 1) // chunk
-    alg = {"fwd_gemm": 2.0 * T * V * d, "bwd_dz": 2.0 * T * V * d / chunks,
-           "bwd_dhdw": 4.0 * T * V * d / chunks}
+    per_step = {"fwd_gemm": 2.0 * T * V * d, "bwd_dz": 2.0 * T * V * d,
+                "bwd_dhdw": 4.0 * T * V * d}
+    alg = {k: v / (per[k][0] / args.steps) for k, v in per_step.items() if k in per}
     dom = max(per, key=lambda k: per[k][1])
     dom_avg_ms = per[dom][1] / per[dom][0]
     roofline = None
@@ -432,7 +437,8 @@ def bench_ours(args):
         "data": "synthetic",
         "config": {"workload": workload_desc(c), "T": T, "d": d, "V": V, "K": K, "chunk": chunk,
                    "global_batch_tokens": tokens, "parallelism": f"dp{ws_n} (independent batches)",
-                   "l2": "inputs larger than L2 (W 788 MB, dZ chunk buffer 263 MB vs 126 MB L2); "
+                   "backward_blocking": {"rows": Cr, "vocab_slab": Sv, "slabs": n_slabs},
+                   "l2": "inputs larger than L2 (W 788 MB, dZ buffer 263 MB vs 126 MB L2); "
                          "no flush"},
         "tflops": round(tflops, 1),
         "pct_peak_sustained": round(tflops / float(peaks.get("bf16_tflops_sustained", 1400.0)), 4),

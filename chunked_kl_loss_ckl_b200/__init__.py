@@ -22,7 +22,7 @@ import torch
 __all__ = [
     "LIB_PATH", "CklError", "Trace", "KERNEL_NAMES", "lib", "workspace_bytes", "new_workspace",
     "forward", "backward", "read_device_status", "status_string", "chunked_kl_loss",
-    "topk_cache", "single_pass_workspace_bytes", "forward_backward",
+    "topk_cache", "single_pass_workspace_bytes", "forward_backward", "backward_plan",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libckl.so")
@@ -67,6 +67,8 @@ def _load() -> ctypes.CDLL:
     L.ckl_backward.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i64, vp, vp, vp, vp, i32,
                                vp, sz, vp, tr]
     L.ckl_backward.restype = ctypes.c_int
+    L.ckl_backward_plan.argtypes = [i64, i64, i64, i32, i64, ctypes.POINTER(i64)]
+    L.ckl_backward_plan.restype = ctypes.c_int
     L.ckl_single_pass_workspace_bytes.argtypes = [i64, i64, i64, i32, i64]
     L.ckl_single_pass_workspace_bytes.restype = sz
     L.ckl_forward_backward.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i64, vp, vp, vp, vp,
@@ -204,6 +206,15 @@ def backward(H, W, idx, logp, mask, lse, grad_loss=None, chunk: int = 1024, dW=N
     if rc != CKL_OK:
         raise CklError(rc, "ckl_backward")
     return dH, dW
+
+
+def backward_plan(T: int, d: int, V: int, K: int, chunk: int):
+    """(rows per row chunk, vocabulary columns per slab, slabs) of ckl_backward."""
+    out = (ctypes.c_int64 * 3)()
+    rc = lib.ckl_backward_plan(T, d, V, K, chunk, out)
+    if rc != CKL_OK:
+        raise CklError(rc, "ckl_backward_plan")
+    return int(out[0]), int(out[1]), int(out[2])
 
 
 def single_pass_workspace_bytes(T: int, d: int, V: int, K: int, chunk: int) -> int:

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -30,13 +31,52 @@ struct Header {
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Blocking of the backward: row chunks of Cr rows x vocabulary slabs of Sv
+// columns (n slabs), every block's dZ fitting the chunk x V buffer.
+struct Plan {
+  int64_t Cr, Sv, n;
+};
+
 struct Layout {
-  size_t pairs, hp, partials, blocksums, dz, hct, z, rowloss, total;
-  int64_t npanels;  // dZ panels of 64 vocabulary columns
-  int64_t cap;      // dZ rows per panel
-  int64_t pitch_t;  // H_c^T row pitch (elements): cap rounded up to 8
+  size_t pairs, hp, partials, blocksums, dz, hct, dh32, z, rowloss, total;
+  int64_t npanels;  // dZ panels of 64 vocabulary columns (row-chunked schedule)
+  int64_t cap;      // rows of one chunk: min(chunk, T)
+  int64_t cr_alloc; // rows the sliced schedule may hold (0 = never sliced)
+  int64_t pitch_t;  // H_c^T row pitch (elements): max(cap, cr_alloc) rounded up to 8
   int64_t zpitch;   // single pass: fp32 logit row pitch (elements), V rounded up to 4
 };
+
+// The rows of a sliced block: the Cr that balances the two fp32 accumulations'
+// traffic (dW re-added once per row chunk, partial dH once per slab) under
+// Cr x Sv = chunk x V, i.e. sqrt(chunk x V), rounded up to 256.
+int64_t sliced_rows(int64_t T, int64_t V, int64_t cap) {
+  if (T <= cap) return 0;
+  int64_t r = static_cast<int64_t>(std::ceil(std::sqrt(static_cast<double>(cap) * V)));
+  r = cdiv(r, 256) * 256;
+  return r > cap ? r : 0;
+}
+
+// Row-chunked (the pages' schedule: one chunk of rows x all V at a time) or
+// sliced (fewer, taller row chunks, each swept in vocabulary slabs), whichever
+// moves fewer bytes of fp32 accumulation: row chunking reads and writes dW
+// (V x d fp32) once per chunk; slicing writes dW once per tall row chunk and
+// reads and writes a partial dH (rows x d fp32) once per slab.
+Plan plan_backward(int64_t T, int64_t d, int64_t V, const Layout& L) {
+  const int64_t Vp = cdiv(V, 64) * 64;
+  const Plan rows_only{L.cap, Vp, 1};
+  if (L.cr_alloc == 0) return rows_only;
+  const int64_t budget = L.cap * Vp;  // dZ entries the workspace holds
+  const int64_t Cr = std::min(T, L.cr_alloc);
+  int64_t Sv = budget / Cr / 256 * 256;
+  if (Sv < 256 || Sv >= Vp) return rows_only;
+  int64_t n = cdiv(Vp, Sv);
+  Sv = cdiv(cdiv(Vp, n), 256) * 256;  // even slabs
+  n = cdiv(Vp, Sv);
+  const double vd4 = 4.0 * static_cast<double>(V) * d, td4 = 4.0 * static_cast<double>(T) * d;
+  const double rows_bytes = (2.0 * cdiv(T, L.cap) - 1.0) * vd4;
+  const double sliced_bytes = (2.0 * cdiv(T, Cr) - 1.0) * vd4 + (2.0 * n - 1.0) * td4 + 1.5 * td4;
+  return sliced_bytes < rows_bytes ? Plan{Cr, Sv, n} : rows_only;
+}
 
 // single_pass adds the chunk's fp32 logits [cap][zpitch] and the rows' loss terms [T].
 Layout layout(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk, bool single_pass) {
@@ -50,15 +90,20 @@ Layout layout(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk, bool si
   off += align256(static_cast<size_t>(T) * kMaxSplits * 16);
   L.blocksums = off;
   off += align256(static_cast<size_t>(cdiv(T, ckl::COMBINE_THREADS)) * 8);
-  // dZ as 64-column panels: [ceil(V/64)][cap][64] bf16, cap = rows of the largest chunk.
+  // dZ as 64-column panels: [ceil(V/64)][cap][64] bf16, cap = rows of the
+  // largest chunk (a sliced block uses the same bytes as [Sv/64][Cr][64]).
   L.npanels = cdiv(V, 64);
   L.cap = std::min(chunk, std::max<int64_t>(T, 1));
   L.dz = off;
   off += align256(static_cast<size_t>(L.npanels) * L.cap * 64 * 2);
   // H_c^T for the dW GEMM: [d][pitch_t] bf16.
-  L.pitch_t = cdiv(L.cap, 8) * 8;
+  L.cr_alloc = sliced_rows(T, V, L.cap);
+  L.pitch_t = cdiv(std::max(L.cap, L.cr_alloc), 8) * 8;
   L.hct = off;
   off += align256(static_cast<size_t>(d) * L.pitch_t * 2);
+  // fp32 dH of a sliced row chunk, summed over its vocabulary slabs.
+  L.dh32 = off;
+  off += align256(static_cast<size_t>(L.cr_alloc) * d * 4);
   L.zpitch = cdiv(V, 4) * 4;
   if (single_pass) {
     L.z = off;
@@ -329,49 +374,136 @@ void fill_common(TcParams& p, uint8_t* w8, const Layout& L, int64_t T, int64_t d
   p.countN = &hdr->countN;
 }
 
-// The dH rows of one chunk and its share of dW, from the chunk's dZ panels:
-// H_c^T (the K-major B operand of the dW GEMM), then one merged GEMM launch.
-int dhdw_chunk(const uint16_t* H, const uint16_t* W, const uint8_t* mask, int64_t T, int64_t d,
-               int64_t V, int32_t K, int64_t c0, int64_t rows, const float* grad_loss,
-               uint16_t* dH, float* dW, int32_t accumulate_dW, uint8_t* w8, const Layout& L,
-               const DevInfo& di, cudaStream_t st, ckl_trace* trace) {
-  const uint16_t* Hc = H + c0 * d;
-  void* dz = w8 + L.dz;
-  void* hct = w8 + L.hct;
-  const int bn = pick_bn(d);
-  {
-    TraceScope ts(trace, st, CKL_KERNEL_OTHER);
-    const dim3 grid(static_cast<unsigned>(cdiv(d, 32)), static_cast<unsigned>(cdiv(rows, 32)));
-    ckl::transpose_rows_kernel<<<grid, 256, 0, st>>>(Hc, static_cast<int>(rows),
-                                                     static_cast<int>(d),
-                                                     static_cast<uint16_t*>(hct),
-                                                     static_cast<int>(L.pitch_t));
-    if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
-  }
+// H_c^T for rows [r0, r0 + rows): the K-major B operand of the dW GEMM.
+int transpose_rows(const uint16_t* H, int64_t d, int64_t r0, int64_t rows, uint8_t* w8,
+                   const Layout& L, cudaStream_t st, ckl_trace* trace) {
+  TraceScope ts(trace, st, CKL_KERNEL_OTHER);
+  const dim3 grid(static_cast<unsigned>(cdiv(d, 32)), static_cast<unsigned>(cdiv(rows, 32)));
+  ckl::transpose_rows_kernel<<<grid, 256, 0, st>>>(H + r0 * d, static_cast<int>(rows),
+                                                   static_cast<int>(d),
+                                                   reinterpret_cast<uint16_t*>(w8 + L.hct),
+                                                   static_cast<int>(L.pitch_t));
+  return cudaGetLastError() == cudaSuccess ? CKL_OK : CKL_ERR_CUDA;
+}
+
+// dZ of one block: rows [r0, r0 + rows) x vocabulary columns [v_lo, v_lo + cols)
+// (v_lo a multiple of 256), recomputed from H and W, into panels
+// [ceil(cols/64)][prow][64] at the start of the dZ buffer.
+int dz_block(const uint16_t* H, const uint16_t* W, const uint8_t* mask, const float* lse,
+             int64_t T, int64_t d, int64_t V, int32_t K, int64_t r0, int64_t rows, int64_t prow,
+             int64_t v_lo, int64_t cols, uint8_t* w8, const Layout& L, const DevInfo& di,
+             cudaStream_t st, ckl_trace* trace) {
   TcParams p;
   std::memset(&p, 0, sizeof(p));
   fill_common(p, w8, L, T, d, V, K, mask);
   p.rows = static_cast<int32_t>(rows);
-  p.row0 = static_cast<int32_t>(c0);
+  p.row0 = static_cast<int32_t>(r0);
+  p.n_rb = static_cast<int32_t>(cdiv(rows, kMB));
+  p.vt0 = static_cast<int32_t>(v_lo / ckl::BN_V);
+  p.n_vt = static_cast<int32_t>(cdiv(cols, ckl::BN_V));
+  p.S = 1;
+  p.n_units = p.n_rb * p.n_vt;  // tiles, dealt out in contiguous ranges
+  p.lse = lse;
+  if (!map2d(&p.tm[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, H + r0 * d, d, rows, d * 2, ckl::BK,
+             ckl::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map2d(&p.tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, V, d * 2, ckl::BK,
+             ckl::BN_V / kSlotCTAs, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map3d(&p.tm[2], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w8 + L.dz, 64, rows, cdiv(cols, 64), 128,
+             prow * 128, 32, ckl::BM, CU_TENSOR_MAP_SWIZZLE_64B))
+    return CKL_ERR_CUDA;
+  TraceScope ts(trace, st, CKL_KERNEL_BWD_DZ);
+  return launch_tc<ckl::MODE_DZ>(p, p.n_units, di, st);
+}
+
+// Quotas of dW tiles for the round-dealt schedule (dw_mode 1): slots below
+// r5 = n5 mod G hold one more dH unit (c5 k-blocks later to start).  Water-
+// filling: the smallest finishing k-block t whose per-class quotas
+// floor((t - start) / (c6 + 1)) cover n6 tiles, then the excess trimmed from
+// the class that finishes later.  Class quota Q for its first E slots and
+// Q - 1 for the rest.
+void dw_round_quotas(TcParams& p, int64_t G) {
+  const int64_t c = p.c6 + 1;
+  const int64_t a5 = p.n5 / G, r5 = p.n5 % G;
+  const int64_t s_l = a5 * p.c5, s_h = s_l + p.c5;
+  const int64_t nl = G - r5, nh = r5;
+  auto tot = [&](int64_t t, int64_t& ql, int64_t& qh) {
+    ql = t > s_l ? (t - s_l) / c : 0;
+    qh = t > s_h ? (t - s_h) / c : 0;
+    return nl * ql + nh * qh;
+  };
+  int64_t lo = 0, hi = s_h + (static_cast<int64_t>(p.n6) + 1) * c, ql = 0, qh = 0;
+  while (lo < hi) {
+    const int64_t mid = (lo + hi) / 2;
+    if (tot(mid, ql, qh) >= p.n6) hi = mid;
+    else lo = mid + 1;
+  }
+  int64_t ex = tot(lo, ql, qh) - p.n6;
+  int64_t El = nl, Eh = nh;
+  while (ex > 0) {
+    const int64_t end_l = (ql > 0 && El > 0) ? s_l + ql * c : -1;
+    const int64_t end_h = (qh > 0 && Eh > 0) ? s_h + qh * c : -1;
+    if (end_l >= end_h) {
+      const int64_t take = std::min(ex, El);
+      El -= take;
+      ex -= take;
+      if (El == 0 && ql > 0) { --ql; El = nl; }
+    } else {
+      const int64_t take = std::min(ex, Eh);
+      Eh -= take;
+      ex -= take;
+      if (Eh == 0 && qh > 0) { --qh; Eh = nh; }
+    }
+  }
+  p.dw_Ql = static_cast<int32_t>(ql);
+  p.dw_El = static_cast<int32_t>(El);
+  p.dw_Qh = static_cast<int32_t>(qh);
+  p.dw_Eh = static_cast<int32_t>(Eh);
+}
+
+// dH and dW of one block from its dZ panels (and H_c^T of its rows), one
+// merged GEMM launch.  dh_mode 0 writes dH rows as bf16 (dh_out = dH + r0 d);
+// 1 stores and 2 adds the block's fp32 share into dh_out (the partial dH of
+// a sliced row chunk).  dw_store 1 stores the block's dW rows, 0 adds.
+int dhdw_block(const uint16_t* W, const uint8_t* mask, int64_t T, int64_t d, int64_t V,
+               int32_t K, int64_t r0, int64_t rows, int64_t prow, int64_t v_lo, int64_t cols,
+               int dh_mode, int dw_store, const float* grad_loss, void* dh_out, float* dW,
+               uint8_t* w8, const Layout& L, const DevInfo& di, cudaStream_t st,
+               ckl_trace* trace) {
+  void* dz = w8 + L.dz;
+  const int bn = pick_bn(d);
+  const int64_t npan = cdiv(cols, 64);
+  TcParams p;
+  std::memset(&p, 0, sizeof(p));
+  fill_common(p, w8, L, T, d, V, K, mask);
+  p.rows = static_cast<int32_t>(rows);
+  p.row0 = static_cast<int32_t>(r0);
   p.bn = bn;
   p.n_nt = static_cast<int32_t>(cdiv(d, bn));
-  p.n_mt = static_cast<int32_t>(cdiv(V, kMB));
+  p.n_mt = static_cast<int32_t>(cdiv(cols, kMB));
   p.n5 = static_cast<int32_t>(cdiv(rows, kMB)) * p.n_nt;
   p.n6 = p.n_mt * p.n_nt;
-  p.c5 = static_cast<int32_t>(cdiv(V, ckl::BK));
+  p.c5 = static_cast<int32_t>(npan);
   p.c6 = static_cast<int32_t>(cdiv(rows, ckl::BK));
-  p.dw_store = (c0 == 0 && !accumulate_dW) ? 1 : 0;
+  p.dw_store = dw_store;
+  p.v_lo = static_cast<int32_t>(v_lo);
+  p.dh_mode = dh_mode;
   p.grad_loss = grad_loss;
-  uint16_t* dHc = dH + c0 * d;
-  if (!map3d(&p.tm[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dz, 64, rows, L.npanels, 128,
-             L.cap * 128, ckl::BK, ckl::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+  // dW tiles: contiguous per slot while every slot's dZ panels (kMB x rows
+  // bf16 per vocabulary block) fit in L2 together, else dealt in rounds
+  const int64_t G = std::min<int64_t>(di.slots[ckl::MODE_DHDW], p.n5 + p.n6);
+  p.dw_mode = (kMB * rows * 2 * G > (int64_t(48) << 20)) ? 1 : 0;
+  if (p.dw_mode == 1) dw_round_quotas(p, G);
+  const bool dh_bf16 = (dh_mode == 0);
+  if (!map3d(&p.tm[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dz, 64, rows, npan, 128, prow * 128,
+             ckl::BK, ckl::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !map2d(&p.tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, V, d * 2, 64, ckl::BK,
              CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !map3d2(&p.tm[2], dz, 64, rows, L.npanels, 128, L.cap * 128, 64, ckl::BK, 2) ||
-      !map2d(&p.tm[3], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hct, rows, d, L.pitch_t * 2, ckl::BK,
-             bn / kSlotCTAs, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !map2d(&p.tm[4], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dHc, d, rows, d * 2, 32, ckl::BM,
-             CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !map3d2(&p.tm[2], dz, 64, rows, npan, 128, prow * 128, 64, ckl::BK, 2) ||
+      !map2d(&p.tm[3], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w8 + L.hct, rows, d, L.pitch_t * 2,
+             ckl::BK, bn / kSlotCTAs, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map2d(&p.tm[4], dh_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+             dh_out, d, rows, d * (dh_bf16 ? 2 : 4), 32, ckl::BM,
+             dh_bf16 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B) ||
       !map2d(&p.tm[5], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, dW, d, V, d * 4, 32, ckl::BM,
              CU_TENSOR_MAP_SWIZZLE_128B))
     return CKL_ERR_CUDA;
@@ -457,36 +589,46 @@ int ckl_backward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
     return CKL_OK;
   }
   uint8_t* w8 = static_cast<uint8_t*>(workspace);
-  void* dz = w8 + L.dz;
-
-  for (int64_t c0 = 0; c0 < T; c0 += chunk) {
-    const int64_t rows = std::min<int64_t>(chunk, T - c0);
-    const uint16_t* Hc = H + c0 * d;
-    // ---- dZ for this chunk
-    {
-      TcParams p;
-      std::memset(&p, 0, sizeof(p));
-      fill_common(p, w8, L, T, d, V, K, mask);
-      p.rows = static_cast<int32_t>(rows);
-      p.row0 = static_cast<int32_t>(c0);
-      p.n_rb = static_cast<int32_t>(cdiv(rows, kMB));
-      p.S = choose_splits(p.n_rb, p.n_vt, di.slots[ckl::MODE_DZ]);
-      p.n_units = p.n_rb * p.S;
-      p.lse = lse;
-      if (!map2d(&p.tm[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Hc, d, rows, d * 2, ckl::BK,
-                 ckl::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-          !map2d(&p.tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, V, d * 2, ckl::BK,
-                 ckl::BN_V / kSlotCTAs, CU_TENSOR_MAP_SWIZZLE_128B) ||
-          !map3d(&p.tm[2], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dz, 64, rows, L.npanels, 128,
-                 L.cap * 128, 32, ckl::BM, CU_TENSOR_MAP_SWIZZLE_64B))
-        return CKL_ERR_CUDA;
-      TraceScope ts(trace, st, CKL_KERNEL_BWD_DZ);
-      if (launch_tc<ckl::MODE_DZ>(p, p.n_units, di, st) != CKL_OK) return CKL_ERR_CUDA;
-    }
-    rc = dhdw_chunk(H, W, mask, T, d, V, K, c0, rows, grad_loss, dH, dW, accumulate_dW, w8, L,
-                    di, st, trace);
+  const Plan P = plan_backward(T, d, V, L);
+  float* dh32 = reinterpret_cast<float*>(w8 + L.dh32);
+  for (int64_t r0 = 0; r0 < T; r0 += P.Cr) {
+    const int64_t rows = std::min(P.Cr, T - r0);
+    rc = transpose_rows(H, d, r0, rows, w8, L, st, trace);
     if (rc != CKL_OK) return rc;
+    const int dw_store = (r0 == 0 && !accumulate_dW) ? 1 : 0;
+    for (int64_t s = 0; s < P.n; ++s) {
+      const int64_t v_lo = s * P.Sv;
+      const int64_t cols = std::min(P.Sv, V - v_lo);
+      rc = dz_block(H, W, mask, lse, T, d, V, K, r0, rows, P.Cr, v_lo, cols, w8, L, di, st,
+                    trace);
+      if (rc != CKL_OK) return rc;
+      const int dh_mode = (P.n == 1) ? 0 : (s == 0 ? 1 : 2);
+      void* dh_out = (P.n == 1) ? static_cast<void*>(dH + r0 * d) : static_cast<void*>(dh32);
+      rc = dhdw_block(W, mask, T, d, V, K, r0, rows, P.Cr, v_lo, cols, dh_mode, dw_store,
+                      grad_loss, dh_out, dW, w8, L, di, st, trace);
+      if (rc != CKL_OK) return rc;
+    }
+    if (P.n > 1) {
+      // dH rows of this chunk: the fp32 sum over its slabs, rounded once
+      TraceScope ts(trace, st, CKL_KERNEL_OTHER);
+      const int64_t n4 = rows * d / 4;
+      const unsigned grid = static_cast<unsigned>(std::min<int64_t>(cdiv(n4, 256), 4 * di.sms));
+      ckl::dh_convert_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float4*>(dh32), n4,
+                                                   reinterpret_cast<uint2*>(dH + r0 * d));
+      if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
+    }
   }
+  return CKL_OK;
+}
+
+int ckl_backward_plan(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk,
+                      int64_t* plan) {
+  if (!plan || !sizes_ok(T, d, V, K, chunk)) return CKL_ERR_INVALID_ARG;
+  const Layout L = layout(T, d, V, K, chunk, false);
+  const Plan P = plan_backward(T, d, V, L);
+  plan[0] = P.Cr;
+  plan[1] = P.Sv;
+  plan[2] = P.n;
   return CKL_OK;
 }
 
@@ -556,8 +698,11 @@ int ckl_forward_backward(const uint16_t* H, const uint16_t* W, const int32_t* to
           rowloss, reinterpret_cast<uint16_t*>(w8 + L.dz));
       if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
     }
-    rc = dhdw_chunk(H, W, mask, T, d, V, K, c0, rows, grad_loss, dH, dW, accumulate_dW, w8, L,
-                    di, st, trace);
+    rc = transpose_rows(H, d, c0, rows, w8, L, st, trace);
+    if (rc != CKL_OK) return rc;
+    rc = dhdw_block(W, mask, T, d, V, K, c0, rows, L.cap, 0, V, 0,
+                    (c0 == 0 && !accumulate_dW) ? 1 : 0, grad_loss, dH + c0 * d, dW, w8, L, di,
+                    st, trace);
     if (rc != CKL_OK) return rc;
   }
   {

@@ -83,13 +83,18 @@ struct alignas(64) TcParams {
   int32_t n_rb;     // row blocks of 128 (FWD: over T; DZ / DHDW: over the chunk)
   int32_t n_vt;     // vocabulary tiles of 256
   int32_t S;        // vocabulary splits (FWD / DZ)
-  int32_t n_units;  // FWD / DZ: n_rb * S
+  int32_t n_units;  // FWD: n_rb * S units; DZ: n_rb * n_vt tiles
   int32_t bn;       // DHDW: d-tile width (64, 128, 192 or 256)
   int32_t n_nt;     // DHDW: d tiles
   int32_t n_mt;     // DHDW: vocabulary tiles of 128 (dW rows)
   int32_t n5, n6;   // DHDW: dH units, dW units
   int32_t c5, c6;   // DHDW: k-blocks per dH unit (over V), per dW unit (over rows)
-  int32_t dw_store; // DHDW: 1 = this chunk stores dW, 0 = adds into it
+  int32_t dw_store; // DHDW: 1 = this block stores dW, 0 = adds into it
+  int32_t vt0;      // FWD / DZ: first vocabulary tile of this launch's slab
+  int32_t v_lo;     // DHDW: first vocabulary column of this launch's slab
+  int32_t dh_mode;  // DHDW: 0 = dH as bf16, 1 = store fp32 partial dH, 2 = add into it
+  int32_t dw_mode;  // DHDW: 0 = contiguous dW ranges per slot, 1 = dW tiles dealt in rounds
+  int32_t dw_Ql, dw_El, dw_Qh, dw_Eh;  // DHDW rounds: quotas, see JobIter
   const int2* pairs;      // [T, K] (id, p as bits), sorted by id per row
   float4* partials;       // FWD: [T, S] (max of z log2e, sum 2^(..), sum p z, 0)
   const float* lse;       // DZ: [T]
@@ -339,6 +344,16 @@ zrow_kernel(const float* __restrict__ Z, int64_t zpitch, const float4* __restric
   }
 }
 
+// dH (bf16, round to nearest even) from the fp32 sum of its vocabulary slabs.
+__global__ void __launch_bounds__(256)
+dh_convert_kernel(const float4* __restrict__ src, int64_t n4, uint2* __restrict__ dst) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4 v = src[i];
+    dst[i] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+  }
+}
+
 // loss = (sum of the rows' terms, in a fixed order, in fp64) / N.
 constexpr int ROWSUM_THREADS = 1024;
 
@@ -361,8 +376,9 @@ rowsum_loss_kernel(const float* __restrict__ rowloss, int64_t T, const int* coun
 
 // ------------------------------------------------------------------ tc GEMM
 
-// dW units of this CTA: a contiguous range sized so that every CTA's total
-// k-block count (its round-robin dH units plus its dW units) is near equal.
+// dW units of this slot when each slot takes a contiguous range: sized so
+// that every slot's total k-block count (its round-robin dH units plus its
+// dW units) is near equal.
 __device__ __forceinline__ void dw_range(const TcParams& p, int cta, int G, int& b, int& e) {
   const int64_t c6e = p.c6 + 1;  // +1: the dW epilogue is not free
   const int64_t total = static_cast<int64_t>(p.n5) * p.c5 + static_cast<int64_t>(p.n6) * c6e;
@@ -389,11 +405,50 @@ __device__ __forceinline__ void dw_range(const TcParams& p, int cta, int G, int&
 // accumulator tile: FWD / DZ: (unit, vocabulary tile); DHDW: one unit.
 struct JobIter {
   int mode, G, cta;  // G scheduling slots (CTAs, or CTA pairs); this slot
-  // FWD / DZ
+  // FWD: unit u = (row block u % n_rb, split u / n_rb) over tiles [vt, vt_hi).
+  // DZ: tiles dealt round-robin in vocabulary-major order (tile lin = vt n_rb
+  // + rb), so that the slots work on neighbouring tiles at any time and share
+  // their W tile and H rows in L2; u = the tile's row block.
+  // DHDW: dH units round-robin (u = row block x n_nt + d tile), then dW tiles
+  // (u = vocabulary block x n_nt + d tile), either as a contiguous range per
+  // slot (dw_mode 0: a slot's consecutive tiles share their dZ panels) or
+  // dealt in rounds (dw_mode 1): in round k every slot whose quota exceeds k
+  // takes the next tile, so the tiles in flight are neighbours and share dZ
+  // panels and H_c^T in L2 when one slot's panels alone would not stay there.
+  // Round quotas come in two classes: the r5 = n5 mod G slots with one more
+  // dH unit hold Qh tiles (the first Eh of them) or Qh - 1, the others Ql
+  // (the first El of them) or Ql - 1; the tile index is then closed-form.
   int u, vt, vt_hi;
-  // DHDW
-  int phase;  // 0 = dH units, 1 = dW units, 2 = done
-  int b6, e6;
+  int lin;
+  int phase;  // DHDW: 0 = dH units, 1 = dW tiles, 2 = done
+  int k6, e6;
+  // tiles of a class (n slots, quota Q for the first E, Q - 1 for the rest)
+  // dealt in rounds before round k, and those of its first m slots in round k
+  __device__ static int cls_before(int k, int n, int Q, int E) {
+    if (Q < 1) return 0;
+    return (k < Q - 1 ? k : Q - 1) * n + (k > Q - 1 ? E : 0);
+  }
+  __device__ static int cls_rank(int k, int m, int Q, int E) {
+    if (Q < 1 || k > Q - 1) return 0;
+    return (k < Q - 1) ? m : (m < E ? m : E);
+  }
+  // DHDW: the next dW tile of this slot (k6 counts them), or phase 2
+  __device__ void dw_pick(const TcParams& p) {
+    if (p.dw_mode == 0) {
+      if (k6 >= e6) { phase = 2; return; }
+      u = k6;
+      return;
+    }
+    const int r5 = p.n5 % G;
+    const int nl = G - r5;
+    const bool heavy = cta < r5;
+    const int q = heavy ? p.dw_Qh - 1 + (cta < p.dw_Eh ? 1 : 0)
+                        : p.dw_Ql - 1 + (cta - r5 < p.dw_El ? 1 : 0);
+    if (k6 >= q) { phase = 2; return; }
+    u = cls_before(k6, r5, p.dw_Qh, p.dw_Eh) + cls_before(k6, nl, p.dw_Ql, p.dw_El) +
+        cls_rank(k6, cta < r5 ? cta : r5, p.dw_Qh, p.dw_Eh) +
+        (cta > r5 ? cls_rank(k6, cta - r5, p.dw_Ql, p.dw_El) : 0);
+  }
   __device__ void vt_range(const TcParams& p, int unit, int& lo, int& hi) const {
     const int s = unit / p.n_rb;
     lo = static_cast<int>(static_cast<int64_t>(s) * p.n_vt / p.S);
@@ -403,26 +458,35 @@ struct JobIter {
     mode = mode_;
     G = gridDim.x / per_slot;
     cta = blockIdx.x / per_slot;
-    if (mode != MODE_DHDW) {
+    if (mode == MODE_DZ) {
+      lin = cta;
+      u = lin % p.n_rb;
+      vt = lin / p.n_rb;
+      vt_hi = vt + 1;
+    } else if (mode != MODE_DHDW) {
       u = cta;
       vt = vt_hi = 0;
       if (u < p.n_units) vt_range(p, u, vt, vt_hi);
     } else {
-      dw_range(p, cta, G, b6, e6);
       u = cta;
       phase = 0;
       if (u >= p.n5) {
         phase = 1;
-        u = b6;
-        if (u >= e6) phase = 2;
+        dw_start(p);
       }
     }
   }
   __device__ bool valid(const TcParams& p) const {
+    if (mode == MODE_DZ) return lin < p.n_units;
     return (mode != MODE_DHDW) ? (u < p.n_units) : (phase < 2);
   }
   __device__ void next(const TcParams& p) {
-    if (mode != MODE_DHDW) {
+    if (mode == MODE_DZ) {
+      lin += G;
+      u = lin % p.n_rb;
+      vt = lin / p.n_rb;
+      vt_hi = vt + 1;
+    } else if (mode != MODE_DHDW) {
       if (++vt >= vt_hi) {
         u += G;
         if (u < p.n_units) vt_range(p, u, vt, vt_hi);
@@ -431,15 +495,25 @@ struct JobIter {
       u += G;
       if (u >= p.n5) {
         phase = 1;
-        u = b6;
-        if (u >= e6) phase = 2;
+        dw_start(p);
       }
     } else {
-      if (++u >= e6) phase = 2;
+      ++k6;
+      dw_pick(p);
     }
   }
-  // FWD / DZ: is this the first / last tile of its unit?
+  __device__ void dw_start(const TcParams& p) {
+    if (p.dw_mode == 0) {
+      dw_range(p, cta, G, k6, e6);
+    } else {
+      k6 = 0;
+    }
+    dw_pick(p);
+  }
+  // FWD / DZ: is this the first / last tile of its unit?  (DZ: every tile
+  // starts its row state afresh.)
   __device__ bool first_of_unit(const TcParams& p) const {
+    if (mode == MODE_DZ) return true;
     int lo, hi;
     vt_range(p, u, lo, hi);
     return vt == lo;
@@ -526,7 +600,7 @@ tc_kernel(const __grid_constant__ TcParams p) {
           const int rb = it.u % p.n_rb;
           nkb = (p.d + BK - 1) / BK;
           a_y = rb * MB + static_cast<int>(rank) * BM;
-          b_y = it.vt * BN_V + static_cast<int>(rank) * (BN_V / (PAIR ? 2 : 1));
+          b_y = (p.vt0 + it.vt) * BN_V + static_cast<int>(rank) * (BN_V / (PAIR ? 2 : 1));
         } else if (it.phase == 0) {
           kind = 5;
           nkb = p.c5;
@@ -566,11 +640,12 @@ tc_kernel(const __grid_constant__ TcParams p) {
             if (PAIR) {
               tma_load_3d_pair(sa, &p.tm[0], fb, 0, a_y, kb);
               for (int j = 0; j < half_n / 64; ++j)
-                tma_load_2d_pair(sb + j * ATOM_BYTES, &p.tm[1], fb, b_x + 64 * j, kb * BK);
+                tma_load_2d_pair(sb + j * ATOM_BYTES, &p.tm[1], fb, b_x + 64 * j,
+                                 p.v_lo + kb * BK);
             } else {
               tma_load_3d(sa, &p.tm[0], fb, 0, a_y, kb);
               for (int j = 0; j < half_n / 64; ++j)
-                tma_load_2d(sb + j * ATOM_BYTES, &p.tm[1], fb, b_x + 64 * j, kb * BK);
+                tma_load_2d(sb + j * ATOM_BYTES, &p.tm[1], fb, b_x + 64 * j, p.v_lo + kb * BK);
             }
           } else {
             // A = dZ^T: one box holding the two 64-column panels of this
@@ -688,7 +763,8 @@ tc_kernel(const __grid_constant__ TcParams p) {
       return __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
     };
     // Publish this warp's rows; the issuer stores the tile once all warps have
-    // (kind 0: dZ panel, 1: dH, 2: dW store, 3: dW add, 4: logits) and then frees the
+    // (kind 0: dZ panel, 1: dH, 2: dW store, 3: dW add, 4: logits, 5: fp32 dH
+    // store, 6: fp32 dH add) and then frees the
     // tile of the store before.
     auto stage_end = [&](int kind, int x, int y, int z) -> bool {
       fence_proxy_async_smem();
@@ -704,7 +780,9 @@ tc_kernel(const __grid_constant__ TcParams p) {
           else if (kind == 1) tma_store_2d(&p.tm[4], buf, x, y);
           else if (kind == 2) tma_store_2d(&p.tm[5], buf, x, y);
           else if (kind == 3) tma_reduce_add_2d(&p.tm[5], buf, x, y);
-          else tma_store_2d(&p.tm[2], buf, x, y);
+          else if (kind == 4) tma_store_2d(&p.tm[2], buf, x, y);
+          else if (kind == 5) tma_store_2d(&p.tm[4], buf, x, y);
+          else tma_reduce_add_2d(&p.tm[4], buf, x, y);
           bulk_commit();
           if (nstore >= 1) {
             bulk_wait_read<1>();
@@ -746,7 +824,7 @@ tc_kernel(const __grid_constant__ TcParams p) {
         const bool want_ids = (MODE == MODE_DZ) ? counts : row_ok;
         if (want_ids) {
           const int2* pr = p.pairs + t * p.K;
-          const int v_lo = it.vt * BN_V;
+          const int v_lo = (p.vt0 + it.vt) * BN_V;
           int lo = 0, hi = p.K;
           while (lo < hi) {
             const int mid = (lo + hi) >> 1;
@@ -763,7 +841,7 @@ tc_kernel(const __grid_constant__ TcParams p) {
       if (MODE == MODE_FWD || MODE == MODE_FWDZ) {
         const int zy0 = (it.u % p.n_rb) * MB + row0_cta;  // FWDZ: first chunk row of this CTA
         for (int c = 0; c < BN_V / 32; ++c) {
-          const int v0 = it.vt * BN_V + c * 32;
+          const int v0 = (p.vt0 + it.vt) * BN_V + c * 32;
           if (v0 >= p.V) break;
           float x[32];
           tmem_ld32(tacc + c * 32, x);
@@ -808,7 +886,7 @@ tc_kernel(const __grid_constant__ TcParams p) {
         const int y0 = rb * MB + row0_cta;  // first chunk row of this CTA's 128
         const int v_end = (p.V + 63) & ~63;  // dZ panels span round_up(V, 64) columns
         for (int c = 0; c < BN_V / 32; ++c) {
-          const int v0 = it.vt * BN_V + c * 32;
+          const int v0 = (p.vt0 + it.vt) * BN_V + c * 32;
           if (v0 >= v_end) break;
           float x[32];
           tmem_ld32(tacc + c * 32, x);
@@ -838,13 +916,16 @@ tc_kernel(const __grid_constant__ TcParams p) {
                          pack_bf16x2(x[8 * j + 2], x[8 * j + 3]),
                          pack_bf16x2(x[8 * j + 4], x[8 * j + 5]),
                          pack_bf16x2(x[8 * j + 6], x[8 * j + 7]));
-          if (!stage_end(0, v0 & 63, y0, v0 >> 6)) { ok = false; break; }
+          // panel of this slab's buffer
+          if (!stage_end(0, v0 & 63, y0, (v0 - p.vt0 * BN_V) >> 6)) { ok = false; break; }
         }
       } else {
         // DHDW: scale and write one accumulator tile (this CTA's rows, all columns).
         const bool is_dh = (it.phase == 0);
         const int nt = it.u % p.n_nt;
-        const int y0 = (it.u / p.n_nt) * MB + row0_cta;
+        // dH: rows of the row chunk; dW: vocabulary rows (the slab starts at v_lo)
+        const int y0 = (it.u / p.n_nt) * MB + row0_cta + (is_dh ? 0 : p.v_lo);
+        const bool bf16_out = is_dh && p.dh_mode == 0;
         for (int c = 0; c < p.bn / 32; ++c) {
           const int x0 = nt * p.bn + c * 32;
           if (x0 >= p.d) break;
@@ -852,7 +933,7 @@ tc_kernel(const __grid_constant__ TcParams p) {
           tmem_ld32(tacc + c * 32, x);
           if (!stage_begin()) { ok = false; break; }
           const uint32_t buf = stage_base + (nstore & 1) * EPI_STAGE;
-          if (is_dh) {
+          if (bf16_out) {
             const uint32_t rowa = buf + srow * 64;
             const int sw = (lane >> 1) & 3;
 #pragma unroll
@@ -872,7 +953,9 @@ tc_kernel(const __grid_constant__ TcParams p) {
                            __float_as_uint(x[4 * j + 2] * scale),
                            __float_as_uint(x[4 * j + 3] * scale));
           }
-          if (!stage_end(is_dh ? 1 : (p.dw_store ? 2 : 3), x0, y0, 0)) { ok = false; break; }
+          const int kind = is_dh ? (p.dh_mode == 0 ? 1 : p.dh_mode == 1 ? 5 : 6)
+                                 : (p.dw_store ? 2 : 3);
+          if (!stage_end(kind, x0, y0, 0)) { ok = false; break; }
         }
       }
       tc_fence_before();

@@ -112,6 +112,22 @@ typedef struct ckl_trace {
 CKL_API size_t ckl_workspace_bytes(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk);
 
 /*
+ * The blocking ckl_backward uses for these sizes (host only, no device work):
+ * plan[0] = rows per row chunk (Cr), plan[1] = vocabulary columns per slab
+ * (Sv, a multiple of 256 when plan[2] > 1), plan[2] = slabs per row chunk.
+ * The pages' schedule is one chunk of rows x all V at a time (plan =
+ * {min(chunk, T), round_up(V, 64), 1}).  When the batch spans several chunks
+ * the library may instead take taller row chunks swept in vocabulary slabs,
+ * with Cr x Sv <= min(chunk, T) x round_up(V, 64) (the same dZ buffer): dW is
+ * then re-added once per tall row chunk instead of once per chunk, and a
+ * partial fp32 dH (Cr x d, in the workspace) is added once per slab; it is
+ * chosen when that moves fewer bytes.  Returns CKL_ERR_INVALID_ARG for sizes
+ * outside the supported range or a NULL plan.
+ */
+CKL_API int ckl_backward_plan(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk,
+                              int64_t* plan);
+
+/*
  * Forward: the mean KL over the positions that count, and lse for EVERY row
  * (masked rows too).
  *   H          [T, d] bf16  student hidden states

@@ -22,7 +22,8 @@ def ckl():
 
 
 def test_header_declares_the_entry_points():
-    assert _declared() == ["ckl_backward", "ckl_forward", "ckl_forward_backward",
+    assert _declared() == ["ckl_backward", "ckl_backward_plan", "ckl_forward",
+                           "ckl_forward_backward",
                            "ckl_forward_static_scratch", "ckl_read_device_status",
                            "ckl_single_pass_workspace_bytes", "ckl_status_string",
                            "ckl_topk_cache", "ckl_version", "ckl_workspace_bytes"]
@@ -62,6 +63,41 @@ def test_single_pass_workspace_adds_the_chunk_logits(ckl):
         extra = rows * ((V + 3) // 4 * 4) * 4 + T * 4  # fp32 logits + per-row loss terms
         assert extra <= sp - base <= extra + 512
     assert ckl.lib.ckl_single_pass_workspace_bytes(10, 60, 100, 4, 8) == 0
+
+
+def test_backward_plan_fits_the_dz_buffer_and_covers_V(ckl):
+    """The blocking of the backward: either the row-chunked schedule, or taller
+    row chunks x vocabulary slabs whose dZ block fits the same chunk x V
+    buffer, covering every column exactly once."""
+    import numpy as np
+    rng = np.random.default_rng(0)
+    shapes = [(256, 64, 1024, 16, 64), (8192, 3072, 128256, 100, 1024),
+              (32768, 4096, 128256, 100, 2048), (32768, 2880, 201088, 100, 2048),
+              (262144, 4096, 128256, 100, 4096), (300, 200, 1000, 16, 100), (64, 64, 300, 4, 64),
+              (1, 8, 1, 1, 1), (5000, 8, 70, 3, 7)]
+    for _ in range(300):
+        shapes.append((int(rng.integers(1, 70000)), 8 * int(rng.integers(1, 600)),
+                       int(rng.integers(1, 300000)), int(rng.integers(1, 257)),
+                       int(rng.integers(1, 9000))))
+    n_sliced = 0
+    for T, d, V, K, chunk in shapes:
+        Cr, Sv, n = ckl.backward_plan(T, d, V, K, chunk)
+        cap, Vp = min(chunk, T), -(-V // 64) * 64
+        if n == 1:
+            assert (Cr, Sv) == (cap, Vp), (T, d, V, K, chunk)
+            continue
+        n_sliced += 1
+        assert T > cap and cap < Cr <= T
+        assert Sv % 256 == 0 and Sv >= 256
+        assert -(-Vp // Sv) == n and (n - 1) * Sv < V
+        assert Cr * Sv <= cap * Vp, (T, d, V, K, chunk)
+        # the sliced schedule's extra buffers are in the workspace
+        ws = ckl.lib.ckl_workspace_bytes(T, d, V, K, chunk)
+        assert ws >= cap * Vp * 2 + Cr * d * 6
+    assert n_sliced > 50
+    # the pages' configs: the 8K head is swept in slabs over all of its rows
+    assert ckl.backward_plan(8192, 3072, 128256, 100, 1024) == (8192, 14336, 9)
+    assert ckl.backward_plan(1000, 64, 5000, 8, 1000) == (1000, 5056, 1)  # one chunk
 
 
 def test_workspace_rejects_bad_sizes(ckl):

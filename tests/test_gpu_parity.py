@@ -44,6 +44,16 @@ def test_many_row_blocks_and_vocab_tiles(gpu_lib):
     assert_parity(run_library(gpu_lib, c, chunk=512), _ref(c), "1000x3000x328")
 
 
+def test_sliced_backward_both_dw_schedules(gpu_lib):
+    # Taller row chunks swept in vocabulary slabs: the first row chunk (2048
+    # rows) deals its dW tiles in rounds, the second (1024 rows) gives each
+    # slot a contiguous range; dH is summed in fp32 over the slabs.
+    c = make_inputs(3072, 1024, 8192, 16, seed=17, w_std=0.05, mask=("bernoulli", 0.1))
+    Cr, Sv, n = gpu_lib.backward_plan(3072, 1024, 8192, 16, 512)
+    assert (Cr, n) == (2048, 4) and Cr * Sv <= 512 * 8192
+    assert_parity(run_library(gpu_lib, c, chunk=512), _ref(c), "sliced 3072x8192x1024")
+
+
 def test_lse_is_bitwise_identical_across_chunk_sizes(gpu_lib):
     c = make_inputs(300, 200, 1000, 16, seed=6, w_std=0.3)
     outs = [run_library(gpu_lib, c, chunk=ch) for ch in (64, 128, 300)]
