@@ -582,12 +582,12 @@ def compare(args):
         logp = torch.log_softmax(2.0 * torch.randn(T, K, generator=g, device=dev), dim=1)
         mask = torch.ones(T, dtype=torch.uint8, device=dev)
         row = {"T": T}
-        for name in ("dense", "forward_chunked", "fused_library"):
-            if name != "fused_library" and T > 65536:
+        for name in ("dense", "forward_chunked", "fused_library", "fused_single_pass"):
+            if not name.startswith("fused") and T > 65536:
                 row[name] = "not run (needs more than the 180 GB of one B200)"
                 continue
-            H = H0.detach().clone().requires_grad_(name != "fused_library")
-            W = W0.detach().clone().requires_grad_(name != "fused_library")
+            H = H0.detach().clone().requires_grad_(not name.startswith("fused"))
+            W = W0.detach().clone().requires_grad_(not name.startswith("fused"))
             torch.cuda.synchronize()
             torch.cuda.empty_cache()
             base = torch.cuda.memory_allocated(dev)
@@ -604,6 +604,10 @@ def compare(args):
                         dH, dW = ckl.backward(H, W, idx, logp, mask, lse, chunk=chunk,
                                               workspace=ws)
                         del ws, lse, dH, dW
+                    elif name == "fused_single_pass":
+                        loss, lse, dH, dW = ckl.forward_backward(H, W, idx, logp, mask,
+                                                                 chunk=chunk)
+                        del lse, dH, dW
                     else:
                         H.grad = None
                         W.grad = None

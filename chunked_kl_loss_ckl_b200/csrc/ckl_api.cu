@@ -48,11 +48,15 @@ struct Layout {
 
 // The rows of a sliced block: the Cr that balances the two fp32 accumulations'
 // traffic (dW re-added once per row chunk, partial dH once per slab) under
-// Cr x Sv = chunk x V, i.e. sqrt(chunk x V), rounded up to 256.
-int64_t sliced_rows(int64_t T, int64_t V, int64_t cap) {
+// Cr x Sv = chunk x V, i.e. sqrt(chunk x V), rounded up to 256; but no more
+// than keeps H_c^T (Cr x d bf16, which every round of dW tiles streams) within
+// 48 MiB of the 126 MB L2.
+int64_t sliced_rows(int64_t T, int64_t d, int64_t V, int64_t cap) {
   if (T <= cap) return 0;
   int64_t r = static_cast<int64_t>(std::ceil(std::sqrt(static_cast<double>(cap) * V)));
   r = cdiv(r, 256) * 256;
+  const int64_t r_l2 = (int64_t(48) << 20) / (2 * d) / 256 * 256;
+  r = std::min(r, r_l2);
   return r > cap ? r : 0;
 }
 
@@ -97,7 +101,7 @@ Layout layout(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk, bool si
   L.dz = off;
   off += align256(static_cast<size_t>(L.npanels) * L.cap * 64 * 2);
   // H_c^T for the dW GEMM: [d][pitch_t] bf16.
-  L.cr_alloc = sliced_rows(T, V, L.cap);
+  L.cr_alloc = sliced_rows(T, d, V, L.cap);
   L.pitch_t = cdiv(std::max(L.cap, L.cr_alloc), 8) * 8;
   L.hct = off;
   off += align256(static_cast<size_t>(d) * L.pitch_t * 2);
