@@ -44,6 +44,9 @@ def parse_args(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--dp-allreduce", action="store_true",
+                    help="also time the data-parallel step: loss and dW all-reduced over the "
+                         "ranks with NCCL, overlapped with the backward slab by slab")
     ap.add_argument("--no-single-pass", action="store_true",
                     help="skip timing the single-pass entry point (ckl_forward_backward)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -376,6 +379,40 @@ def bench_ours(args):
             raise SystemExit(f"device status {rc} ({word}) after the single-pass steps")
         del ws_sp
 
+    # ------------------------------------------------------------ data parallel
+    dp_line = None
+    if args.dp_allreduce:
+        import torch.distributed as dist
+        from chunked_kl_loss_ckl_b200.dp import dp_forward_backward
+        own_group = not dist.is_initialized()
+        if own_group:  # one rank: the collectives sum one term
+            import tempfile
+            store = tempfile.mkdtemp()
+            dist.init_process_group("nccl", init_method=f"file://{store}/s", rank=0,
+                                    world_size=1, device_id=dev)
+
+        def dp_step():
+            dp_forward_backward(H, W, idx, logp, mask, chunk=chunk, workspace=ws, dW=dW)
+
+        for _ in range(args.warmup):
+            dp_step()
+        torch.cuda.synchronize()
+        dist.barrier()
+        h0 = torch.cuda.Event(enable_timing=True)
+        h1 = torch.cuda.Event(enable_timing=True)
+        h0.record(stream)
+        for _ in range(args.steps):
+            dp_step()
+        h1.record(stream)
+        torch.cuda.synchronize()
+        ms_dp = max_over_ranks(h0.elapsed_time(h1) / args.steps, ws_n, dev)
+        dp_line = {"value": round(tokens / (ms_dp / 1e3), 1), "unit": "tokens/s",
+                   "ms_per_step": round(ms_dp, 4), "ranks": ws_n,
+                   "exchange": "all-reduce of (loss x N, N), then of dW per vocabulary slab "
+                               "as the backward finishes it (NCCL)"}
+        if own_group:
+            dist.destroy_process_group()
+
     # ------------------------------------------------------------ end to end
     e2e = None
     if not args.no_e2e:
@@ -446,7 +483,7 @@ def bench_ours(args):
         "peak_source": peak_src,
         "flop_convention": "8 d V per token (fwd logits, bwd recompute, dH, dW)",
         "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
-        "single_pass": single,
+        "single_pass": single, "dp_step": dp_line,
         "gpu_launches": gpu_launches, "clocks": clocks,
         "workspace_bytes": ws.numel(),
         "peak_mem_bytes": int(torch.cuda.max_memory_allocated(dev)),

@@ -23,6 +23,7 @@ __all__ = [
     "LIB_PATH", "CklError", "Trace", "KERNEL_NAMES", "lib", "workspace_bytes", "new_workspace",
     "forward", "backward", "read_device_status", "status_string", "chunked_kl_loss",
     "topk_cache", "single_pass_workspace_bytes", "forward_backward", "backward_plan",
+    "DW_READY_FN",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libckl.so")
@@ -49,12 +50,17 @@ class _Trace(ctypes.Structure):
                 ("kernel_id", ctypes.POINTER(ctypes.c_int32))]
 
 
+# void (*)(int64_t v_begin, int64_t v_end, void* user)
+DW_READY_FN = ctypes.CFUNCTYPE(None, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p)
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with "
                           "`python -m chunked_kl_loss_ckl_b200._build` (nvcc, sm_100a)")
     L = ctypes.CDLL(LIB_PATH)
-    for name in ("ckl_forward", "ckl_backward", "ckl_forward_backward", "ckl_topk_cache"):
+    for name in ("ckl_forward", "ckl_backward", "ckl_backward_ex", "ckl_forward_backward",
+                 "ckl_topk_cache"):
         if not hasattr(L, name):
             raise ImportError(f"{LIB_PATH} lacks {name}: it is older than its sources; rebuild "
                               "with `python -m chunked_kl_loss_ckl_b200._build --force`")
@@ -67,6 +73,9 @@ def _load() -> ctypes.CDLL:
     L.ckl_backward.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i64, vp, vp, vp, vp, i32,
                                vp, sz, vp, tr]
     L.ckl_backward.restype = ctypes.c_int
+    L.ckl_backward_ex.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i64, vp, vp, vp, vp, i32,
+                                  vp, sz, vp, tr, DW_READY_FN, vp]
+    L.ckl_backward_ex.restype = ctypes.c_int
     L.ckl_backward_plan.argtypes = [i64, i64, i64, i32, i64, ctypes.POINTER(i64)]
     L.ckl_backward_plan.restype = ctypes.c_int
     L.ckl_single_pass_workspace_bytes.argtypes = [i64, i64, i64, i32, i64]
@@ -188,8 +197,14 @@ def forward(H, W, idx, logp, mask=None, chunk: int = 1024, workspace=None, strea
 
 def backward(H, W, idx, logp, mask, lse, grad_loss=None, chunk: int = 1024, dW=None,
              accumulate_dW: bool = False, workspace=None, stream=None,
-             trace: Trace | None = None, out_dH=None):
-    """dH (bf16, like H) and dW (fp32) by chunked recomputation."""
+             trace: Trace | None = None, out_dH=None, on_dw_ready=None):
+    """dH (bf16, like H) and dW (fp32) by chunked recomputation.
+
+    ``on_dw_ready(v_begin, v_end)``, when given, is called during the call as
+    soon as the launches that last write dW rows [v_begin, v_end) have been
+    enqueued on the stream (ckl_backward_ex); work it orders after them on
+    the stream sees those rows final.
+    """
     T, d, V, K = _check_inputs(H, W, idx, logp, mask)
     if workspace is None:
         workspace = new_workspace(T, d, V, K, chunk, H.device)
@@ -199,12 +214,33 @@ def backward(H, W, idx, logp, mask, lse, grad_loss=None, chunk: int = 1024, dW=N
         accumulate_dW = False
     if grad_loss is not None and (grad_loss.dtype != torch.float32 or not grad_loss.is_cuda):
         raise TypeError("grad_loss must be a CUDA float32 tensor")
-    rc = lib.ckl_backward(_ptr(H), _ptr(W), _ptr(idx), _ptr(logp), _ptr(mask), T, d, V, K, chunk,
-                          _ptr(lse), _ptr(grad_loss), _ptr(dH), _ptr(dW), int(bool(accumulate_dW)),
-                          _ptr(workspace), workspace.numel(), _stream_handle(stream),
-                          _trace_ptr(trace))
+    if on_dw_ready is None:
+        rc = lib.ckl_backward(_ptr(H), _ptr(W), _ptr(idx), _ptr(logp), _ptr(mask), T, d, V, K,
+                              chunk, _ptr(lse), _ptr(grad_loss), _ptr(dH), _ptr(dW),
+                              int(bool(accumulate_dW)), _ptr(workspace), workspace.numel(),
+                              _stream_handle(stream), _trace_ptr(trace))
+        if rc != CKL_OK:
+            raise CklError(rc, "ckl_backward")
+        return dH, dW
+    errors = []
+
+    def _cb(v0, v1, _user):
+        if errors:
+            return
+        try:
+            on_dw_ready(int(v0), int(v1))
+        except BaseException as e:  # no exception may cross the C frames
+            errors.append(e)
+
+    cb = DW_READY_FN(_cb)
+    rc = lib.ckl_backward_ex(_ptr(H), _ptr(W), _ptr(idx), _ptr(logp), _ptr(mask), T, d, V, K,
+                             chunk, _ptr(lse), _ptr(grad_loss), _ptr(dH), _ptr(dW),
+                             int(bool(accumulate_dW)), _ptr(workspace), workspace.numel(),
+                             _stream_handle(stream), _trace_ptr(trace), cb, None)
+    if errors:
+        raise errors[0]
     if rc != CKL_OK:
-        raise CklError(rc, "ckl_backward")
+        raise CklError(rc, "ckl_backward_ex")
     return dH, dW
 
 

@@ -577,6 +577,17 @@ int ckl_backward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
                  int32_t K, int64_t chunk, const float* lse, const float* grad_loss,
                  uint16_t* dH, float* dW, int32_t accumulate_dW, void* workspace,
                  size_t workspace_bytes, void* stream, ckl_trace* trace) {
+  return ckl_backward_ex(H, W, topk_idx, topk_logp, mask, T, d, V, K, chunk, lse, grad_loss, dH,
+                         dW, accumulate_dW, workspace, workspace_bytes, stream, trace, nullptr,
+                         nullptr);
+}
+
+int ckl_backward_ex(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
+                    const float* topk_logp, const uint8_t* mask, int64_t T, int64_t d, int64_t V,
+                    int32_t K, int64_t chunk, const float* lse, const float* grad_loss,
+                    uint16_t* dH, float* dW, int32_t accumulate_dW, void* workspace,
+                    size_t workspace_bytes, void* stream, ckl_trace* trace,
+                    ckl_dw_ready_fn on_dw_ready, void* user) {
   if (!dW || !aligned16(dW)) return CKL_ERR_INVALID_ARG;
   if (T > 0 && (!lse || !aligned4(lse) || !dH || !aligned16(dH))) return CKL_ERR_INVALID_ARG;
   if (grad_loss && !aligned4(grad_loss)) return CKL_ERR_INVALID_ARG;
@@ -590,6 +601,7 @@ int ckl_backward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
     if (!accumulate_dW &&
         cudaMemsetAsync(dW, 0, static_cast<size_t>(V) * d * sizeof(float), st) != cudaSuccess)
       return CKL_ERR_CUDA;
+    if (on_dw_ready) on_dw_ready(0, V, user);
     return CKL_OK;
   }
   uint8_t* w8 = static_cast<uint8_t*>(workspace);
@@ -611,6 +623,8 @@ int ckl_backward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
       rc = dhdw_block(W, mask, T, d, V, K, r0, rows, P.Cr, v_lo, cols, dh_mode, dw_store,
                       grad_loss, dh_out, dW, w8, L, di, st, trace);
       if (rc != CKL_OK) return rc;
+      // the last row chunk's launch is the last to write these dW rows
+      if (on_dw_ready && r0 + rows == T) on_dw_ready(v_lo, v_lo + cols, user);
     }
     if (P.n > 1) {
       // dH rows of this chunk: the fp32 sum over its slabs, rounded once

@@ -201,6 +201,28 @@ CKL_API int ckl_forward_backward(const uint16_t* H, const uint16_t* W, const int
                                  size_t workspace_bytes, void* stream, ckl_trace* trace);
 
 /*
+ * ckl_backward with a host callback for overlapping the gradient exchange of
+ * data-parallel training (no counterpart in the pages, which run on one GPU).
+ * on_dw_ready(v_begin, v_end, user) is called on the calling host thread,
+ * in increasing v order, as soon as the launches that write dW rows
+ * [v_begin, v_end) for the last time have been ENQUEUED on `stream` (not
+ * completed): work the callback orders after them on `stream` (an event, a
+ * collective on a stream that waits for `stream`) sees those rows final while
+ * the rest of the backward keeps running.  The ranges partition [0, V):
+ * one per vocabulary slab when the backward is sliced (ckl_backward_plan),
+ * else one for all of V after the last chunk.  The callback must not call
+ * into this library.  on_dw_ready may be NULL (then this is ckl_backward).
+ */
+typedef void (*ckl_dw_ready_fn)(int64_t v_begin, int64_t v_end, void* user);
+CKL_API int ckl_backward_ex(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
+                            const float* topk_logp, const uint8_t* mask, int64_t T, int64_t d,
+                            int64_t V, int32_t K, int64_t chunk, const float* lse,
+                            const float* grad_loss, uint16_t* dH, float* dW,
+                            int32_t accumulate_dW, void* workspace, size_t workspace_bytes,
+                            void* stream, ckl_trace* trace, ckl_dw_ready_fn on_dw_ready,
+                            void* user);
+
+/*
  * Reads the device status word of the last call that used `workspace`:
  * synchronises `stream`, copies the word to *device_status (a host pointer)
  * and returns the matching ckl_status (CKL_OK when the word is 0).

@@ -22,7 +22,7 @@ def ckl():
 
 
 def test_header_declares_the_entry_points():
-    assert _declared() == ["ckl_backward", "ckl_backward_plan", "ckl_forward",
+    assert _declared() == ["ckl_backward", "ckl_backward_ex", "ckl_backward_plan", "ckl_forward",
                            "ckl_forward_backward",
                            "ckl_forward_static_scratch", "ckl_read_device_status",
                            "ckl_single_pass_workspace_bytes", "ckl_status_string",

@@ -71,3 +71,77 @@ def test_two_gloo_ranks(tmp_path):
     for x in r:
         assert abs(float(x["loss"]) - full["loss"]) < 1e-12 * full["loss"]
         np.testing.assert_allclose(x["dw"], full["dW"], rtol=1e-10, atol=1e-14)
+
+
+# ---------------------------------------------------------------- data parallel
+class _OracleOps:
+    """Stands in for the CUDA library on CPU: the oracle's dense forward and
+    backward of the rank's own rows, with the library's interface (fp32/bf16
+    outputs, dW written range by range with on_dw_ready after each range)."""
+
+    def __init__(self, c):
+        self.c = c
+
+    def forward(self, H, W, idx, logp, mask, chunk, workspace=None):
+        import oracle
+        c = self.c
+        r = oracle.dense(c["H"], c["W"], c["idx"], c["logp"], c["mask"], g=1.0)
+        return (torch.tensor([r["loss"]], dtype=torch.float32),
+                torch.from_numpy(r["lse"].astype(np.float32)))
+
+    def backward(self, H, W, idx, logp, mask, lse, grad_loss=None, chunk=1024, dW=None,
+                 workspace=None, on_dw_ready=None):
+        import oracle
+        c = self.c
+        g = 1.0 if grad_loss is None else float(grad_loss.item())
+        r = oracle.dense(c["H"], c["W"], c["idx"], c["logp"], c["mask"], g=g)
+        V = dW.shape[0]
+        for v0, v1 in ((0, V // 3), (V // 3, 2 * V // 3), (2 * V // 3, V)):
+            dW[v0:v1] = torch.from_numpy(r["dW"][v0:v1].astype(np.float32))
+            on_dw_ready(v0, v1)
+        return torch.from_numpy(r["dH"].astype(np.float32)), dW
+
+
+def _dp_worker(rank, world, port, out_dir):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        from chunked_kl_loss_ckl_b200.dp import dp_forward_backward
+        from ckl_synth import make_inputs
+        c = make_inputs(40, 16, 60, 5, seed=5, w_std=0.4, mask=("bernoulli", 0.2))
+        lo, hi = (0, 13) if rank == 0 else (13, 40)   # uneven shards
+        part = dict(c, H=c["H"][lo:hi], idx=c["idx"][lo:hi], logp=c["logp"][lo:hi],
+                    mask=c["mask"][lo:hi], T=hi - lo)
+        ops = _OracleOps(part)
+        Ht = torch.zeros(hi - lo, 16)
+        Wt = torch.zeros(60, 16)
+        g = torch.tensor([0.7], dtype=torch.float32)
+        mt = torch.from_numpy(np.ascontiguousarray(part["mask"], dtype=np.uint8))
+        loss, lse, dH, dW = dp_forward_backward(Ht, Wt, None, None, mask=mt, chunk=8,
+                                                grad_loss=g, ops=ops)
+        np.savez(os.path.join(out_dir, f"dp{rank}.npz"), loss=loss.numpy(), dH=dH.numpy(),
+                 dW=dW.numpy(), lo=lo, hi=hi)
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def test_data_parallel_step_two_gloo_ranks(tmp_path):
+    """dp_forward_backward on two ranks with uneven shards equals the
+    unsharded loss and gradients: the global mean, dH rows scaled by the
+    global N, dW summed over ranks range by range."""
+    world = 2
+    mp.spawn(_dp_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True)
+    r = [np.load(tmp_path / f"dp{i}.npz") for i in range(world)]
+    import oracle
+    from ckl_synth import make_inputs
+    c = make_inputs(40, 16, 60, 5, seed=5, w_std=0.4, mask=("bernoulli", 0.2))
+    full = oracle.dense(c["H"], c["W"], c["idx"], c["logp"], c["mask"], g=0.7)
+    for x in r:
+        assert abs(float(x["loss"][0]) - full["loss"]) <= 1e-6 * full["loss"]
+        np.testing.assert_allclose(x["dW"], full["dW"], rtol=1e-5, atol=1e-7)
+        lo, hi = int(x["lo"]), int(x["hi"])
+        np.testing.assert_allclose(x["dH"], full["dH"][lo:hi], rtol=1e-5, atol=1e-7)
