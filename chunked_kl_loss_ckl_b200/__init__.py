@@ -23,7 +23,7 @@ __all__ = [
     "LIB_PATH", "CklError", "Trace", "KERNEL_NAMES", "lib", "workspace_bytes", "new_workspace",
     "forward", "backward", "read_device_status", "status_string", "chunked_kl_loss",
     "topk_cache", "single_pass_workspace_bytes", "forward_backward", "backward_plan",
-    "DW_READY_FN",
+    "DW_READY_FN", "forward_f32", "backward_f32",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libckl.so")
@@ -78,6 +78,14 @@ def _load() -> ctypes.CDLL:
     L.ckl_backward_ex.restype = ctypes.c_int
     L.ckl_backward_plan.argtypes = [i64, i64, i64, i32, i64, ctypes.POINTER(i64)]
     L.ckl_backward_plan.restype = ctypes.c_int
+    L.ckl_workspace_bytes_f32.argtypes = [i64, i64, i64, i32, i64]
+    L.ckl_workspace_bytes_f32.restype = sz
+    L.ckl_forward_f32.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i64, vp, vp, vp, sz, vp,
+                                  tr]
+    L.ckl_forward_f32.restype = ctypes.c_int
+    L.ckl_backward_f32.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i64, vp, vp, vp, vp,
+                                   i32, vp, sz, vp, tr]
+    L.ckl_backward_f32.restype = ctypes.c_int
     L.ckl_single_pass_workspace_bytes.argtypes = [i64, i64, i64, i32, i64]
     L.ckl_single_pass_workspace_bytes.restype = sz
     L.ckl_forward_backward.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i64, vp, vp, vp, vp,
@@ -145,9 +153,12 @@ def _trace_ptr(trace):
     return None if trace is None else ctypes.byref(trace.c)
 
 
-def _check_inputs(H, W, idx, logp, mask):
-    for name, t, dts in (("H", H, (torch.bfloat16, torch.int16, torch.uint16)),
-                         ("W", W, (torch.bfloat16, torch.int16, torch.uint16)),
+_BF16 = (torch.bfloat16, torch.int16, torch.uint16)
+
+
+def _check_inputs(H, W, idx, logp, mask, dtype=None):
+    hw = _BF16 if dtype is None else (dtype,)
+    for name, t, dts in (("H", H, hw), ("W", W, hw),
                          ("topk_idx", idx, (torch.int32,)), ("topk_logp", logp, (torch.float32,))):
         if not t.is_cuda:
             raise ValueError(f"{name} must be a CUDA tensor")
@@ -251,6 +262,50 @@ def backward_plan(T: int, d: int, V: int, K: int, chunk: int):
     if rc != CKL_OK:
         raise CklError(rc, "ckl_backward_plan")
     return int(out[0]), int(out[1]), int(out[2])
+
+
+def forward_f32(H, W, idx, logp, mask=None, chunk: int = 1024, workspace=None, stream=None,
+                trace: Trace | None = None):
+    """ckl_forward on fp32 H and W (tf32 tensor-core products)."""
+    T, d, V, K = _check_inputs(H, W, idx, logp, mask, dtype=torch.float32)
+    if workspace is None:
+        n = lib.ckl_workspace_bytes_f32(T, d, V, K, chunk)
+        if n == 0:
+            raise CklError(1, "ckl_workspace_bytes_f32")
+        workspace = torch.empty(n, dtype=torch.uint8, device=H.device)
+    loss = torch.empty(1, dtype=torch.float32, device=H.device)
+    lse = torch.empty(T, dtype=torch.float32, device=H.device)
+    rc = lib.ckl_forward_f32(_ptr(H), _ptr(W), _ptr(idx), _ptr(logp), _ptr(mask), T, d, V, K,
+                             chunk, _ptr(loss), _ptr(lse), _ptr(workspace), workspace.numel(),
+                             _stream_handle(stream), _trace_ptr(trace))
+    if rc != CKL_OK:
+        raise CklError(rc, "ckl_forward_f32")
+    return loss, lse
+
+
+def backward_f32(H, W, idx, logp, mask, lse, grad_loss=None, chunk: int = 1024, dW=None,
+                 accumulate_dW: bool = False, workspace=None, stream=None,
+                 trace: Trace | None = None):
+    """ckl_backward on fp32 H and W: dH and dW in fp32."""
+    T, d, V, K = _check_inputs(H, W, idx, logp, mask, dtype=torch.float32)
+    if workspace is None:
+        n = lib.ckl_workspace_bytes_f32(T, d, V, K, chunk)
+        if n == 0:
+            raise CklError(1, "ckl_workspace_bytes_f32")
+        workspace = torch.empty(n, dtype=torch.uint8, device=H.device)
+    dH = torch.empty(T, d, dtype=torch.float32, device=H.device)
+    if dW is None:
+        dW = torch.empty(V, d, dtype=torch.float32, device=H.device)
+        accumulate_dW = False
+    if grad_loss is not None and (grad_loss.dtype != torch.float32 or not grad_loss.is_cuda):
+        raise TypeError("grad_loss must be a CUDA float32 tensor")
+    rc = lib.ckl_backward_f32(_ptr(H), _ptr(W), _ptr(idx), _ptr(logp), _ptr(mask), T, d, V, K,
+                              chunk, _ptr(lse), _ptr(grad_loss), _ptr(dH), _ptr(dW),
+                              int(bool(accumulate_dW)), _ptr(workspace), workspace.numel(),
+                              _stream_handle(stream), _trace_ptr(trace))
+    if rc != CKL_OK:
+        raise CklError(rc, "ckl_backward_f32")
+    return dH, dW
 
 
 def single_pass_workspace_bytes(T: int, d: int, V: int, K: int, chunk: int) -> int:

@@ -8,6 +8,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "../../include/ckl.h"
 #include "ckl_kernels.cuh"
@@ -44,18 +45,19 @@ struct Layout {
   int64_t cr_alloc; // rows the sliced schedule may hold (0 = never sliced)
   int64_t pitch_t;  // H_c^T row pitch (elements): max(cap, cr_alloc) rounded up to 8
   int64_t zpitch;   // single pass: fp32 logit row pitch (elements), V rounded up to 4
+  int eb;           // bytes per H / W / dZ element: 2 (bf16) or 4 (fp32, tf32 MMAs)
 };
 
 // The rows of a sliced block: the Cr that balances the two fp32 accumulations'
 // traffic (dW re-added once per row chunk, partial dH once per slab) under
 // Cr x Sv = chunk x V, i.e. sqrt(chunk x V), rounded up to 256; but no more
 // than keeps H_c^T (Cr x d bf16, which every round of dW tiles streams) within
-// 48 MiB of the 126 MB L2.
-int64_t sliced_rows(int64_t T, int64_t d, int64_t V, int64_t cap) {
+// 48 MiB of the 126 MB L2.  eb = bytes per element.
+int64_t sliced_rows(int64_t T, int64_t d, int64_t V, int64_t cap, int eb) {
   if (T <= cap) return 0;
   int64_t r = static_cast<int64_t>(std::ceil(std::sqrt(static_cast<double>(cap) * V)));
   r = cdiv(r, 256) * 256;
-  const int64_t r_l2 = (int64_t(48) << 20) / (2 * d) / 256 * 256;
+  const int64_t r_l2 = (int64_t(48) << 20) / (eb * d) / 256 * 256;
   r = std::min(r, r_l2);
   return r > cap ? r : 0;
 }
@@ -83,8 +85,12 @@ Plan plan_backward(int64_t T, int64_t d, int64_t V, const Layout& L) {
 }
 
 // single_pass adds the chunk's fp32 logits [cap][zpitch] and the rows' loss terms [T].
-Layout layout(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk, bool single_pass) {
+// eb = 4: the fp32 entry points (dZ and H_c^T in fp32; dH accumulates in the
+// caller's fp32 output, so no partial-dH buffer).
+Layout layout(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk, bool single_pass,
+              int eb = 2) {
   Layout L{};
+  L.eb = eb;
   size_t off = kHeaderBytes;
   L.pairs = off;
   off += align256(static_cast<size_t>(T) * K * 8);
@@ -99,15 +105,15 @@ Layout layout(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk, bool si
   L.npanels = cdiv(V, 64);
   L.cap = std::min(chunk, std::max<int64_t>(T, 1));
   L.dz = off;
-  off += align256(static_cast<size_t>(L.npanels) * L.cap * 64 * 2);
+  off += align256(static_cast<size_t>(L.npanels) * L.cap * 64 * eb);
   // H_c^T for the dW GEMM: [d][pitch_t] bf16.
-  L.cr_alloc = sliced_rows(T, d, V, L.cap);
+  L.cr_alloc = sliced_rows(T, d, V, L.cap, eb);
   L.pitch_t = cdiv(std::max(L.cap, L.cr_alloc), 8) * 8;
   L.hct = off;
-  off += align256(static_cast<size_t>(d) * L.pitch_t * 2);
+  off += align256(static_cast<size_t>(d) * L.pitch_t * eb);
   // fp32 dH of a sliced row chunk, summed over its vocabulary slabs.
   L.dh32 = off;
-  off += align256(static_cast<size_t>(L.cr_alloc) * d * 4);
+  if (eb == 2) off += align256(static_cast<size_t>(L.cr_alloc) * d * 4);
   L.zpitch = cdiv(V, 4) * 4;
   if (single_pass) {
     L.z = off;
@@ -177,17 +183,18 @@ bool map3d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// bf16 3-D map with a box of depth b2 along dim 2, 128-byte swizzle.
-bool map3d2(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t p1,
-            uint64_t p2, uint32_t b0, uint32_t b1, uint32_t b2) {
+// 3-D map with a box of depth b2 along dim 2 (128-byte swizzle by default).
+bool map3d2(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1,
+            uint64_t d2, uint64_t p1, uint64_t p2, uint32_t b0, uint32_t b1, uint32_t b2,
+            CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {d0, d1, d2};
   const cuuint64_t strides[2] = {p1, p2};
   const cuuint32_t box[3] = {b0, b1, b2};
   const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -203,6 +210,13 @@ struct DevInfo {
   bool attrs_set = false;
   int slots[4] = {0, 0, 0, 0};  // co-resident CTA pairs per GEMM mode
 };
+
+// Element type of a launch's operands: bf16 (kind::f16) or fp32 (kind::tf32).
+template <bool F32>
+constexpr CUtensorMapDataType kDT =
+    F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+template <bool F32>
+constexpr uint32_t kKE = F32 ? 32 : 64;  // K (and panel) elements per 128-byte row
 
 template <int MODE>
 cudaLaunchConfig_t tc_config(int slots, cudaStream_t st, cudaLaunchAttribute* attr) {
@@ -228,6 +242,13 @@ bool setup_mode(DevInfo& di) {
                            cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) !=
       cudaSuccess)
     return false;
+  // the fp32 form has the same shared memory and threads, so the same occupancy
+  if constexpr (MODE != ckl::MODE_FWDZ) {
+    if (cudaFuncSetAttribute(ckl::tc_kernel<MODE, kPair, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) !=
+        cudaSuccess)
+      return false;
+  }
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = tc_config<MODE>(di.sms / kSlotCTAs, nullptr, attr);
   int n = 0;
@@ -241,13 +262,14 @@ bool setup_mode(DevInfo& di) {
 }
 
 // Launches one persistent GEMM on min(co-resident slots, units) CTA pairs.
-template <int MODE>
+template <int MODE, bool F32 = false>
 int launch_tc(const TcParams& p, int64_t units, const DevInfo& di, cudaStream_t st) {
   const int slots = static_cast<int>(std::min<int64_t>(di.slots[MODE], units));
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = tc_config<MODE>(slots, st, attr);
-  return cudaLaunchKernelEx(&cfg, ckl::tc_kernel<MODE, kPair>, p) == cudaSuccess ? CKL_OK
-                                                                                 : CKL_ERR_CUDA;
+  return cudaLaunchKernelEx(&cfg, ckl::tc_kernel<MODE, kPair, F32>, p) == cudaSuccess
+             ? CKL_OK
+             : CKL_ERR_CUDA;
 }
 
 bool device_info(DevInfo& out) {
@@ -334,17 +356,17 @@ int status_from_word(int32_t w) {
 }
 
 // Shared front half of forward and backward: checks, header reset, prep.
-int common_prep(const uint16_t* H, const uint16_t* W, const int32_t* idx, const float* logp,
+int common_prep(const void* H, const void* W, const int32_t* idx, const float* logp,
                 const uint8_t* mask, int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk,
                 void* ws, size_t ws_bytes, cudaStream_t st, ckl_trace* trace, DevInfo& di,
-                Layout& L, bool single_pass = false) {
+                Layout& L, bool single_pass = false, int eb = 2) {
   if (!sizes_ok(T, d, V, K, chunk)) return CKL_ERR_INVALID_ARG;
   // H, topk_idx and topk_logp may be NULL only for an empty batch.
   if (!W || !ws || (T > 0 && (!H || !idx || !logp))) return CKL_ERR_INVALID_ARG;
   if (!aligned16(H) || !aligned16(W) || !aligned16(ws) || !aligned4(idx) || !aligned4(logp))
     return CKL_ERR_INVALID_ARG;
   if (K > ckl::PREP_MAXK) return CKL_ERR_UNSUPPORTED;
-  L = layout(T, d, V, K, chunk, single_pass);
+  L = layout(T, d, V, K, chunk, single_pass, eb);
   if (ws_bytes < L.total) return CKL_ERR_WORKSPACE;
   if (!device_info(di)) return CKL_ERR_CUDA;
   if (di.major != 10) return CKL_ERR_UNSUPPORTED;
@@ -379,24 +401,29 @@ void fill_common(TcParams& p, uint8_t* w8, const Layout& L, int64_t T, int64_t d
 }
 
 // H_c^T for rows [r0, r0 + rows): the K-major B operand of the dW GEMM.
-int transpose_rows(const uint16_t* H, int64_t d, int64_t r0, int64_t rows, uint8_t* w8,
+template <bool F32>
+int transpose_rows(const void* H, int64_t d, int64_t r0, int64_t rows, uint8_t* w8,
                    const Layout& L, cudaStream_t st, ckl_trace* trace) {
+  using E = std::conditional_t<F32, float, uint16_t>;
   TraceScope ts(trace, st, CKL_KERNEL_OTHER);
   const dim3 grid(static_cast<unsigned>(cdiv(d, 32)), static_cast<unsigned>(cdiv(rows, 32)));
-  ckl::transpose_rows_kernel<<<grid, 256, 0, st>>>(H + r0 * d, static_cast<int>(rows),
-                                                   static_cast<int>(d),
-                                                   reinterpret_cast<uint16_t*>(w8 + L.hct),
-                                                   static_cast<int>(L.pitch_t));
+  ckl::transpose_rows_kernel<E><<<grid, 256, 0, st>>>(
+      static_cast<const E*>(H) + r0 * d, static_cast<int>(rows), static_cast<int>(d),
+      reinterpret_cast<E*>(w8 + L.hct), static_cast<int>(L.pitch_t));
   return cudaGetLastError() == cudaSuccess ? CKL_OK : CKL_ERR_CUDA;
 }
 
 // dZ of one block: rows [r0, r0 + rows) x vocabulary columns [v_lo, v_lo + cols)
 // (v_lo a multiple of 256), recomputed from H and W, into panels
-// [ceil(cols/64)][prow][64] at the start of the dZ buffer.
-int dz_block(const uint16_t* H, const uint16_t* W, const uint8_t* mask, const float* lse,
-             int64_t T, int64_t d, int64_t V, int32_t K, int64_t r0, int64_t rows, int64_t prow,
+// [ceil(cols/PW)][prow][PW] at the start of the dZ buffer (PW = 64 bf16 or
+// 32 fp32 columns: 128 bytes).
+template <bool F32>
+int dz_block(const void* H, const void* W, const uint8_t* mask, const float* lse, int64_t T,
+             int64_t d, int64_t V, int32_t K, int64_t r0, int64_t rows, int64_t prow,
              int64_t v_lo, int64_t cols, uint8_t* w8, const Layout& L, const DevInfo& di,
              cudaStream_t st, ckl_trace* trace) {
+  constexpr int eb = F32 ? 4 : 2;
+  constexpr uint32_t PW = kKE<F32>;
   TcParams p;
   std::memset(&p, 0, sizeof(p));
   fill_common(p, w8, L, T, d, V, K, mask);
@@ -406,17 +433,18 @@ int dz_block(const uint16_t* H, const uint16_t* W, const uint8_t* mask, const fl
   p.vt0 = static_cast<int32_t>(v_lo / ckl::BN_V);
   p.n_vt = static_cast<int32_t>(cdiv(cols, ckl::BN_V));
   p.S = 1;
-  p.n_units = p.n_rb * p.n_vt;  // tiles, dealt out in contiguous ranges
+  p.n_units = p.n_rb * p.n_vt;  // tiles, dealt out round-robin
   p.lse = lse;
-  if (!map2d(&p.tm[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, H + r0 * d, d, rows, d * 2, ckl::BK,
-             ckl::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !map2d(&p.tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, V, d * 2, ckl::BK,
-             ckl::BN_V / kSlotCTAs, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !map3d(&p.tm[2], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w8 + L.dz, 64, rows, cdiv(cols, 64), 128,
-             prow * 128, 32, ckl::BM, CU_TENSOR_MAP_SWIZZLE_64B))
+  const uint8_t* Hr = static_cast<const uint8_t*>(H) + r0 * d * eb;
+  if (!map2d(&p.tm[0], kDT<F32>, Hr, d, rows, d * eb, kKE<F32>, ckl::BM,
+             CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map2d(&p.tm[1], kDT<F32>, W, d, V, d * eb, kKE<F32>, ckl::BN_V / kSlotCTAs,
+             CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map3d(&p.tm[2], kDT<F32>, w8 + L.dz, PW, rows, cdiv(cols, PW), 128, prow * 128, 32,
+             ckl::BM, F32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
     return CKL_ERR_CUDA;
   TraceScope ts(trace, st, CKL_KERNEL_BWD_DZ);
-  return launch_tc<ckl::MODE_DZ>(p, p.n_units, di, st);
+  return launch_tc<ckl::MODE_DZ, F32>(p, p.n_units, di, st);
 }
 
 // Quotas of dW tiles for the round-dealt schedule (dw_mode 1): slots below
@@ -467,15 +495,18 @@ void dw_round_quotas(TcParams& p, int64_t G) {
 // dH and dW of one block from its dZ panels (and H_c^T of its rows), one
 // merged GEMM launch.  dh_mode 0 writes dH rows as bf16 (dh_out = dH + r0 d);
 // 1 stores and 2 adds the block's fp32 share into dh_out (the partial dH of
-// a sliced row chunk).  dw_store 1 stores the block's dW rows, 0 adds.
-int dhdw_block(const uint16_t* W, const uint8_t* mask, int64_t T, int64_t d, int64_t V,
-               int32_t K, int64_t r0, int64_t rows, int64_t prow, int64_t v_lo, int64_t cols,
-               int dh_mode, int dw_store, const float* grad_loss, void* dh_out, float* dW,
-               uint8_t* w8, const Layout& L, const DevInfo& di, cudaStream_t st,
-               ckl_trace* trace) {
+// a sliced row chunk, or the fp32 entry points' dH rows).  dw_store 1 stores
+// the block's dW rows, 0 adds.
+template <bool F32>
+int dhdw_block(const void* W, const uint8_t* mask, int64_t T, int64_t d, int64_t V, int32_t K,
+               int64_t r0, int64_t rows, int64_t prow, int64_t v_lo, int64_t cols, int dh_mode,
+               int dw_store, const float* grad_loss, void* dh_out, float* dW, uint8_t* w8,
+               const Layout& L, const DevInfo& di, cudaStream_t st, ckl_trace* trace) {
+  constexpr int eb = F32 ? 4 : 2;
+  constexpr uint32_t KE = kKE<F32>;  // also the panel width
   void* dz = w8 + L.dz;
   const int bn = pick_bn(d);
-  const int64_t npan = cdiv(cols, 64);
+  const int64_t npan = cdiv(cols, KE);
   TcParams p;
   std::memset(&p, 0, sizeof(p));
   fill_common(p, w8, L, T, d, V, K, mask);
@@ -487,53 +518,51 @@ int dhdw_block(const uint16_t* W, const uint8_t* mask, int64_t T, int64_t d, int
   p.n5 = static_cast<int32_t>(cdiv(rows, kMB)) * p.n_nt;
   p.n6 = p.n_mt * p.n_nt;
   p.c5 = static_cast<int32_t>(npan);
-  p.c6 = static_cast<int32_t>(cdiv(rows, ckl::BK));
+  p.c6 = static_cast<int32_t>(cdiv(rows, KE));
   p.dw_store = dw_store;
   p.v_lo = static_cast<int32_t>(v_lo);
   p.dh_mode = dh_mode;
   p.grad_loss = grad_loss;
   // dW tiles: contiguous per slot while every slot's dZ panels (kMB x rows
-  // bf16 per vocabulary block) fit in L2 together, else dealt in rounds
+  // per vocabulary block) fit in L2 together, else dealt in rounds
   const int64_t G = std::min<int64_t>(di.slots[ckl::MODE_DHDW], p.n5 + p.n6);
-  p.dw_mode = (kMB * rows * 2 * G > (int64_t(48) << 20)) ? 1 : 0;
+  p.dw_mode = (kMB * rows * eb * G > (int64_t(48) << 20)) ? 1 : 0;
   if (p.dw_mode == 1) dw_round_quotas(p, G);
-  const bool dh_bf16 = (dh_mode == 0);
-  if (!map3d(&p.tm[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dz, 64, rows, npan, 128, prow * 128,
-             ckl::BK, ckl::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !map2d(&p.tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, V, d * 2, 64, ckl::BK,
+  const bool dh_low = (dh_mode == 0);  // bf16 dH
+  // the MN-major operands (W for dH, dZ^T for dW): tf32 ones take the 128-byte
+  // swizzle with 32-byte chunks, the only MN-major layout of kind::tf32
+  constexpr CUtensorMapSwizzle mn_sw =
+      F32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B;
+  if (!map3d(&p.tm[0], kDT<F32>, dz, KE, rows, npan, 128, prow * 128, KE, ckl::BM,
              CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !map3d2(&p.tm[2], dz, 64, rows, npan, 128, prow * 128, 64, ckl::BK, 2) ||
-      !map2d(&p.tm[3], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w8 + L.hct, rows, d, L.pitch_t * 2,
-             ckl::BK, bn / kSlotCTAs, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !map2d(&p.tm[4], dh_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-             dh_out, d, rows, d * (dh_bf16 ? 2 : 4), 32, ckl::BM,
-             dh_bf16 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map2d(&p.tm[1], kDT<F32>, W, d, V, d * eb, KE, KE, mn_sw) ||
+      !map3d2(&p.tm[2], kDT<F32>, dz, KE, rows, npan, 128, prow * 128, KE, KE,
+              static_cast<uint32_t>(ckl::BM / KE), mn_sw) ||
+      !map2d(&p.tm[3], kDT<F32>, w8 + L.hct, rows, d, L.pitch_t * eb, KE, bn / kSlotCTAs,
+             CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map2d(&p.tm[4], dh_low ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+             dh_out, d, rows, d * (dh_low ? 2 : 4), 32, ckl::BM,
+             dh_low ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B) ||
       !map2d(&p.tm[5], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, dW, d, V, d * 4, 32, ckl::BM,
              CU_TENSOR_MAP_SWIZZLE_128B))
     return CKL_ERR_CUDA;
   TraceScope ts(trace, st, CKL_KERNEL_BWD_DHDW);
-  return launch_tc<ckl::MODE_DHDW>(p, p.n5 + p.n6, di, st);
+  return launch_tc<ckl::MODE_DHDW, F32>(p, p.n5 + p.n6, di, st);
 }
 
-}  // namespace
-
-extern "C" {
-
-size_t ckl_workspace_bytes(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk) {
-  if (!sizes_ok(T, d, V, K, chunk)) return 0;
-  return layout(T, d, V, K, chunk, false).total;
-}
-
-int ckl_forward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
-                const float* topk_logp, const uint8_t* mask, int64_t T, int64_t d, int64_t V,
-                int32_t K, int64_t chunk, float* loss, float* lse, void* workspace,
-                size_t workspace_bytes, void* stream, ckl_trace* trace) {
+// The forward (S1-S4) on bf16 or fp32 H and W.
+template <bool F32>
+int forward_impl(const void* H, const void* W, const int32_t* topk_idx, const float* topk_logp,
+                 const uint8_t* mask, int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk,
+                 float* loss, float* lse, void* workspace, size_t workspace_bytes, void* stream,
+                 ckl_trace* trace) {
+  constexpr int eb = F32 ? 4 : 2;
   if (!loss || !aligned4(loss) || (T > 0 && (!lse || !aligned4(lse)))) return CKL_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   DevInfo di;
   Layout L;
   int rc = common_prep(H, W, topk_idx, topk_logp, mask, T, d, V, K, chunk, workspace,
-                       workspace_bytes, st, trace, di, L);
+                       workspace_bytes, st, trace, di, L, false, eb);
   if (rc != CKL_OK) return rc;
   uint8_t* w8 = static_cast<uint8_t*>(workspace);
   Header* hdr = reinterpret_cast<Header*>(w8);
@@ -551,14 +580,14 @@ int ckl_forward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
   p.n_rb = static_cast<int32_t>(cdiv(T, kMB));
   p.S = choose_splits(p.n_rb, p.n_vt, di.slots[ckl::MODE_FWD]);
   p.n_units = p.n_rb * p.S;
-  if (!map2d(&p.tm[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, H, d, T, d * 2, ckl::BK, ckl::BM,
+  if (!map2d(&p.tm[0], kDT<F32>, H, d, T, d * eb, kKE<F32>, ckl::BM,
              CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !map2d(&p.tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, V, d * 2, ckl::BK,
-             ckl::BN_V / kSlotCTAs, CU_TENSOR_MAP_SWIZZLE_128B))
+      !map2d(&p.tm[1], kDT<F32>, W, d, V, d * eb, kKE<F32>, ckl::BN_V / kSlotCTAs,
+             CU_TENSOR_MAP_SWIZZLE_128B))
     return CKL_ERR_CUDA;
   {
     TraceScope ts(trace, st, CKL_KERNEL_FWD_GEMM);
-    if (launch_tc<ckl::MODE_FWD>(p, p.n_units, di, st) != CKL_OK) return CKL_ERR_CUDA;
+    if (launch_tc<ckl::MODE_FWD, F32>(p, p.n_units, di, st) != CKL_OK) return CKL_ERR_CUDA;
   }
   {
     TraceScope ts(trace, st, CKL_KERNEL_FWD_COMBINE);
@@ -570,6 +599,94 @@ int ckl_forward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
     if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
   }
   return CKL_OK;
+}
+
+// The blocked backward (S0, S1, S5-S7) on bf16 or fp32 H and W; dH is bf16
+// or fp32 like H.
+template <bool F32>
+int backward_impl(const void* H, const void* W, const int32_t* topk_idx, const float* topk_logp,
+                  const uint8_t* mask, int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk,
+                  const float* lse, const float* grad_loss, void* dH, float* dW,
+                  int32_t accumulate_dW, void* workspace, size_t workspace_bytes, void* stream,
+                  ckl_trace* trace, ckl_dw_ready_fn on_dw_ready, void* user) {
+  constexpr int eb = F32 ? 4 : 2;
+  if (!dW || !aligned16(dW)) return CKL_ERR_INVALID_ARG;
+  if (T > 0 && (!lse || !aligned4(lse) || !dH || !aligned16(dH))) return CKL_ERR_INVALID_ARG;
+  if (grad_loss && !aligned4(grad_loss)) return CKL_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DevInfo di;
+  Layout L;
+  int rc = common_prep(H, W, topk_idx, topk_logp, mask, T, d, V, K, chunk, workspace,
+                       workspace_bytes, st, trace, di, L, false, eb);
+  if (rc != CKL_OK) return rc;
+  if (T == 0) {
+    if (!accumulate_dW &&
+        cudaMemsetAsync(dW, 0, static_cast<size_t>(V) * d * sizeof(float), st) != cudaSuccess)
+      return CKL_ERR_CUDA;
+    if (on_dw_ready) on_dw_ready(0, V, user);
+    return CKL_OK;
+  }
+  uint8_t* w8 = static_cast<uint8_t*>(workspace);
+  const Plan P = plan_backward(T, d, V, L);
+  float* dh32 = reinterpret_cast<float*>(w8 + L.dh32);
+  for (int64_t r0 = 0; r0 < T; r0 += P.Cr) {
+    const int64_t rows = std::min(P.Cr, T - r0);
+    rc = transpose_rows<F32>(H, d, r0, rows, w8, L, st, trace);
+    if (rc != CKL_OK) return rc;
+    const int dw_store = (r0 == 0 && !accumulate_dW) ? 1 : 0;
+    for (int64_t s = 0; s < P.n; ++s) {
+      const int64_t v_lo = s * P.Sv;
+      const int64_t cols = std::min(P.Sv, V - v_lo);
+      rc = dz_block<F32>(H, W, mask, lse, T, d, V, K, r0, rows, P.Cr, v_lo, cols, w8, L, di,
+                         st, trace);
+      if (rc != CKL_OK) return rc;
+      // bf16 dH: one slab writes it, several sum into the fp32 partial first;
+      // fp32 dH: the slabs store / add into the output itself
+      int dh_mode;
+      void* dh_out;
+      if (F32) {
+        dh_mode = (s == 0) ? 1 : 2;
+        dh_out = static_cast<uint8_t*>(dH) + r0 * d * 4;
+      } else {
+        dh_mode = (P.n == 1) ? 0 : (s == 0 ? 1 : 2);
+        dh_out = (P.n == 1) ? static_cast<void*>(static_cast<uint8_t*>(dH) + r0 * d * 2)
+                            : static_cast<void*>(dh32);
+      }
+      rc = dhdw_block<F32>(W, mask, T, d, V, K, r0, rows, P.Cr, v_lo, cols, dh_mode, dw_store,
+                           grad_loss, dh_out, dW, w8, L, di, st, trace);
+      if (rc != CKL_OK) return rc;
+      // the last row chunk's launch is the last to write these dW rows
+      if (on_dw_ready && r0 + rows == T) on_dw_ready(v_lo, v_lo + cols, user);
+    }
+    if (!F32 && P.n > 1) {
+      // dH rows of this chunk: the fp32 sum over its slabs, rounded once
+      TraceScope ts(trace, st, CKL_KERNEL_OTHER);
+      const int64_t n4 = rows * d / 4;
+      const unsigned grid = static_cast<unsigned>(std::min<int64_t>(cdiv(n4, 256), 4 * di.sms));
+      ckl::dh_convert_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float4*>(dh32), n4,
+                                                   reinterpret_cast<uint2*>(
+                                                       static_cast<uint8_t*>(dH) + r0 * d * 2));
+      if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
+    }
+  }
+  return CKL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ckl_workspace_bytes(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk) {
+  if (!sizes_ok(T, d, V, K, chunk)) return 0;
+  return layout(T, d, V, K, chunk, false).total;
+}
+
+int ckl_forward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
+                const float* topk_logp, const uint8_t* mask, int64_t T, int64_t d, int64_t V,
+                int32_t K, int64_t chunk, float* loss, float* lse, void* workspace,
+                size_t workspace_bytes, void* stream, ckl_trace* trace) {
+  return forward_impl<false>(H, W, topk_idx, topk_logp, mask, T, d, V, K, chunk, loss, lse,
+                             workspace, workspace_bytes, stream, trace);
 }
 
 int ckl_backward(const uint16_t* H, const uint16_t* W, const int32_t* topk_idx,
@@ -588,55 +705,32 @@ int ckl_backward_ex(const uint16_t* H, const uint16_t* W, const int32_t* topk_id
                     uint16_t* dH, float* dW, int32_t accumulate_dW, void* workspace,
                     size_t workspace_bytes, void* stream, ckl_trace* trace,
                     ckl_dw_ready_fn on_dw_ready, void* user) {
-  if (!dW || !aligned16(dW)) return CKL_ERR_INVALID_ARG;
-  if (T > 0 && (!lse || !aligned4(lse) || !dH || !aligned16(dH))) return CKL_ERR_INVALID_ARG;
-  if (grad_loss && !aligned4(grad_loss)) return CKL_ERR_INVALID_ARG;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  DevInfo di;
-  Layout L;
-  int rc = common_prep(H, W, topk_idx, topk_logp, mask, T, d, V, K, chunk, workspace,
-                       workspace_bytes, st, trace, di, L);
-  if (rc != CKL_OK) return rc;
-  if (T == 0) {
-    if (!accumulate_dW &&
-        cudaMemsetAsync(dW, 0, static_cast<size_t>(V) * d * sizeof(float), st) != cudaSuccess)
-      return CKL_ERR_CUDA;
-    if (on_dw_ready) on_dw_ready(0, V, user);
-    return CKL_OK;
-  }
-  uint8_t* w8 = static_cast<uint8_t*>(workspace);
-  const Plan P = plan_backward(T, d, V, L);
-  float* dh32 = reinterpret_cast<float*>(w8 + L.dh32);
-  for (int64_t r0 = 0; r0 < T; r0 += P.Cr) {
-    const int64_t rows = std::min(P.Cr, T - r0);
-    rc = transpose_rows(H, d, r0, rows, w8, L, st, trace);
-    if (rc != CKL_OK) return rc;
-    const int dw_store = (r0 == 0 && !accumulate_dW) ? 1 : 0;
-    for (int64_t s = 0; s < P.n; ++s) {
-      const int64_t v_lo = s * P.Sv;
-      const int64_t cols = std::min(P.Sv, V - v_lo);
-      rc = dz_block(H, W, mask, lse, T, d, V, K, r0, rows, P.Cr, v_lo, cols, w8, L, di, st,
-                    trace);
-      if (rc != CKL_OK) return rc;
-      const int dh_mode = (P.n == 1) ? 0 : (s == 0 ? 1 : 2);
-      void* dh_out = (P.n == 1) ? static_cast<void*>(dH + r0 * d) : static_cast<void*>(dh32);
-      rc = dhdw_block(W, mask, T, d, V, K, r0, rows, P.Cr, v_lo, cols, dh_mode, dw_store,
-                      grad_loss, dh_out, dW, w8, L, di, st, trace);
-      if (rc != CKL_OK) return rc;
-      // the last row chunk's launch is the last to write these dW rows
-      if (on_dw_ready && r0 + rows == T) on_dw_ready(v_lo, v_lo + cols, user);
-    }
-    if (P.n > 1) {
-      // dH rows of this chunk: the fp32 sum over its slabs, rounded once
-      TraceScope ts(trace, st, CKL_KERNEL_OTHER);
-      const int64_t n4 = rows * d / 4;
-      const unsigned grid = static_cast<unsigned>(std::min<int64_t>(cdiv(n4, 256), 4 * di.sms));
-      ckl::dh_convert_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float4*>(dh32), n4,
-                                                   reinterpret_cast<uint2*>(dH + r0 * d));
-      if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
-    }
-  }
-  return CKL_OK;
+  return backward_impl<false>(H, W, topk_idx, topk_logp, mask, T, d, V, K, chunk, lse, grad_loss,
+                              dH, dW, accumulate_dW, workspace, workspace_bytes, stream, trace,
+                              on_dw_ready, user);
+}
+
+size_t ckl_workspace_bytes_f32(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk) {
+  if (!sizes_ok(T, d, V, K, chunk)) return 0;
+  return layout(T, d, V, K, chunk, false, 4).total;
+}
+
+int ckl_forward_f32(const float* H, const float* W, const int32_t* topk_idx,
+                    const float* topk_logp, const uint8_t* mask, int64_t T, int64_t d, int64_t V,
+                    int32_t K, int64_t chunk, float* loss, float* lse, void* workspace,
+                    size_t workspace_bytes, void* stream, ckl_trace* trace) {
+  return forward_impl<true>(H, W, topk_idx, topk_logp, mask, T, d, V, K, chunk, loss, lse,
+                            workspace, workspace_bytes, stream, trace);
+}
+
+int ckl_backward_f32(const float* H, const float* W, const int32_t* topk_idx,
+                     const float* topk_logp, const uint8_t* mask, int64_t T, int64_t d,
+                     int64_t V, int32_t K, int64_t chunk, const float* lse,
+                     const float* grad_loss, float* dH, float* dW, int32_t accumulate_dW,
+                     void* workspace, size_t workspace_bytes, void* stream, ckl_trace* trace) {
+  return backward_impl<true>(H, W, topk_idx, topk_logp, mask, T, d, V, K, chunk, lse, grad_loss,
+                             dH, dW, accumulate_dW, workspace, workspace_bytes, stream, trace,
+                             nullptr, nullptr);
 }
 
 int ckl_backward_plan(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk,
@@ -716,9 +810,9 @@ int ckl_forward_backward(const uint16_t* H, const uint16_t* W, const int32_t* to
           rowloss, reinterpret_cast<uint16_t*>(w8 + L.dz));
       if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
     }
-    rc = transpose_rows(H, d, c0, rows, w8, L, st, trace);
+    rc = transpose_rows<false>(H, d, c0, rows, w8, L, st, trace);
     if (rc != CKL_OK) return rc;
-    rc = dhdw_block(W, mask, T, d, V, K, c0, rows, L.cap, 0, V, 0,
+    rc = dhdw_block<false>(W, mask, T, d, V, K, c0, rows, L.cap, 0, V, 0,
                     (c0 == 0 && !accumulate_dW) ? 1 : 0, grad_loss, dH + c0 * d, dW, w8, L, di,
                     st, trace);
     if (rc != CKL_OK) return rc;

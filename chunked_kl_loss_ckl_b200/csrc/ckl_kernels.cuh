@@ -252,11 +252,13 @@ combine_kernel(const float4* __restrict__ partials, int S, const float* __restri
 }
 
 // H_c^T for the dW GEMM: Hc [rows, d] (pitch d) -> HcT [d, pitch_t] (rows
-// contiguous), 32 x 32 tiles through shared memory.
+// contiguous), 32 x 32 tiles through shared memory.  E = uint16_t (bf16) or
+// float (the fp32 entry points).
+template <typename E>
 __global__ void __launch_bounds__(256)
-transpose_rows_kernel(const uint16_t* __restrict__ Hc, int rows, int d, uint16_t* __restrict__ HcT,
+transpose_rows_kernel(const E* __restrict__ Hc, int rows, int d, E* __restrict__ HcT,
                       int pitch_t) {
-  __shared__ uint16_t tile[32][33];
+  __shared__ E tile[32][33];
   const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8 threads
 #pragma unroll
@@ -521,10 +523,21 @@ struct JobIter {
   __device__ bool last_of_unit() const { return vt + 1 == vt_hi; }
 };
 
-template <int MODE, bool PAIR>
+// F32: fp32 operands on kind::tf32 MMAs.  A 128-byte swizzle row holds 64
+// bf16 or 32 fp32 elements, so a stage carries K = 64 or 32 in the same
+// bytes, and an MMA takes K = 16 or 8: four MMAs per stage either way, the
+// same shared-memory layout, the same cycles per stage.
+template <int MODE, bool PAIR, bool F32 = false>
 __global__ void __launch_bounds__(Cfg<MODE, PAIR>::THREADS, 1)
 tc_kernel(const __grid_constant__ TcParams p) {
   using C = Cfg<MODE, PAIR>;
+  constexpr int KE = F32 ? 32 : 64;               // K elements per stage (one 128-byte row)
+  constexpr int KI = F32 ? 8 : 16;                // K per MMA instruction
+  constexpr uint32_t ATOM_B = 128u * KE;          // one MN-major atom column: KE x KE elements
+  constexpr uint32_t MN_STEP = 128u * KI;         // MN-major descriptor advance per MMA
+  // MN-major operands: bf16 in the 128-byte swizzle (8-row atoms, SBO 1024);
+  // tf32 in the 128-byte / 32-byte-base swizzle (4-row atoms, SBO 512)
+  constexpr uint32_t MN_SBO = F32 ? 512u : 1024u;
   constexpr int STAGES = C::STAGES;
   constexpr int EPI_WARPS = C::EPI_WARPS;
   constexpr int B_STAGE = C::B_STAGE;
@@ -598,7 +611,7 @@ tc_kernel(const __grid_constant__ TcParams p) {
         const int half_n = PAIR ? p.bn / 2 : p.bn;  // B rows / columns this CTA stages
         if (MODE != MODE_DHDW) {
           const int rb = it.u % p.n_rb;
-          nkb = (p.d + BK - 1) / BK;
+          nkb = (p.d + KE - 1) / KE;
           a_y = rb * MB + static_cast<int>(rank) * BM;
           b_y = (p.vt0 + it.vt) * BN_V + static_cast<int>(rank) * (BN_V / (PAIR ? 2 : 1));
         } else if (it.phase == 0) {
@@ -612,7 +625,7 @@ tc_kernel(const __grid_constant__ TcParams p) {
           a_x = (it.u / p.n_nt) * MB + static_cast<int>(rank) * BM;      // vocabulary rows
           b_x = (it.u % p.n_nt) * p.bn + static_cast<int>(rank) * half_n;
         }
-        const uint32_t bytes = (MODE != MODE_DHDW) ? A_BYTES + B_STAGE : A_BYTES + half_n * BK * 2;
+        const uint32_t bytes = (MODE != MODE_DHDW) ? A_BYTES + B_STAGE : A_BYTES + half_n * 128;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, p.status)) { ok = false; break; }
           uint32_t fb = bar_full + 8 * stage;
@@ -628,35 +641,34 @@ tc_kernel(const __grid_constant__ TcParams p) {
           const uint32_t sb = sbase + C::B_OFF + stage * B_STAGE;
           if (MODE != MODE_DHDW) {
             if (PAIR) {
-              tma_load_2d_pair(sa, &p.tm[0], fb, kb * BK, a_y);
-              tma_load_2d_pair(sb, &p.tm[1], fb, kb * BK, b_y);
+              tma_load_2d_pair(sa, &p.tm[0], fb, kb * KE, a_y);
+              tma_load_2d_pair(sb, &p.tm[1], fb, kb * KE, b_y);
             } else {
-              tma_load_2d(sa, &p.tm[0], fb, kb * BK, a_y);
-              tma_load_2d(sb, &p.tm[1], fb, kb * BK, b_y);
+              tma_load_2d(sa, &p.tm[0], fb, kb * KE, a_y);
+              tma_load_2d(sb, &p.tm[1], fb, kb * KE, b_y);
             }
           } else if (kind == 5) {
             // dZ is stored as 64-column panels: k-block kb is panel kb.  W is
             // MN-major here: one 64-column atom per box.
             if (PAIR) {
               tma_load_3d_pair(sa, &p.tm[0], fb, 0, a_y, kb);
-              for (int j = 0; j < half_n / 64; ++j)
-                tma_load_2d_pair(sb + j * ATOM_BYTES, &p.tm[1], fb, b_x + 64 * j,
-                                 p.v_lo + kb * BK);
+              for (int j = 0; j < half_n / KE; ++j)
+                tma_load_2d_pair(sb + j * ATOM_B, &p.tm[1], fb, b_x + KE * j, p.v_lo + kb * KE);
             } else {
               tma_load_3d(sa, &p.tm[0], fb, 0, a_y, kb);
-              for (int j = 0; j < half_n / 64; ++j)
-                tma_load_2d(sb + j * ATOM_BYTES, &p.tm[1], fb, b_x + 64 * j, p.v_lo + kb * BK);
+              for (int j = 0; j < half_n / KE; ++j)
+                tma_load_2d(sb + j * ATOM_B, &p.tm[1], fb, b_x + KE * j, p.v_lo + kb * KE);
             }
           } else {
             // A = dZ^T: one box holding the two 64-column panels of this
             // vocabulary row block (8 KB each, one MN-major atom column each).
             // B = H_c^T (d rows x chunk rows, chunk rows contiguous): K-major.
             if (PAIR) {
-              tma_load_3d_pair(sa, &p.tm[2], fb, 0, kb * BK, a_x / 64);
-              tma_load_2d_pair(sb, &p.tm[3], fb, kb * BK, b_x);
+              tma_load_3d_pair(sa, &p.tm[2], fb, 0, kb * KE, a_x / KE);
+              tma_load_2d_pair(sb, &p.tm[3], fb, kb * KE, b_x);
             } else {
-              tma_load_3d(sa, &p.tm[2], fb, 0, kb * BK, a_x / 64);
-              tma_load_2d(sb, &p.tm[3], fb, kb * BK, b_x);
+              tma_load_3d(sa, &p.tm[2], fb, 0, kb * KE, a_x / KE);
+              tma_load_2d(sb, &p.tm[3], fb, kb * KE, b_x);
             }
           }
           ++issued;
@@ -690,18 +702,21 @@ tc_kernel(const __grid_constant__ TcParams p) {
         int nkb;
         uint32_t idesc;
         uint32_t a_step, b_step, a_lbo, b_lbo;
+        bool a_mn = false, b_mn = false;
         if (MODE != MODE_DHDW) {
-          nkb = (p.d + BK - 1) / BK;
-          idesc = idesc_bf16(MMA_M, BN_V, 0, 0);
+          nkb = (p.d + KE - 1) / KE;
+          idesc = F32 ? idesc_tf32(MMA_M, BN_V, 0, 0) : idesc_bf16(MMA_M, BN_V, 0, 0);
           a_step = 32; b_step = 32; a_lbo = 16; b_lbo = 16;
         } else if (it.phase == 0) {
           nkb = p.c5;
-          idesc = idesc_bf16(MMA_M, p.bn, 0, 1);
-          a_step = 32; b_step = 2048; a_lbo = 16; b_lbo = ATOM_BYTES;
+          idesc = F32 ? idesc_tf32(MMA_M, p.bn, 0, 1) : idesc_bf16(MMA_M, p.bn, 0, 1);
+          a_step = 32; b_step = MN_STEP; a_lbo = 16; b_lbo = ATOM_B;
+          b_mn = true;
         } else {
           nkb = p.c6;
-          idesc = idesc_bf16(MMA_M, p.bn, 1, 0);
-          a_step = 2048; b_step = 32; a_lbo = ATOM_BYTES; b_lbo = 16;
+          idesc = F32 ? idesc_tf32(MMA_M, p.bn, 1, 0) : idesc_bf16(MMA_M, p.bn, 1, 0);
+          a_step = MN_STEP; b_step = 32; a_lbo = ATOM_B; b_lbo = 16;
+          a_mn = true;
         }
         if (!mbar_wait(bar_tempty + 8 * acc, acc_phase ^ 1u, p.status)) { ok = false; break; }
         tc_fence_after();
@@ -712,11 +727,20 @@ tc_kernel(const __grid_constant__ TcParams p) {
           const uint32_t sa = sbase + C::A_OFF + stage * A_BYTES;
           const uint32_t sb = sbase + C::B_OFF + stage * B_STAGE;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = sdesc_sw128(sa + kk * a_step, a_lbo, 1024);
-            const uint64_t bd = sdesc_sw128(sb + kk * b_step, b_lbo, 1024);
-            if (PAIR) umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
-            else umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < KE / KI; ++kk) {
+            // a_mn / b_mn: that operand is MN-major (dH's W, dW's dZ^T)
+            const uint64_t ad = (F32 && a_mn) ? sdesc_sw128_b32(sa + kk * a_step, a_lbo, MN_SBO)
+                                              : sdesc_sw128(sa + kk * a_step, a_lbo, 1024);
+            const uint64_t bd = (F32 && b_mn) ? sdesc_sw128_b32(sb + kk * b_step, b_lbo, MN_SBO)
+                                              : sdesc_sw128(sb + kk * b_step, b_lbo, 1024);
+            const uint32_t acc_in = (kb | kk) != 0 ? 1u : 0u;
+            if constexpr (F32) {
+              if (PAIR) umma_tf32_pair(d_tmem, ad, bd, idesc, acc_in);
+              else umma_tf32(d_tmem, ad, bd, idesc, acc_in);
+            } else {
+              if (PAIR) umma_bf16_pair(d_tmem, ad, bd, idesc, acc_in);
+              else umma_bf16(d_tmem, ad, bd, idesc, acc_in);
+            }
           }
           if (PAIR) umma_commit_pair(bar_empty + 8 * stage, 3);
           else umma_commit(bar_empty + 8 * stage);
@@ -907,17 +931,30 @@ tc_kernel(const __grid_constant__ TcParams p) {
             for (int j = 0; j < 32; ++j) if (v0 + j >= p.V) x[j] = 0.f;
           }
           if (!stage_begin()) { ok = false; break; }
-          // 64-byte rows, 64-byte swizzle: 16-byte unit j of row r at unit j ^ ((r >> 1) & 3)
-          const uint32_t rowa = stage_base + (nstore & 1) * EPI_STAGE + srow * 64;
-          const int sw = (lane >> 1) & 3;
+          if constexpr (F32) {
+            // fp32 panels are 32 columns wide: this chunk is one whole panel.
+            // 128-byte rows, 128-byte swizzle: unit j of row r at unit j ^ (r & 7)
+            const uint32_t rowa = stage_base + (nstore & 1) * EPI_STAGE + srow * 128;
+            const int sw = lane & 7;
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            st_shared_v4(rowa + ((j ^ sw) << 4), pack_bf16x2(x[8 * j], x[8 * j + 1]),
-                         pack_bf16x2(x[8 * j + 2], x[8 * j + 3]),
-                         pack_bf16x2(x[8 * j + 4], x[8 * j + 5]),
-                         pack_bf16x2(x[8 * j + 6], x[8 * j + 7]));
-          // panel of this slab's buffer
-          if (!stage_end(0, v0 & 63, y0, (v0 - p.vt0 * BN_V) >> 6)) { ok = false; break; }
+            for (int j = 0; j < 8; ++j)
+              st_shared_v4(rowa + ((j ^ sw) << 4), __float_as_uint(x[4 * j]),
+                           __float_as_uint(x[4 * j + 1]), __float_as_uint(x[4 * j + 2]),
+                           __float_as_uint(x[4 * j + 3]));
+            if (!stage_end(0, 0, y0, (v0 - p.vt0 * BN_V) >> 5)) { ok = false; break; }
+          } else {
+            // 64-byte rows, 64-byte swizzle: 16-byte unit j of row r at unit j ^ ((r >> 1) & 3)
+            const uint32_t rowa = stage_base + (nstore & 1) * EPI_STAGE + srow * 64;
+            const int sw = (lane >> 1) & 3;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              st_shared_v4(rowa + ((j ^ sw) << 4), pack_bf16x2(x[8 * j], x[8 * j + 1]),
+                           pack_bf16x2(x[8 * j + 2], x[8 * j + 3]),
+                           pack_bf16x2(x[8 * j + 4], x[8 * j + 5]),
+                           pack_bf16x2(x[8 * j + 6], x[8 * j + 7]));
+            // panel of this slab's buffer
+            if (!stage_end(0, v0 & 63, y0, (v0 - p.vt0 * BN_V) >> 6)) { ok = false; break; }
+          }
         }
       } else {
         // DHDW: scale and write one accumulator tile (this CTA's rows, all columns).

@@ -71,15 +71,15 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
 
 
 def _normal_bf16(rng: np.random.Generator, rows: int, cols: int, std: float,
-                 block_rows: int = 16384) -> np.ndarray:
-    out = np.empty((rows, cols), dtype=np.uint16)
+                 block_rows: int = 16384, fp32: bool = False) -> np.ndarray:
+    out = np.empty((rows, cols), dtype=np.float32 if fp32 else np.uint16)
     s = np.float32(std)
     for r0 in range(0, rows, block_rows):
         r1 = min(rows, r0 + block_rows)
         x = rng.standard_normal((r1 - r0, cols), dtype=np.float32)
         if std != 1.0:
             x *= s
-        out[r0:r1] = f32_to_bf16_bits(x)
+        out[r0:r1] = x if fp32 else f32_to_bf16_bits(x)
     return out
 
 
@@ -207,19 +207,22 @@ def _make_mask(rng: np.random.Generator, T: int, spec) -> np.ndarray | None:
 def make_inputs(T: int, d: int, V: int, K: int, *, seed: int = 0, h_std: float = 1.0,
                 w_std: float = 0.02, teacher_std: float = 2.0, zipf_s: float = 1.1,
                 mask=None, neighbourhood=None, student_topk=None, chunk: int | None = None,
-                name: str = "custom") -> dict:
+                name: str = "custom", fp32: bool = False) -> dict:
     """Draw one workload.
 
     Returns a dict with ``H`` (uint16 bf16 bits, [T, d]), ``W`` (uint16 bf16
     bits, [V, d]), ``idx`` (int32 [T, K]), ``logp`` (float32 [T, K]), ``mask``
-    (uint8 [T] or None = every position counts) and the sizes.
+    (uint8 [T] or None = every position counts) and the sizes.  ``fp32``:
+    H and W are the same draws kept in float32, not rounded to bf16.
     ``neighbourhood=(top, take)`` draws ``take`` ids per row uniformly from the
     row's top-``top`` student logits (``student_topk(H, W, top)`` returns them,
     descending) and the remaining ``K - take`` from Zipf, excluding those.
     """
+    if fp32 and neighbourhood is not None:
+        raise ValueError("the student top-n neighbourhood is drawn from bf16 inputs")
     rng = np.random.Generator(np.random.PCG64(seed))
-    H = _normal_bf16(rng, T, d, h_std)
-    W = _normal_bf16(rng, V, d, w_std)
+    H = _normal_bf16(rng, T, d, h_std, fp32=fp32)
+    W = _normal_bf16(rng, V, d, w_std, fp32=fp32)
     if neighbourhood is None:
         idx = _zipf_distinct(rng, T, K, V, zipf_s) if T > 0 else np.empty((0, K), np.int32)
     else:
@@ -241,9 +244,10 @@ def make_inputs(T: int, d: int, V: int, K: int, *, seed: int = 0, h_std: float =
                 logp=np.ascontiguousarray(logp, dtype=np.float32), mask=m)
 
 
-def make_config(name: str, seed: int = 0, student_topk=None) -> dict:
-    """One of the five named workloads (see ``CONFIGS``)."""
+def make_config(name: str, seed: int = 0, student_topk=None, fp32: bool = False) -> dict:
+    """One of the five named workloads (see ``CONFIGS``); ``fp32`` keeps H
+    and W in float32 (the tiny workload is an fp32 case)."""
     c = dict(CONFIGS[name])
     return make_inputs(c["T"], c["d"], c["V"], c["K"], seed=seed, w_std=c["w_std"],
                        mask=c.get("mask"), neighbourhood=c.get("neighbourhood"),
-                       student_topk=student_topk, chunk=c["chunk"], name=name)
+                       student_topk=student_topk, chunk=c["chunk"], name=name, fp32=fp32)

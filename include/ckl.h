@@ -223,6 +223,28 @@ CKL_API int ckl_backward_ex(const uint16_t* H, const uint16_t* W, const int32_t*
                             void* user);
 
 /*
+ * fp32 inputs (the pages' fp32 case): the same loss and gradients with H and
+ * W in fp32, multiplied on the tensor cores as tf32 (tcgen05 kind::tf32,
+ * fp32 accumulation; 10-bit mantissa products).  dH is fp32 (like H); dZ is
+ * held in fp32, so the workspace (ckl_workspace_bytes_f32) holds 4 bytes per
+ * dZ entry instead of 2.  Arguments, layouts, status and error behaviour as
+ * in ckl_forward / ckl_backward, with float in place of bf16.
+ */
+CKL_API size_t ckl_workspace_bytes_f32(int64_t T, int64_t d, int64_t V, int32_t K,
+                                       int64_t chunk);
+CKL_API int ckl_forward_f32(const float* H, const float* W, const int32_t* topk_idx,
+                            const float* topk_logp, const uint8_t* mask, int64_t T, int64_t d,
+                            int64_t V, int32_t K, int64_t chunk, float* loss, float* lse,
+                            void* workspace, size_t workspace_bytes, void* stream,
+                            ckl_trace* trace);
+CKL_API int ckl_backward_f32(const float* H, const float* W, const int32_t* topk_idx,
+                             const float* topk_logp, const uint8_t* mask, int64_t T, int64_t d,
+                             int64_t V, int32_t K, int64_t chunk, const float* lse,
+                             const float* grad_loss, float* dH, float* dW,
+                             int32_t accumulate_dW, void* workspace, size_t workspace_bytes,
+                             void* stream, ckl_trace* trace);
+
+/*
  * Reads the device status word of the last call that used `workspace`:
  * synchronises `stream`, copies the word to *device_status (a host pointer)
  * and returns the matching ckl_status (CKL_OK when the word is 0).

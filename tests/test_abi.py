@@ -22,11 +22,12 @@ def ckl():
 
 
 def test_header_declares_the_entry_points():
-    assert _declared() == ["ckl_backward", "ckl_backward_ex", "ckl_backward_plan", "ckl_forward",
-                           "ckl_forward_backward",
-                           "ckl_forward_static_scratch", "ckl_read_device_status",
-                           "ckl_single_pass_workspace_bytes", "ckl_status_string",
-                           "ckl_topk_cache", "ckl_version", "ckl_workspace_bytes"]
+    assert _declared() == ["ckl_backward", "ckl_backward_ex", "ckl_backward_f32",
+                           "ckl_backward_plan", "ckl_forward", "ckl_forward_backward",
+                           "ckl_forward_f32", "ckl_forward_static_scratch",
+                           "ckl_read_device_status", "ckl_single_pass_workspace_bytes",
+                           "ckl_status_string", "ckl_topk_cache", "ckl_version",
+                           "ckl_workspace_bytes", "ckl_workspace_bytes_f32"]
 
 
 def test_library_exports_every_declared_symbol(ckl):
@@ -98,6 +99,16 @@ def test_backward_plan_fits_the_dz_buffer_and_covers_V(ckl):
     # the pages' configs: the 8K head is swept in slabs over all of its rows
     assert ckl.backward_plan(8192, 3072, 128256, 100, 1024) == (8192, 14336, 9)
     assert ckl.backward_plan(1000, 64, 5000, 8, 1000) == (1000, 5056, 1)  # one chunk
+
+
+def test_f32_workspace_holds_fp32_dz(ckl):
+    for T, d, V, K, chunk in ((256, 64, 1024, 16, 64), (8192, 3072, 128256, 100, 1024),
+                              (100, 8, 1003, 5, 64)):
+        f32 = ckl.lib.ckl_workspace_bytes_f32(T, d, V, K, chunk)
+        dz = min(chunk, T) * (-(-V // 64) * 64)          # dZ entries
+        assert f32 >= dz * 4 + T * K * 8                  # fp32 dZ + sorted pairs
+        assert f32 > ckl.lib.ckl_workspace_bytes(T, d, V, K, chunk) - T * d * 4
+    assert ckl.lib.ckl_workspace_bytes_f32(10, 60, 100, 4, 8) == 0
 
 
 def test_workspace_rejects_bad_sizes(ckl):

@@ -77,3 +77,14 @@ def test_neighbourhood_case_takes_half_from_student_top():
     for t in range(30):
         assert set(c["idx"][t, :5]) <= set(top[t])
         assert len(set(c["idx"][t])) == 10
+
+
+def test_fp32_option_keeps_the_same_draws_unrounded():
+    from ckl_synth import f32_to_bf16_bits, make_inputs
+    a = make_inputs(50, 24, 300, 7, seed=3, w_std=0.3, mask=("bernoulli", 0.2))
+    b = make_inputs(50, 24, 300, 7, seed=3, w_std=0.3, mask=("bernoulli", 0.2), fp32=True)
+    assert b["H"].dtype == np.float32 and b["W"].dtype == np.float32
+    assert np.array_equal(f32_to_bf16_bits(b["H"]), a["H"])
+    assert np.array_equal(f32_to_bf16_bits(b["W"]), a["W"])
+    for k in ("idx", "logp", "mask"):
+        assert np.array_equal(a[k], b[k])
