@@ -422,37 +422,48 @@ def bench_ours(args):
         hlogp = pin(c["logp"])
         hmask = None if c["mask"] is None else pin(c["mask"])
         hloss = torch.empty(1, dtype=torch.float32).pin_memory()
-        Hi = H.view(torch.int16)
         bi = hH.numel() * 2 + hidx.numel() * 4 + hlogp.numel() * 4 + (0 if hmask is None else
                                                                         hmask.numel())
 
-        def e2e_step():
-            Hi.copy_(hH, non_blocking=True)
-            idx.copy_(hidx, non_blocking=True)
-            logp.copy_(hlogp, non_blocking=True)
-            if hmask is not None:
-                mask.copy_(hmask, non_blocking=True)
-            step()
-            hloss.copy_(loss, non_blocking=True)
+        # the public staging helper: batch i + 1 crosses PCIe on a side
+        # stream while the loss of batch i runs (each batch is copied once,
+        # inside the timed region)
+        from chunked_kl_loss_ckl_b200.staging import Stager
+        host = [hH, hidx, hlogp] + ([hmask] if hmask is not None else [])
+        stager = Stager(host, dev, stream)
 
-        for _ in range(max(1, args.warmup // 2)):
-            e2e_step()
+        def e2e_run(n):
+            stager.put(host)
+            for i in range(n):
+                bufs = stager.get()
+                if i + 1 < n:
+                    stager.put(host)
+                Hs, ids, lp = bufs[0].view(torch.bfloat16), bufs[1], bufs[2]
+                ms = bufs[3] if hmask is not None else None
+                ckl.forward(Hs, W, ids, lp, ms, chunk, workspace=ws, out_loss=loss, out_lse=lse)
+                ckl.backward(Hs, W, ids, lp, ms, lse, chunk=chunk, dW=dW, accumulate_dW=False,
+                             workspace=ws, out_dH=dH)
+                stager.release()
+                hloss.copy_(loss, non_blocking=True)
+
+        e2e_run(max(1, args.warmup // 2))
         torch.cuda.synchronize()
         if ws_n > 1:
             torch.distributed.barrier()
         f0 = torch.cuda.Event(enable_timing=True)
         f1 = torch.cuda.Event(enable_timing=True)
         f0.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
+        stager.copy_stream.wait_stream(stream)  # no copy starts before f0
+        e2e_run(args.steps)
         f1.record(stream)
         torch.cuda.synchronize()
         ms_e2e = max_over_ranks(f0.elapsed_time(f1) / args.steps, ws_n, dev)
         e2e = {"value": round(tokens / (ms_e2e / 1e3), 1), "unit": "tokens/s",
                "ms_per_step": round(ms_e2e, 4), "h2d_bytes_per_step": int(bi),
                "d2h_bytes_per_step": 4,
-               "copied": "H, topk_idx, topk_logp, mask host->device; loss device->host; "
-                         "W stays resident (a model parameter)"}
+               "copied": "H, topk_idx, topk_logp, mask host->device (staged on a side stream, "
+                         "batch i+1 during step i); loss device->host; W stays resident "
+                         "(a model parameter)"}
 
     cpu = None
     if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:

@@ -284,6 +284,7 @@ __global__ void zero_loss_kernel(float* loss) { *loss = 0.f; }
 // the 64-column panel layout the dH/dW GEMM reads (columns V .. round_up(V, 64)
 // are written 0).  Same arithmetic as the recompute path's dZ epilogue.
 constexpr int ZROW_THREADS = 512;
+constexpr int ZROW_UNROLL = 4;
 
 __global__ void __launch_bounds__(ZROW_THREADS)
 zrow_kernel(const float* __restrict__ Z, int64_t zpitch, const float4* __restrict__ partials,
@@ -316,19 +317,32 @@ zrow_kernel(const float* __restrict__ Z, int64_t zpitch, const float4* __restric
   const bool counts = s_counts != 0;
   const float* zr = Z + static_cast<int64_t>(r) * zpitch;
   const int vend = (V + 63) & ~63;
-  // softmax part, four columns per thread and step
-  for (int v = 4 * threadIdx.x; v < vend; v += 4 * ZROW_THREADS) {
-    float q[4] = {0.f, 0.f, 0.f, 0.f};
-    if (counts && v < V) {
-      const float4 z = *reinterpret_cast<const float4*>(zr + v);
-      const float zz[4] = {z.x, z.y, z.z, z.w};
+  // softmax part, four columns per thread and load; ZROW_UNROLL loads in
+  // flight per thread before any of them is used
+  for (int v0 = 4 * threadIdx.x; v0 < vend; v0 += 4 * ZROW_THREADS * ZROW_UNROLL) {
+    float4 z[ZROW_UNROLL];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) q[j] = (v + j < V) ? ex2_approx(fmaf(zz[j], LOG2E, -lse2)) : 0.f;
+    for (int u = 0; u < ZROW_UNROLL; ++u) {
+      const int v = v0 + u * 4 * ZROW_THREADS;
+      z[u] = (counts && v < V) ? *reinterpret_cast<const float4*>(zr + v)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    uint2 o;
-    o.x = pack_bf16x2(q[0], q[1]);
-    o.y = pack_bf16x2(q[2], q[3]);
-    *reinterpret_cast<uint2*>(dz + ((static_cast<int64_t>(v >> 6) * cap + r) << 6) + (v & 63)) = o;
+#pragma unroll
+    for (int u = 0; u < ZROW_UNROLL; ++u) {
+      const int v = v0 + u * 4 * ZROW_THREADS;
+      if (v >= vend) break;
+      float q[4] = {0.f, 0.f, 0.f, 0.f};
+      if (counts && v < V) {
+        const float zz[4] = {z[u].x, z[u].y, z[u].z, z[u].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          q[j] = (v + j < V) ? ex2_approx(fmaf(zz[j], LOG2E, -lse2)) : 0.f;
+      }
+      uint2 o;
+      o.x = pack_bf16x2(q[0], q[1]);
+      o.y = pack_bf16x2(q[2], q[3]);
+      *reinterpret_cast<uint2*>(dz + ((static_cast<int64_t>(v >> 6) * cap + r) << 6) + (v & 63)) = o;
+    }
   }
   __syncthreads();
   // teacher entries: the first of each run of equal ids rewrites its column

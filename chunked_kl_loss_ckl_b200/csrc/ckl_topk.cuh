@@ -8,17 +8,21 @@
 //
 // One CTA per row (persistent over rows), three passes over the row (the
 // first from HBM, the others mostly from L2):
-//   1. the largest key (packed 16-bit maxima, two keys per instruction);
+//   1. the largest logit (packed bf16 maxima, two per instruction);
 //   2. the row's sum of exp(z - max) (log-sum-exp = max + log of it), and a
-//      histogram of the 256 keys just below the largest (one bucket per bf16
-//      value, two binades) whose block scan finds the K-th largest key; only
+//      histogram of the 128 keys just below the largest (one bucket per bf16
+//      value, one binade) whose block scan finds the K-th largest key; only
 //      if fewer than K elements fall there does the window slide down, 4096
 //      keys at a time, in further passes;
 //   3. every element at or above that key is gathered, and a bitonic sort of
 //      (key, -id) in shared memory puts them in order: descending logit,
 //      equal logits by smaller id.
 // Keys are the bf16 bit patterns mapped to an order-preserving 16-bit code
-// (-0 counts as +0), so every comparison is exact.
+// (-0 counts as +0), so every comparison is exact.  The passes compare the
+// values themselves (bf16 widens exactly; key order is value order) and form
+// a key only for the elements that enter the histogram or the candidates,
+// which keeps the instruction count per logit low: the kernel reads each
+// logit once from HBM and is otherwise bound by its issue rate.
 #pragma once
 
 #include <cstdint>
@@ -31,7 +35,7 @@ namespace ckl {
 
 constexpr int TK_THREADS = 512;
 constexpr int TK_WIN = 4096;  // keys per histogram window
-constexpr int TK_WIN0 = 256;  // keys in the first window (two binades of bf16)
+constexpr int TK_WIN0 = 128;  // keys in the first window (one binade of bf16)
 constexpr int TK_CAP = 2048;  // elements the final sort holds (K plus the ties at the K-th)
 
 __device__ __forceinline__ uint32_t bf16_key(uint32_t b) {
@@ -52,32 +56,43 @@ __device__ __forceinline__ uint32_t bf16_key2(uint32_t w) {
 
 constexpr int TK_UNROLL = 2;  // independent 16-byte loads in flight per thread
 
-// Largest key of the row.
-__device__ __forceinline__ uint32_t tk_row_max(const uint16_t* z, int V, bool vec8) {
-  uint32_t m2 = 0;
+__device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Largest logit of the row (packed bf16 maxima, two per instruction).
+__device__ __forceinline__ float tk_row_max(const uint16_t* z, int V, bool vec8) {
+  float m = -INFINITY;
   if (vec8) {
     const uint4* z4 = reinterpret_cast<const uint4*>(z);
     const int n8 = V / 8;
+    uint32_t m2 = 0xFF80FF80u;  // -inf, -inf
     for (int base = threadIdx.x; base < n8; base += TK_THREADS * TK_UNROLL) {
       uint4 v[TK_UNROLL];
 #pragma unroll
       for (int u = 0; u < TK_UNROLL; ++u) {
         const int i = base + u * TK_THREADS;
-        v[u] = (i < n8) ? z4[i] : make_uint4(0u, 0u, 0u, 0u);
+        v[u] = (i < n8) ? z4[i] : make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u);
       }
 #pragma unroll
       for (int u = 0; u < TK_UNROLL; ++u)
-        m2 = __vmaxu2(m2, __vmaxu2(__vmaxu2(bf16_key2(v[u].x), bf16_key2(v[u].y)),
-                                   __vmaxu2(bf16_key2(v[u].z), bf16_key2(v[u].w))));
+        m2 = bf16x2_max(m2, bf16x2_max(bf16x2_max(v[u].x, v[u].y), bf16x2_max(v[u].z, v[u].w)));
     }
+    m = fmaxf(bf16_lo(m2), bf16_hi(m2));
   } else {
-    for (int i = threadIdx.x; i < V; i += TK_THREADS) m2 = __vmaxu2(m2, bf16_key(z[i]));
+    for (int i = threadIdx.x; i < V; i += TK_THREADS)
+      m = fmaxf(m, __uint_as_float(static_cast<uint32_t>(z[i]) << 16));
   }
-  return max(m2 & 0xFFFFu, m2 >> 16);
+  return m;
 }
 
-// Calls f(key, id) for every element of the row, eight bf16 per 16-byte load
-// when the row allows it.
+// Calls f(value, raw bf16 bits, id) for every element of the row, eight bf16
+// per 16-byte load when the row allows it.  The id is a constant offset from
+// the load's index, so it costs nothing where f does not use it.
 template <typename F>
 __device__ __forceinline__ void tk_for_row(const uint16_t* z, int V, bool vec8, F&& f) {
   if (vec8) {
@@ -97,14 +112,17 @@ __device__ __forceinline__ void tk_for_row(const uint16_t* z, int V, bool vec8, 
           const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            f(bf16_key(w[j] & 0xFFFFu), 8 * i + 2 * j);
-            f(bf16_key(w[j] >> 16), 8 * i + 2 * j + 1);
+            f(bf16_lo(w[j]), w[j] & 0xFFFFu, 8 * i + 2 * j);
+            f(bf16_hi(w[j]), w[j] >> 16, 8 * i + 2 * j + 1);
           }
         }
       }
     }
   } else {
-    for (int i = threadIdx.x; i < V; i += TK_THREADS) f(bf16_key(z[i]), i);
+    for (int i = threadIdx.x; i < V; i += TK_THREADS) {
+      const uint32_t b = z[i];
+      f(__uint_as_float(b << 16), b, i);
+    }
   }
 }
 
@@ -114,7 +132,6 @@ topk_cache_kernel(const uint16_t* __restrict__ logits, int64_t T, int V, int K, 
   __shared__ uint32_t hist[TK_WIN];
   __shared__ unsigned long long cand[TK_CAP];
   __shared__ float s_s[TK_THREADS / 32];
-  __shared__ uint32_t s_k[TK_THREADS / 32];
   __shared__ uint32_t s_part[TK_THREADS / 32];
   __shared__ uint32_t s_thr, s_ncand, s_found, s_total;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -122,17 +139,19 @@ topk_cache_kernel(const uint16_t* __restrict__ logits, int64_t T, int V, int K, 
   for (int64_t row = blockIdx.x; row < T; row += gridDim.x) {
     const uint16_t* z = logits + row * static_cast<int64_t>(V);
 
-    // ---- pass 1: the largest key
-    uint32_t kmax = tk_row_max(z, V, vec8 != 0);
+    // ---- pass 1: the largest logit
+    float zm = tk_row_max(z, V, vec8 != 0);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
-    if (lane == 0) s_k[warp] = kmax;
+    for (int o = 16; o > 0; o >>= 1) zm = fmaxf(zm, __shfl_xor_sync(0xffffffffu, zm, o));
+    if (lane == 0) s_s[warp] = zm;
     for (int j = tid; j < TK_WIN; j += TK_THREADS) hist[j] = 0;
     if (tid == 0) { s_found = 0; s_thr = 0; }
     __syncthreads();
-    kmax = 0;
-    for (int w = 0; w < TK_THREADS / 32; ++w) kmax = max(kmax, s_k[w]);
-    const float zmax = key_value(kmax);  // the row's largest logit
+    float zmax = -INFINITY;
+    for (int w = 0; w < TK_THREADS / 32; ++w) zmax = fmaxf(zmax, s_s[w]);
+    __syncthreads();  // s_s is reused below
+    // its key (bf16 bits of the value; -0 counts as +0)
+    const uint32_t kmax = bf16_key(__float_as_uint(zmax) >> 16);
 
     // ---- pass 2: sum of exp against the maximum, and the first window's
     // histogram; further windows (4096 keys each) only when needed
@@ -141,12 +160,14 @@ topk_cache_kernel(const uint16_t* __restrict__ logits, int64_t T, int V, int K, 
     float lse = 0.f;
     for (int win = 0;; ++win) {
       const int lo = top - (win == 0 ? TK_WIN0 : TK_WIN) + 1;
+      // the window's bounds as values: key order is value order
+      const float v_lo = lo > 0 ? key_value(static_cast<uint32_t>(lo)) : -INFINITY;
+      const float v_top = key_value(static_cast<uint32_t>(top));
       if (win == 0) {
         float s = 0.f;
-        tk_for_row(z, V, vec8 != 0, [&](uint32_t k, int) {
-          s += ex2_approx((key_value(k) - zmax) * LOG2E);
-          const int kk = static_cast<int>(k);
-          if (kk >= lo) atomicAdd(&hist[top - kk], 1u);
+        tk_for_row(z, V, vec8 != 0, [&](float v, uint32_t raw, int) {
+          s += ex2_approx((v - zmax) * LOG2E);  // v - zmax is exact near the max
+          if (v >= v_lo) atomicAdd(&hist[top - static_cast<int>(bf16_key(raw))], 1u);
         });
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
@@ -154,9 +175,8 @@ topk_cache_kernel(const uint16_t* __restrict__ logits, int64_t T, int V, int K, 
       } else {
         for (int j = tid; j < TK_WIN; j += TK_THREADS) hist[j] = 0;
         __syncthreads();
-        tk_for_row(z, V, vec8 != 0, [&](uint32_t k, int) {
-          const int kk = static_cast<int>(k);
-          if (kk <= top && kk >= lo) atomicAdd(&hist[top - kk], 1u);
+        tk_for_row(z, V, vec8 != 0, [&](float v, uint32_t raw, int) {
+          if (v <= v_top && v >= v_lo) atomicAdd(&hist[top - static_cast<int>(bf16_key(raw))], 1u);
         });
       }
       __syncthreads();
@@ -200,15 +220,17 @@ topk_cache_kernel(const uint16_t* __restrict__ logits, int64_t T, int V, int K, 
       __syncthreads();
     }
     const uint32_t thr = s_thr;
+    const float v_thr = key_value(thr);
 
-    // ---- pass 3: gather every element at or above the threshold key
+    // ---- pass 3: gather every element at or above the threshold
     if (tid == 0) s_ncand = 0;
     __syncthreads();
-    tk_for_row(z, V, vec8 != 0, [&](uint32_t k, int i) {
-      if (k >= thr) {
+    tk_for_row(z, V, vec8 != 0, [&](float v, uint32_t raw, int i) {
+      if (v >= v_thr) {
         const uint32_t slot = atomicAdd(&s_ncand, 1u);
         if (slot < TK_CAP)
-          cand[slot] = (static_cast<unsigned long long>(k) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(i));
+          cand[slot] = (static_cast<unsigned long long>(bf16_key(raw)) << 32) |
+                       (0xFFFFFFFFu - static_cast<uint32_t>(i));
       }
     });
     __syncthreads();
