@@ -23,7 +23,7 @@ __all__ = [
     "LIB_PATH", "CklError", "Trace", "KERNEL_NAMES", "lib", "workspace_bytes", "new_workspace",
     "forward", "backward", "read_device_status", "status_string", "chunked_kl_loss",
     "topk_cache", "single_pass_workspace_bytes", "forward_backward", "backward_plan",
-    "DW_READY_FN", "forward_f32", "backward_f32",
+    "DW_READY_FN", "forward_f32", "backward_f32", "selftest_wait_timeout",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libckl.so")
@@ -93,6 +93,8 @@ def _load() -> ctypes.CDLL:
     L.ckl_forward_backward.restype = ctypes.c_int
     L.ckl_topk_cache.argtypes = [vp, i64, i64, i32, vp, vp, vp, vp]
     L.ckl_topk_cache.restype = ctypes.c_int
+    L.ckl_selftest_wait_timeout.argtypes = [i64, vp, sz, vp]
+    L.ckl_selftest_wait_timeout.restype = ctypes.c_int
     L.ckl_read_device_status.argtypes = [vp, vp, ctypes.POINTER(i32)]
     L.ckl_read_device_status.restype = ctypes.c_int
     L.ckl_status_string.argtypes = [i32]
@@ -366,6 +368,15 @@ def topk_cache(logits, K: int, stream=None, status=None):
     if rc != CKL_OK:
         raise CklError(rc, "ckl_topk_cache")
     return idx, logp, st
+
+
+def selftest_wait_timeout(limit_s: float, workspace, stream=None) -> None:
+    """Launch the bounded-wait self-test (ckl_selftest_wait_timeout); read the
+    result with read_device_status(workspace)."""
+    rc = lib.ckl_selftest_wait_timeout(int(limit_s * 1e9), _ptr(workspace), workspace.numel(),
+                                       _stream_handle(stream))
+    if rc != CKL_OK:
+        raise CklError(rc, "ckl_selftest_wait_timeout")
 
 
 def read_device_status(workspace, stream=None):

@@ -850,6 +850,22 @@ int ckl_topk_cache(const uint16_t* teacher_logits, int64_t T, int64_t V, int32_t
   return cudaGetLastError() == cudaSuccess ? CKL_OK : CKL_ERR_CUDA;
 }
 
+int ckl_selftest_wait_timeout(int64_t limit_ns, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  if (!workspace || !aligned16(workspace) || workspace_bytes < kHeaderBytes)
+    return CKL_ERR_INVALID_ARG;
+  if (limit_ns < 1000000 || limit_ns > 4000000000ll) return CKL_ERR_INVALID_ARG;
+  DevInfo di;
+  if (!device_info(di)) return CKL_ERR_CUDA;
+  if (di.major != 10) return CKL_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(workspace, 0, kHeaderBytes, st) != cudaSuccess) return CKL_ERR_CUDA;
+  Header* hdr = static_cast<Header*>(workspace);
+  ckl::wait_timeout_selftest_kernel<<<1, 32, 0, st>>>(&hdr->status,
+                                                      static_cast<uint64_t>(limit_ns));
+  return cudaGetLastError() == cudaSuccess ? CKL_OK : CKL_ERR_CUDA;
+}
+
 int ckl_read_device_status(const void* workspace, void* stream, int32_t* device_status) {
   if (!workspace || !device_status) return CKL_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

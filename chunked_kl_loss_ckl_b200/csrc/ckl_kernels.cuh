@@ -35,11 +35,10 @@
 namespace ckl {
 
 constexpr int BM = 128;           // rows per tile (TMEM lanes)
-constexpr int BK = 64;            // bf16 elements per 128-byte swizzle row
+constexpr int BK = 64;            // bf16 elements per 128-byte swizzle row (32 for fp32)
 constexpr int BN_V = 256;         // vocabulary columns per logit tile
 constexpr int A_BYTES = BM * BK * 2;        // 16 KB
 constexpr int B_BYTES = 256 * BK * 2;       // 32 KB (largest B tile)
-constexpr int ATOM_BYTES = 64 * BK * 2;     // one 64-wide MN-major atom column, 8 KB
 constexpr int EPI_STAGE = BM * 128;         // one 128-row x 128-byte staging tile, 16 KB
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COLS = 256;          // TMEM columns per accumulator buffer
@@ -276,6 +275,22 @@ transpose_rows_kernel(const E* __restrict__ Hc, int rows, int d, E* __restrict__
 
 // Loss of an empty batch (T = 0).
 __global__ void zero_loss_kernel(float* loss) { *loss = 0.f; }
+
+// Self-test of the bounded waits: one CTA waits, with the kernels' own wait,
+// on an mbarrier that nothing arrives on.  The wait runs out after limit_ns,
+// records CKL_DEV_TIMEOUT in *status and the kernel returns normally, so the
+// context stays usable.
+__global__ void wait_timeout_selftest_kernel(int* status, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    mbar_init(b, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait_ns(b, 0, status, limit_ns);
+  __syncthreads();
+}
 
 // ------------------------------------------------------------------ single pass
 // One chunk row per CTA, after the FWDZ GEMM: merge the row's vocabulary

@@ -55,19 +55,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait for the phase with the given parity to complete.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* status) {
+// Bounded wait for the phase with the given parity to complete: false, with
+// CKL_DEV_TIMEOUT recorded, once limit_ns have passed.
+__device__ __forceinline__ bool mbar_wait_ns(uint32_t bar, uint32_t parity, int* status,
+                                             uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > CKL_WAIT_NS) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       atomicOr(status, CKL_DEV_TIMEOUT);
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* status) {
+  return mbar_wait_ns(bar, parity, status, CKL_WAIT_NS);
 }
 
 // ---------------------------------------------------------------- TMA

@@ -245,6 +245,19 @@ CKL_API int ckl_backward_f32(const float* H, const float* W, const int32_t* topk
                              void* stream, ckl_trace* trace);
 
 /*
+ * Self-test of the kernels' bounded waits (failure detection without a GPU
+ * fault; no counterpart in the pages).  Launches one CTA on `stream` that
+ * waits, with the same time-bounded mbarrier wait every kernel uses, on a
+ * barrier nothing arrives on.  After limit_ns (1 ms .. 4 s) the wait gives
+ * up, CKL_DEV_TIMEOUT is recorded in the status word at the start of
+ * `workspace` (>= 256 bytes, 16-byte aligned), and the kernel returns: the
+ * context stays usable.  ckl_read_device_status(workspace, ...) then returns
+ * CKL_ERR_TIMEOUT.  Returns CKL_ERR_INVALID_ARG for a bad limit or workspace.
+ */
+CKL_API int ckl_selftest_wait_timeout(int64_t limit_ns, void* workspace, size_t workspace_bytes,
+                                      void* stream);
+
+/*
  * Reads the device status word of the last call that used `workspace`:
  * synchronises `stream`, copies the word to *device_status (a host pointer)
  * and returns the matching ckl_status (CKL_OK when the word is 0).

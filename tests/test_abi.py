@@ -25,7 +25,8 @@ def test_header_declares_the_entry_points():
     assert _declared() == ["ckl_backward", "ckl_backward_ex", "ckl_backward_f32",
                            "ckl_backward_plan", "ckl_forward", "ckl_forward_backward",
                            "ckl_forward_f32", "ckl_forward_static_scratch",
-                           "ckl_read_device_status", "ckl_single_pass_workspace_bytes",
+                           "ckl_read_device_status", "ckl_selftest_wait_timeout",
+                           "ckl_single_pass_workspace_bytes",
                            "ckl_status_string", "ckl_topk_cache", "ckl_version",
                            "ckl_workspace_bytes", "ckl_workspace_bytes_f32"]
 
@@ -153,6 +154,11 @@ def test_host_checks_return_before_any_device_work(ckl):
     assert L.ckl_forward_backward(fake, fake, fake, fake, nul, 4, 64, 100, 4, 8, nul, fake, fake,
                                   fake, fake, 0, fake, small, nul, nul) == 3
     assert L.ckl_read_device_status(nul, nul, nul) == 1
+    # the wait self-test: limit outside [1 ms, 4 s], or no workspace
+    assert L.ckl_selftest_wait_timeout(10, fake, 1 << 20, nul) == 1
+    assert L.ckl_selftest_wait_timeout(5_000_000_000, fake, 1 << 20, nul) == 1
+    assert L.ckl_selftest_wait_timeout(50_000_000, nul, 1 << 20, nul) == 1
+    assert L.ckl_selftest_wait_timeout(50_000_000, fake, 16, nul) == 1
     # top-K cache: K must be in [1, min(V, 2048)]
     assert L.ckl_topk_cache(fake, 4, 100, 0, fake, fake, nul, nul) == 1
     assert L.ckl_topk_cache(fake, 4, 100, 101, fake, fake, nul, nul) == 1
