@@ -334,14 +334,21 @@ int choose_splits(int64_t n_rb, int64_t n_vt, int sms) {
   return best;
 }
 
+// d-tile width of the dH / dW GEMMs.  A narrower tile wastes fewer padded
+// columns but reads more shared memory per FLOP: at M = 256 (a CTA pair) and
+// N = 128 each MMA needs as many operand bytes per clock as shared memory
+// delivers, so those tiles run well below the tensor peak (a d = 2880 head
+// measured 690 against 1270 TFLOP/s).  Cost per column: padded width, times
+// 1.5 for N = 128 (2 for N = 64).
 int pick_bn(int64_t d) {
   int best = 256;
-  int64_t best_waste = cdiv(d, 256) * 256 - d;
+  double best_cost = static_cast<double>(cdiv(d, 256) * 256);
   for (int bn : {192, 128, 64}) {
     if (kPair && bn % 128 != 0) continue;  // each CTA of a pair stages bn/2 columns
-    const int64_t w = cdiv(d, bn) * bn - d;
-    if (w < best_waste) {
-      best_waste = w;
+    const double slow = bn >= 192 ? 1.0 : bn == 128 ? 1.5 : 2.0;
+    const double cost = static_cast<double>(cdiv(d, bn) * bn) * slow;
+    if (cost < best_cost) {
+      best_cost = cost;
       best = bn;
     }
   }
