@@ -316,12 +316,13 @@ struct TraceScope {
 };
 
 // Vocabulary splits S for n_rb row blocks: the most even makespan over the
-// SMs (every unit = one row block x one contiguous run of vocabulary tiles).
-int choose_splits(int64_t n_rb, int64_t n_vt, int sms) {
-  int best = 1;
+// SMs (every unit = one row block x one contiguous run of vocabulary tiles),
+// with S in [smin, smax].
+int choose_splits(int64_t n_rb, int64_t n_vt, int sms, int smin = 1, int smax_in = kMaxSplits) {
+  int best = std::max(1, std::min<int>(smin, static_cast<int>(n_vt)));
   double best_cost = 1e300;
-  const int smax = static_cast<int>(std::min<int64_t>(kMaxSplits, n_vt));
-  for (int S = 1; S <= smax; ++S) {
+  const int smax = static_cast<int>(std::min<int64_t>(std::min(kMaxSplits, smax_in), n_vt));
+  for (int S = std::max(1, smin); S <= smax; ++S) {
     const int64_t units = n_rb * S;
     const int64_t waves = cdiv(units, sms);
     const double per_unit = static_cast<double>(cdiv(n_vt, S)) + 0.25;  // +: unit set-up
@@ -340,6 +341,22 @@ int choose_splits(int64_t n_rb, int64_t n_vt, int sms) {
 // delivers, so those tiles run well below the tensor peak (a d = 2880 head
 // measured 690 against 1270 TFLOP/s).  Cost per column: padded width, times
 // 1.5 for N = 128 (2 for N = 64).
+// Splits and unit order of a forward launch over n_rb row blocks: when the
+// row blocks' H (kMB x d each) does not fit in 48 MiB of L2 together, number
+// the units split-fastest with S near sqrt(slots), so that the units in
+// flight share about slots / S row blocks and S W tiles.
+void forward_schedule(TcParams& p, int64_t d, int eb, int slots) {
+  const int64_t hblk = kMB * d * eb;
+  if (static_cast<int64_t>(p.n_rb) * hblk > (int64_t(48) << 20)) {
+    p.split_fast = 1;
+    p.S = choose_splits(p.n_rb, p.n_vt, slots, 4, 16);
+  } else {
+    p.split_fast = 0;
+    p.S = choose_splits(p.n_rb, p.n_vt, slots);
+  }
+  p.n_units = p.n_rb * p.S;
+}
+
 int pick_bn(int64_t d) {
   int best = 256;
   double best_cost = static_cast<double>(cdiv(d, 256) * 256);
@@ -585,8 +602,7 @@ int forward_impl(const void* H, const void* W, const int32_t* topk_idx, const fl
   p.rows = static_cast<int32_t>(T);
   p.row0 = 0;
   p.n_rb = static_cast<int32_t>(cdiv(T, kMB));
-  p.S = choose_splits(p.n_rb, p.n_vt, di.slots[ckl::MODE_FWD]);
-  p.n_units = p.n_rb * p.S;
+  forward_schedule(p, d, eb, di.slots[ckl::MODE_FWD]);
   if (!map2d(&p.tm[0], kDT<F32>, H, d, T, d * eb, kKE<F32>, ckl::BM,
              CU_TENSOR_MAP_SWIZZLE_128B) ||
       !map2d(&p.tm[1], kDT<F32>, W, d, V, d * eb, kKE<F32>, ckl::BN_V / kSlotCTAs,
@@ -794,8 +810,7 @@ int ckl_forward_backward(const uint16_t* H, const uint16_t* W, const int32_t* to
     p.rows = static_cast<int32_t>(rows);
     p.row0 = static_cast<int32_t>(c0);
     p.n_rb = static_cast<int32_t>(cdiv(rows, kMB));
-    p.S = choose_splits(p.n_rb, p.n_vt, di.slots[ckl::MODE_FWDZ]);
-    p.n_units = p.n_rb * p.S;
+    forward_schedule(p, d, 2, di.slots[ckl::MODE_FWDZ]);
     if (!map2d(&p.tm[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Hc, d, rows, d * 2, ckl::BK, ckl::BM,
                CU_TENSOR_MAP_SWIZZLE_128B) ||
         !map2d(&p.tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, V, d * 2, ckl::BK,

@@ -93,6 +93,7 @@ struct alignas(64) TcParams {
   int32_t v_lo;     // DHDW: first vocabulary column of this launch's slab
   int32_t dh_mode;  // DHDW: 0 = dH as bf16, 1 = store fp32 partial dH, 2 = add into it
   int32_t dw_mode;  // DHDW: 0 = contiguous dW ranges per slot, 1 = dW tiles dealt in rounds
+  int32_t split_fast;  // FWD: units numbered split-fastest (see JobIter)
   int32_t dw_Ql, dw_El, dw_Qh, dw_Eh;  // DHDW rounds: quotas, see JobIter
   const int2* pairs;      // [T, K] (id, p as bits), sorted by id per row
   float4* partials;       // FWD: [T, S] (max of z log2e, sum 2^(..), sum p z, 0)
@@ -480,8 +481,19 @@ struct JobIter {
         cls_rank(k6, cta < r5 ? cta : r5, p.dw_Qh, p.dw_Eh) +
         (cta > r5 ? cls_rank(k6, cta - r5, p.dw_Ql, p.dw_El) : 0);
   }
+  // FWD unit -> (row block, split).  Row-block-fastest by default: the units
+  // in flight sweep the same W tiles of a split, and every row block's H
+  // stays in L2.  When all of H does not fit there (split_fast), split-
+  // fastest: the units in flight hold about G / S row blocks and S W tiles.
+  // (DZ: u is the row block itself.)
+  __device__ int unit_rb(const TcParams& p, int unit) const {
+    return (mode != MODE_DZ && p.split_fast) ? unit / p.S : unit % p.n_rb;
+  }
+  __device__ int unit_s(const TcParams& p, int unit) const {
+    return p.split_fast ? unit % p.S : unit / p.n_rb;
+  }
   __device__ void vt_range(const TcParams& p, int unit, int& lo, int& hi) const {
-    const int s = unit / p.n_rb;
+    const int s = unit_s(p, unit);
     lo = static_cast<int>(static_cast<int64_t>(s) * p.n_vt / p.S);
     hi = static_cast<int>(static_cast<int64_t>(s + 1) * p.n_vt / p.S);
   }
@@ -639,7 +651,7 @@ tc_kernel(const __grid_constant__ TcParams p) {
         int a_x = 0, a_y = 0, b_x = 0, b_y = 0, kind = 0;
         const int half_n = PAIR ? p.bn / 2 : p.bn;  // B rows / columns this CTA stages
         if (MODE != MODE_DHDW) {
-          const int rb = it.u % p.n_rb;
+          const int rb = it.unit_rb(p, it.u);
           nkb = (p.d + KE - 1) / KE;
           a_y = rb * MB + static_cast<int>(rank) * BM;
           b_y = (p.vt0 + it.vt) * BN_V + static_cast<int>(rank) * (BN_V / (PAIR ? 2 : 1));
@@ -866,7 +878,7 @@ tc_kernel(const __grid_constant__ TcParams p) {
     it.init(p, MODE, PAIR ? 2 : 1);
     for (; ok && it.valid(p); it.next(p)) {
       if (MODE != MODE_DHDW && it.first_of_unit(p)) {
-        const int rb = it.u % p.n_rb;
+        const int rb = it.unit_rb(p, it.u);
         const int r = rb * MB + row_in_tile;  // row within T (FWD) or the chunk (DZ)
         row_ok = r < p.rows;
         t = static_cast<int64_t>(p.row0) + r;
@@ -892,7 +904,7 @@ tc_kernel(const __grid_constant__ TcParams p) {
       const uint32_t tacc = tmem_base + lane_off + static_cast<uint32_t>(acc) * ACC_COLS;
 
       if (MODE == MODE_FWD || MODE == MODE_FWDZ) {
-        const int zy0 = (it.u % p.n_rb) * MB + row0_cta;  // FWDZ: first chunk row of this CTA
+        const int zy0 = it.unit_rb(p, it.u) * MB + row0_cta;  // FWDZ: first chunk row of this CTA
         for (int c = 0; c < BN_V / 32; ++c) {
           const int v0 = (p.vt0 + it.vt) * BN_V + c * 32;
           if (v0 >= p.V) break;
@@ -1030,7 +1042,7 @@ tc_kernel(const __grid_constant__ TcParams p) {
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
 
       if ((MODE == MODE_FWD || MODE == MODE_FWDZ) && it.last_of_unit() && row_ok) {
-        const int s = it.u / p.n_rb;
+        const int s = it.unit_s(p, it.u);
         p.partials[t * p.S + s] = make_float4(run_m, run_s, run_pz, 0.f);
       }
     }

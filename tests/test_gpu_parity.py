@@ -54,6 +54,13 @@ def test_sliced_backward_both_dw_schedules(gpu_lib):
     assert_parity(run_library(gpu_lib, c, chunk=512), _ref(c), "sliced 3072x8192x1024")
 
 
+def test_forward_units_split_fastest_when_H_exceeds_L2(gpu_lib):
+    # 25 row blocks of 256 x 4096 bf16 (52 MB) do not fit the forward's 48 MiB
+    # L2 budget together: its units are numbered split-fastest
+    c = make_inputs(6400, 4096, 1536, 8, seed=18, w_std=0.02, mask=("bernoulli", 0.1))
+    assert_parity(run_library(gpu_lib, c, chunk=1024), _ref(c), "split-fastest forward")
+
+
 def test_lse_is_bitwise_identical_across_chunk_sizes(gpu_lib):
     c = make_inputs(300, 200, 1000, 16, seed=6, w_std=0.3)
     outs = [run_library(gpu_lib, c, chunk=ch) for ch in (64, 128, 300)]
