@@ -104,10 +104,12 @@ typedef struct ckl_trace {
  * Workspace bytes needed by ckl_forward / ckl_backward for these sizes.
  * Linear in T: per token K*8 (sorted teacher pairs) + 4 (sum p log p) +
  * 64*16 (vocabulary-split partials) + 8/256 bytes, plus, independent of T
- * once T >= chunk, a chunk x V bf16 buffer for dZ (min(chunk, T) rows of
- * round_up(V, 64) entries), a transposed copy of one chunk of H
- * (d x round_up(min(chunk, T), 8) bf16) and a 256-byte header.  Returns 0
- * for sizes outside the supported range.
+ * once T > chunk, a chunk x V bf16 buffer for dZ (min(chunk, T) rows of
+ * round_up(V, 64) entries), and for the blocked backward (ckl_backward_plan)
+ * a transposed copy of up to R rows of H (d x R bf16) and an fp32 partial dH
+ * of R rows (R x d fp32), R = min(round_up(sqrt(chunk V), 256), the rows of
+ * 48 MiB of H) or 0 when T <= chunk, and a 256-byte header.  Returns 0 for
+ * sizes outside the supported range.
  */
 CKL_API size_t ckl_workspace_bytes(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk);
 
@@ -151,11 +153,15 @@ CKL_API int ckl_forward(const uint16_t* H, const uint16_t* W, const int32_t* top
                 size_t workspace_bytes, void* stream, ckl_trace* trace);
 
 /*
- * Backward by recomputation, one chunk of rows at a time: each chunk's
- * logits are rebuilt from H and W, turned into the unscaled logit gradient
+ * Backward by recomputation, one block at a time: each block's logits are
+ * rebuilt from H and W, turned into the unscaled logit gradient
  * dZ = exp(z - lse) - scatter(p) (0 on rows that do not count), stored as
- * bf16 in the workspace (at most chunk x V), then fed to two tensor-core
- * GEMMs: dH_c = s dZ_c W and dW (+)= s dZ_c^T H_c, with s = g / N.
+ * bf16 in the workspace (at most chunk x V entries), then fed to two
+ * tensor-core GEMMs: dH_c = s dZ_c W and dW (+)= s dZ_c^T H_c, with
+ * s = g / N.  A block is one chunk of rows x all V (the pages' schedule) or,
+ * when that moves fewer bytes, a taller row chunk x a vocabulary slab of the
+ * same size (ckl_backward_plan reports which); the results are the same up
+ * to fp32 summation order.
  *   lse        [T]    fp32  from ckl_forward on the same inputs
  *   grad_loss  [1]    fp32  upstream gradient g (device); NULL = 1
  *   dH         [T, d] bf16  out (fp32 accumulation, rounded once)
