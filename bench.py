@@ -55,6 +55,8 @@ def parse_args(argv=None):
                     help="measure workspace and peak device memory vs T at the 256K shape")
     ap.add_argument("--topk", action="store_true",
                     help="time the teacher top-K cache producer (T=8192, V=128256, K=100)")
+    ap.add_argument("--f32", action="store_true",
+                    help="time the fp32-input entry points (tf32 tensor cores) on the workload")
     ap.add_argument("--compare", action="store_true",
                     help="peak memory and time vs T: dense / forward-chunked PyTorch losses "
                          "against the fused library, at the 32K shape")
@@ -689,6 +691,53 @@ def compare(args):
           flush=True)
 
 
+def bench_f32(args):
+    """Forward + backward of the fp32-input entry points (tf32 products) on the
+    workload with H and W kept in fp32; TFLOP/s against the tf32 peak taken as
+    the measured sustained bf16 peak x the nominal tf32 / bf16 ratio (1.1 / 2.25)."""
+    import torch
+    import chunked_kl_loss_ckl_b200 as ckl
+    from ckl_synth import make_config
+    dev = torch.device("cuda", 0)
+    c = make_config(args.config, seed=args.seed, fp32=True)
+    T, d, V, K, chunk = c["T"], c["d"], c["V"], c["K"], c["chunk"]
+    H = torch.from_numpy(c["H"]).to(dev)
+    W = torch.from_numpy(c["W"]).to(dev)
+    idx = torch.from_numpy(c["idx"]).to(dev)
+    logp = torch.from_numpy(c["logp"]).to(dev)
+    mask = None if c["mask"] is None else torch.from_numpy(c["mask"]).to(dev)
+    ws = torch.empty(ckl.lib.ckl_workspace_bytes_f32(T, d, V, K, chunk), dtype=torch.uint8,
+                     device=dev)
+    dW = torch.empty(V, d, dtype=torch.float32, device=dev)
+
+    def step():
+        loss, lse = ckl.forward_f32(H, W, idx, logp, mask, chunk, workspace=ws)
+        ckl.backward_f32(H, W, idx, logp, mask, lse, chunk=chunk, dW=dW, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    rc, word = ckl.read_device_status(ws)
+    ms = e0.elapsed_time(e1) / args.steps
+    peaks, src = load_peaks()
+    tf32_peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])) \
+        * 1.1 / 2.25
+    tflops = flops_per_token(c) * T / (ms / 1e3) / 1e12
+    print(json.dumps({"path": "fp32 inputs, tf32 tensor cores", "workload": workload_desc(c),
+                      "value": round(T / (ms / 1e3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 4),
+                      "tflops": round(tflops, 1), "tf32_peak": round(tf32_peak, 1),
+                      "frac": round(tflops / tf32_peak, 4),
+                      "peak_source": f"{src} bf16_tflops_sustained x 1.1 / 2.25 (nominal tf32 / bf16)",
+                      "status": rc}), flush=True)
+
+
 def bench_topk(args):
     """The teacher top-K cache producer: one pass over [T, V] bf16 logits,
     HBM-bound; achieved GB/s = (T V 2 + T K 8) bytes / kernel time."""
@@ -730,6 +779,9 @@ def main(argv=None):
         return
     if args.topk:
         bench_topk(args)
+        return
+    if args.f32:
+        bench_f32(args)
         return
     if args.impl == "reference":
         bench_reference(args)
