@@ -134,49 +134,134 @@ def rank_seed(base: int, rank: int) -> int:
 
 # ----------------------------------------------------------------- clocks
 class ClockSampler:
+    """SM clock, power and clock-event reasons of one GPU, sampled on a host
+    thread every ``period_s`` through NVML (or ``nvidia-smi -lms`` when NVML
+    is unavailable), each sample stamped with ``time.perf_counter()``.
+    ``stop(t0, t1)`` summarises only the samples taken inside [t0, t1], the
+    host interval that brackets the timed region."""
+
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, gpu_uuid: str | None):
+    def __init__(self, gpu_uuid: str | None, period_s: float = 0.02):
+        import threading
+        self.samples = []          # (t, sm MHz, max sm MHz, power W or None, reasons)
+        self.source = None
+        self._stop = threading.Event()
+        self._thread = None
         self.proc = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = (pynvml.nvmlDeviceGetHandleByUUID(gpu_uuid.encode()) if gpu_uuid
+                 else pynvml.nvmlDeviceGetHandleByIndex(0))
+            bits = {"hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
+            smax = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+
+            def poll():
+                while not self._stop.is_set():
+                    t = time.perf_counter()
+                    try:
+                        sm = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                        pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1e3
+                        r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.samples.append((t, sm, smax, pw,
+                                             {n for n, b in bits.items() if r & b}))
+                    except Exception:
+                        pass
+                    self._stop.wait(period_s)
+
+            self.source = f"NVML, every {int(period_s * 1e3)} ms"
+            self._thread = threading.Thread(target=poll, daemon=True)
+            self._thread.start()
+            return
+        except Exception:
+            pass
         cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-               "-lms", "100"]
+               "-lms", str(max(10, int(period_s * 1e3)))]
         if gpu_uuid:
             cmd += ["-i", gpu_uuid]
         try:
             self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
                                          text=True)
         except OSError:
-            self.proc = None
+            return
+        self.source = f"nvidia-smi -lms {max(10, int(period_s * 1e3))}"
 
-    def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        sm, smax, reasons = [], [], set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for line in out.strip().splitlines():
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
+        def read():
+            for line in self.proc.stdout:
+                t = time.perf_counter()
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm, smax = float(parts[1]), float(parts[2])
+                except ValueError:
+                    continue
+                try:
+                    pw = float(parts[3])
+                except ValueError:
+                    pw = None
+                self.samples.append((t, sm, smax, pw, {n for n, v in zip(self.NAMES, parts[5:9])
+                                                        if v.lower() == "active"}))
+
+        import threading
+        self._thread = threading.Thread(target=read, daemon=True)
+        self._thread.start()
+
+    def stop(self, t0: float | None = None, t1: float | None = None):
+        self._stop.set()
+        if self.proc is not None:
+            self.proc.terminate()
             try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
-                "reasons": sorted(reasons)}
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self._thread is not None:
+            self._thread.join(timeout=5)
+        return summarise_clocks(self.samples, t0, t1, self.source)
+
+
+def summarise_clocks(samples, t0=None, t1=None, source=None):
+    """Median / min SM clock, median power and the reasons seen, over the
+    samples with t0 <= t <= t1 (all of them when no window is given)."""
+    inside = [s for s in samples if (t0 is None or s[0] >= t0) and (t1 is None or s[0] <= t1)]
+    if not inside:
+        return None
+    sm = [s[1] for s in inside]
+    pw = [s[3] for s in inside if s[3] is not None]
+    reasons = set()
+    for s in inside:
+        reasons |= s[4]
+    return {"sm_mhz": statistics.median(sm), "sm_min_mhz": min(sm),
+            "sm_max_mhz": max(s[2] for s in inside),
+            "power_w": round(statistics.median(pw), 1) if pw else None,
+            "samples": len(inside), "reasons": sorted(reasons),
+            "window_s": None if t0 is None or t1 is None else round(t1 - t0, 3),
+            "source": f"{source}; only samples inside the timed region"}
+
+
+def cpu_description():
+    """(model name, logical CPUs this process may run on)."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:
+        n = os.cpu_count() or 1
+    return model, n
 
 
 # ----------------------------------------------------------------- CPU oracle
@@ -271,15 +356,17 @@ def bench_ours(args):
         torch.distributed.barrier()
     torch.cuda.synchronize()
     sampler = ClockSampler(uuid)
-    time.sleep(0.3)
+    time.sleep(0.1)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    t_begin = time.perf_counter()
     e0.record(stream)
     for _ in range(args.steps):
         step(trace)
     e1.record(stream)
     torch.cuda.synchronize()
-    clocks = sampler.stop()
+    t_end = time.perf_counter()
+    clocks = sampler.stop(t_begin, t_end)
     if ws_n > 1:
         torch.distributed.barrier()
     ms_total = e0.elapsed_time(e1)
@@ -470,7 +557,9 @@ def bench_ours(args):
     cpu = None
     if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
         tps, rows, secs, threads = cpu_oracle_sample(c, args.cpu_seconds)
+        model, ncpu = cpu_description()
         cpu = {"value": round(tps, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "cpu_model": model, "nproc": ncpu,
                "sample": f"fp64 oracle (numpy, chunked form) on the first {rows} tokens of the "
                          f"same workload, full V and d: loss, lse, dH, dW; {secs:.1f} s"}
 
@@ -530,7 +619,8 @@ def bench_reference(args):
         "config": {"workload": workload_desc(c), "T": c["T"], "d": c["d"], "V": c["V"],
                    "K": c["K"], "chunk": c["chunk"], "sample_rows_per_step": rows},
         "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": threads,
-                         "kind": "oracle",
+                         "kind": "oracle", "cpu_model": cpu_description()[0],
+                         "nproc": cpu_description()[1],
                          "sample": f"fp64 oracle on {rows} tokens per step (full V, d)"},
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},

@@ -23,7 +23,8 @@ __all__ = [
     "LIB_PATH", "CklError", "Trace", "KERNEL_NAMES", "lib", "workspace_bytes", "new_workspace",
     "forward", "backward", "read_device_status", "status_string", "chunked_kl_loss",
     "topk_cache", "single_pass_workspace_bytes", "forward_backward", "backward_plan",
-    "DW_READY_FN", "forward_f32", "backward_f32", "selftest_wait_timeout",
+    "DW_READY_FN", "forward_f32", "backward_f32", "selftest_wait_timeout", "dp_local_stats",
+    "dp_finish",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libckl.so")
@@ -95,6 +96,10 @@ def _load() -> ctypes.CDLL:
     L.ckl_topk_cache.restype = ctypes.c_int
     L.ckl_selftest_wait_timeout.argtypes = [i64, vp, sz, vp]
     L.ckl_selftest_wait_timeout.restype = ctypes.c_int
+    L.ckl_dp_local_stats.argtypes = [vp, vp, vp]
+    L.ckl_dp_local_stats.restype = ctypes.c_int
+    L.ckl_dp_finish.argtypes = [vp, vp, vp, vp, vp]
+    L.ckl_dp_finish.restype = ctypes.c_int
     L.ckl_read_device_status.argtypes = [vp, vp, ctypes.POINTER(i32)]
     L.ckl_read_device_status.restype = ctypes.c_int
     L.ckl_status_string.argtypes = [i32]
@@ -377,6 +382,33 @@ def selftest_wait_timeout(limit_s: float, workspace, stream=None) -> None:
                                        _stream_handle(stream))
     if rc != CKL_OK:
         raise CklError(rc, "ckl_selftest_wait_timeout")
+
+
+def dp_local_stats(workspace, stream=None):
+    """[4] fp64 device tensor after ckl_forward with ``workspace``: (sum of KL
+    over this rank's counted positions, N_r) twice; sum the first two over
+    the ranks, keep the last two (ckl_dp_local_stats)."""
+    stats = torch.empty(4, dtype=torch.float64, device=workspace.device)
+    rc = lib.ckl_dp_local_stats(_ptr(workspace), _ptr(stats), _stream_handle(stream))
+    if rc != CKL_OK:
+        raise CklError(rc, "ckl_dp_local_stats")
+    return stats
+
+
+def dp_finish(stats, grad_loss=None, stream=None):
+    """(global loss [1], this rank's upstream gradient g N_r / N [1]) from the
+    stats whose first two entries were summed over the ranks (ckl_dp_finish)."""
+    if stats.dtype != torch.float64 or not stats.is_cuda or stats.numel() != 4:
+        raise ValueError("stats must be the [4] fp64 CUDA tensor of dp_local_stats")
+    if grad_loss is not None and (grad_loss.dtype != torch.float32 or not grad_loss.is_cuda):
+        raise TypeError("grad_loss must be a CUDA float32 tensor")
+    loss = torch.empty(1, dtype=torch.float32, device=stats.device)
+    g_local = torch.empty(1, dtype=torch.float32, device=stats.device)
+    rc = lib.ckl_dp_finish(_ptr(stats), _ptr(grad_loss), _ptr(loss), _ptr(g_local),
+                           _stream_handle(stream))
+    if rc != CKL_OK:
+        raise CklError(rc, "ckl_dp_finish")
+    return loss, g_local
 
 
 def read_device_status(workspace, stream=None):

@@ -27,6 +27,8 @@ struct Header {
   int32_t status;   // CKL_DEV_* bits
   int32_t countN;   // positions that count
   uint32_t ticket;  // combine: blocks finished
+  uint32_t pad;
+  double numer;     // sum over the positions that count of KL_t (fp64), written with the loss
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -84,13 +86,12 @@ Plan plan_backward(int64_t T, int64_t d, int64_t V, const Layout& L) {
   return sliced_bytes < rows_bytes ? Plan{Cr, Sv, n} : rows_only;
 }
 
-// single_pass adds the chunk's fp32 logits [cap][zpitch] and the rows' loss terms [T].
-// eb = 4: the fp32 entry points (dZ and H_c^T in fp32; dH accumulates in the
-// caller's fp32 output, so no partial-dH buffer).
-Layout layout(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk, bool single_pass,
-              int eb = 2) {
+// The forward's part of the workspace: header, sorted teacher pairs, sum p log p,
+// the vocabulary-split partials (sized for kMaxSplits) and the combine's block
+// sums.  Every layout starts with it, at the same offsets.
+Layout forward_layout(int64_t T, int32_t K) {
   Layout L{};
-  L.eb = eb;
+  L.eb = 2;
   size_t off = kHeaderBytes;
   L.pairs = off;
   off += align256(static_cast<size_t>(T) * K * 8);
@@ -100,6 +101,18 @@ Layout layout(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk, bool si
   off += align256(static_cast<size_t>(T) * kMaxSplits * 16);
   L.blocksums = off;
   off += align256(static_cast<size_t>(cdiv(T, ckl::COMBINE_THREADS)) * 8);
+  L.total = off;
+  return L;
+}
+
+// single_pass adds the chunk's fp32 logits [cap][zpitch] and the rows' loss terms [T].
+// eb = 4: the fp32 entry points (dZ and H_c^T in fp32; dH accumulates in the
+// caller's fp32 output, so no partial-dH buffer).
+Layout layout(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk, bool single_pass,
+              int eb = 2) {
+  Layout L = forward_layout(T, K);
+  L.eb = eb;
+  size_t off = L.total;
   // dZ as 64-column panels: [ceil(V/64)][cap][64] bf16, cap = rows of the
   // largest chunk (a sliced block uses the same bytes as [Sv/64][Cr][64]).
   L.npanels = cdiv(V, 64);
@@ -379,6 +392,23 @@ int status_from_word(int32_t w) {
   return CKL_OK;
 }
 
+// Header reset, then S1 (prep) into the workspace at w8 laid out by L.
+int clear_and_prep(const int32_t* idx, const float* logp, const uint8_t* mask, int64_t T,
+                   int32_t K, int64_t V, uint8_t* w8, const Layout& L, cudaStream_t st,
+                   ckl_trace* trace) {
+  if (cudaMemsetAsync(w8, 0, kHeaderBytes, st) != cudaSuccess) return CKL_ERR_CUDA;
+  if (T > 0) {
+    Header* hdr = reinterpret_cast<Header*>(w8);
+    TraceScope ts(trace, st, CKL_KERNEL_PREP);
+    const unsigned grid = static_cast<unsigned>(cdiv(T, ckl::PREP_WARPS));
+    ckl::prep_kernel<<<grid, ckl::PREP_WARPS * 32, 0, st>>>(
+        idx, logp, mask, T, K, V, reinterpret_cast<int2*>(w8 + L.pairs),
+        reinterpret_cast<float*>(w8 + L.hp), &hdr->status, &hdr->countN);
+    if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
+  }
+  return CKL_OK;
+}
+
 // Shared front half of forward and backward: checks, header reset, prep.
 int common_prep(const void* H, const void* W, const int32_t* idx, const float* logp,
                 const uint8_t* mask, int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk,
@@ -395,18 +425,7 @@ int common_prep(const void* H, const void* W, const int32_t* idx, const float* l
   if (!device_info(di)) return CKL_ERR_CUDA;
   if (di.major != 10) return CKL_ERR_UNSUPPORTED;
   if (!encode_fn()) return CKL_ERR_CUDA;
-  uint8_t* w8 = static_cast<uint8_t*>(ws);
-  if (cudaMemsetAsync(w8, 0, kHeaderBytes, st) != cudaSuccess) return CKL_ERR_CUDA;
-  if (T > 0) {
-    Header* hdr = reinterpret_cast<Header*>(w8);
-    TraceScope ts(trace, st, CKL_KERNEL_PREP);
-    const unsigned grid = static_cast<unsigned>(cdiv(T, ckl::PREP_WARPS));
-    ckl::prep_kernel<<<grid, ckl::PREP_WARPS * 32, 0, st>>>(
-        idx, logp, mask, T, K, V, reinterpret_cast<int2*>(w8 + L.pairs),
-        reinterpret_cast<float*>(w8 + L.hp), &hdr->status, &hdr->countN);
-    if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
-  }
-  return CKL_OK;
+  return clear_and_prep(idx, logp, mask, T, K, V, static_cast<uint8_t*>(ws), L, st, trace);
 }
 
 void fill_common(TcParams& p, uint8_t* w8, const Layout& L, int64_t T, int64_t d, int64_t V,
@@ -574,28 +593,19 @@ int dhdw_block(const void* W, const uint8_t* mask, int64_t T, int64_t d, int64_t
   return launch_tc<ckl::MODE_DHDW, F32>(p, p.n5 + p.n6, di, st);
 }
 
-// The forward (S1-S4) on bf16 or fp32 H and W.
+// S2-S4 once the prep has run: the logit GEMM with its online log-sum-exp and
+// teacher gather, then the combine (lse, loss).  T = 0 only writes loss = 0.
 template <bool F32>
-int forward_impl(const void* H, const void* W, const int32_t* topk_idx, const float* topk_logp,
-                 const uint8_t* mask, int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk,
-                 float* loss, float* lse, void* workspace, size_t workspace_bytes, void* stream,
-                 ckl_trace* trace) {
+int forward_gemm_combine(const void* H, const void* W, const uint8_t* mask, int64_t T, int64_t d,
+                         int64_t V, int32_t K, float* loss, float* lse, uint8_t* w8,
+                         const Layout& L, const DevInfo& di, cudaStream_t st, ckl_trace* trace) {
   constexpr int eb = F32 ? 4 : 2;
-  if (!loss || !aligned4(loss) || (T > 0 && (!lse || !aligned4(lse)))) return CKL_ERR_INVALID_ARG;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  DevInfo di;
-  Layout L;
-  int rc = common_prep(H, W, topk_idx, topk_logp, mask, T, d, V, K, chunk, workspace,
-                       workspace_bytes, st, trace, di, L, false, eb);
-  if (rc != CKL_OK) return rc;
-  uint8_t* w8 = static_cast<uint8_t*>(workspace);
   Header* hdr = reinterpret_cast<Header*>(w8);
   if (T == 0) {
     TraceScope ts(trace, st, CKL_KERNEL_OTHER);
     ckl::zero_loss_kernel<<<1, 1, 0, st>>>(loss);
     return cudaGetLastError() == cudaSuccess ? CKL_OK : CKL_ERR_CUDA;
   }
-
   TcParams p;
   std::memset(&p, 0, sizeof(p));
   fill_common(p, w8, L, T, d, V, K, mask);
@@ -618,10 +628,28 @@ int forward_impl(const void* H, const void* W, const int32_t* topk_idx, const fl
     ckl::combine_kernel<<<grid, ckl::COMBINE_THREADS, 0, st>>>(
         reinterpret_cast<const float4*>(w8 + L.partials), p.S,
         reinterpret_cast<const float*>(w8 + L.hp), mask, T, lse,
-        reinterpret_cast<double*>(w8 + L.blocksums), &hdr->ticket, &hdr->countN, loss);
+        reinterpret_cast<double*>(w8 + L.blocksums), &hdr->ticket, &hdr->countN, loss,
+        &hdr->numer);
     if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
   }
   return CKL_OK;
+}
+
+// The forward (S1-S4) on bf16 or fp32 H and W.
+template <bool F32>
+int forward_impl(const void* H, const void* W, const int32_t* topk_idx, const float* topk_logp,
+                 const uint8_t* mask, int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk,
+                 float* loss, float* lse, void* workspace, size_t workspace_bytes, void* stream,
+                 ckl_trace* trace) {
+  if (!loss || !aligned4(loss) || (T > 0 && (!lse || !aligned4(lse)))) return CKL_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DevInfo di;
+  Layout L;
+  int rc = common_prep(H, W, topk_idx, topk_logp, mask, T, d, V, K, chunk, workspace,
+                       workspace_bytes, st, trace, di, L, false, F32 ? 4 : 2);
+  if (rc != CKL_OK) return rc;
+  return forward_gemm_combine<F32>(H, W, mask, T, d, V, K, loss, lse,
+                                  static_cast<uint8_t*>(workspace), L, di, st, trace);
 }
 
 // The blocked backward (S0, S1, S5-S7) on bf16 or fp32 H and W; dH is bf16
@@ -841,7 +869,8 @@ int ckl_forward_backward(const uint16_t* H, const uint16_t* W, const int32_t* to
   }
   {
     TraceScope ts(trace, st, CKL_KERNEL_FWD_COMBINE);
-    ckl::rowsum_loss_kernel<<<1, ckl::ROWSUM_THREADS, 0, st>>>(rowloss, T, &hdr->countN, loss);
+    ckl::rowsum_loss_kernel<<<1, ckl::ROWSUM_THREADS, 0, st>>>(rowloss, T, &hdr->countN, loss,
+                                                                &hdr->numer);
     if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
   }
   return CKL_OK;
@@ -888,6 +917,25 @@ int ckl_selftest_wait_timeout(int64_t limit_ns, void* workspace, size_t workspac
   return cudaGetLastError() == cudaSuccess ? CKL_OK : CKL_ERR_CUDA;
 }
 
+int ckl_dp_local_stats(const void* workspace, double* stats, void* stream) {
+  if (!workspace || !stats || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(stats) & 7u))
+    return CKL_ERR_INVALID_ARG;
+  const Header* hdr = static_cast<const Header*>(workspace);
+  ckl::dp_local_stats_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(&hdr->numer,
+                                                                          &hdr->countN, stats);
+  return cudaGetLastError() == cudaSuccess ? CKL_OK : CKL_ERR_CUDA;
+}
+
+int ckl_dp_finish(const double* stats, const float* grad_loss, float* loss, float* grad_local,
+                  void* stream) {
+  if (!stats || !loss || !grad_local || (reinterpret_cast<uintptr_t>(stats) & 7u) ||
+      !aligned4(loss) || !aligned4(grad_local) || !aligned4(grad_loss))
+    return CKL_ERR_INVALID_ARG;
+  ckl::dp_finish_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(stats, grad_loss, loss,
+                                                                      grad_local);
+  return cudaGetLastError() == cudaSuccess ? CKL_OK : CKL_ERR_CUDA;
+}
+
 int ckl_read_device_status(const void* workspace, void* stream, int32_t* device_status) {
   if (!workspace || !device_status) return CKL_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -922,27 +970,55 @@ int32_t ckl_version(void) { return kVersion; }
 // Forward with library-owned static scratch, for callers that cannot
 // allocate device memory.  The buffer is a file-scope device array; host code
 // must never hand its name to a kernel (on the host the name is only a
-// stand-in), so each device's real address is looked up once with
-// cudaGetSymbolAddress and kept.
+// stand-in), so the real device address is looked up with
+// cudaGetSymbolAddress on each device and kept.
 namespace {
 
 static __device__ __align__(256) uint8_t g_static_scratch[CKL_STATIC_SCRATCH_BYTES];
 
 __global__ void copy_status_kernel(const int32_t* src, int32_t* dst) { *dst = *src; }
 
-// Device address of g_static_scratch on the current device, or null.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+CtxGetCurrentFn ctx_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+// Device address of g_static_scratch on the current device, or null.  The
+// address is kept per device together with the context it was looked up in;
+// when the current context differs (after cudaDeviceReset, say, the module
+// is loaded again) it is looked up again.
 void* static_scratch_ptr() {
   static std::mutex mu;
-  static void* ptrs[64] = {};
+  struct Entry {
+    CUcontext ctx;
+    void* ptr;
+  };
+  static Entry cache[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
   std::lock_guard<std::mutex> lock(mu);
-  if (ptrs[dev] == nullptr) {
+  Entry& e = cache[dev];
+  CUcontext ctx = nullptr;
+  CtxGetCurrentFn get = ctx_current_fn();
+  const bool known = get && get(&ctx) == CUDA_SUCCESS && ctx != nullptr;
+  if (e.ptr == nullptr || !known || ctx != e.ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess) return nullptr;
-    ptrs[dev] = p;
+    // the lookup makes the device's primary context current if none was
+    if (get && get(&ctx) == CUDA_SUCCESS) e.ctx = ctx;
+    e.ptr = p;
   }
-  return ptrs[dev];
+  return e.ptr;
 }
 
 }  // namespace
@@ -960,70 +1036,27 @@ int ckl_forward_static_scratch(const uint16_t* H, const uint16_t* W, const int32
       !aligned4(lse) || !aligned4(device_status))
     return CKL_ERR_INVALID_ARG;
   if (K > ckl::PREP_MAXK) return CKL_ERR_UNSUPPORTED;
+  // The forward's own layout (as in ckl_forward, partials sized for the largest
+  // split count), so the limit depends on T and K only; checked before any
+  // device call.
+  const Layout L = forward_layout(T, K);
+  if (L.total > CKL_STATIC_SCRATCH_BYTES) return CKL_ERR_WORKSPACE;
   DevInfo di;
   if (!device_info(di)) return CKL_ERR_CUDA;
   if (di.major != 10) return CKL_ERR_UNSUPPORTED;
   if (!encode_fn()) return CKL_ERR_CUDA;
-
-  // Forward-only layout, sized with the split count this device will use.
-  const int64_t n_rb = cdiv(T, kMB);
-  const int64_t n_vt = cdiv(V, ckl::BN_V);
-  const int S = (T > 0) ? choose_splits(n_rb, n_vt, di.slots[ckl::MODE_FWD]) : 1;
-  size_t off = kHeaderBytes;
-  const size_t o_pairs = off;
-  off += align256(static_cast<size_t>(T) * K * 8);
-  const size_t o_hp = off;
-  off += align256(static_cast<size_t>(T) * 4);
-  const size_t o_part = off;
-  off += align256(static_cast<size_t>(T) * S * 16);
-  const size_t o_bs = off;
-  off += align256(static_cast<size_t>(cdiv(T, ckl::COMBINE_THREADS)) * 8);
-  if (off > CKL_STATIC_SCRATCH_BYTES) return CKL_ERR_WORKSPACE;
-
   uint8_t* w8 = static_cast<uint8_t*>(static_scratch_ptr());
   if (!w8) return CKL_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  Header* hdr = reinterpret_cast<Header*>(w8);
-  // The buffer still holds the previous call's words: clear the header.
-  if (cudaMemsetAsync(w8, 0, kHeaderBytes, st) != cudaSuccess) return CKL_ERR_CUDA;
-  if (T == 0) {
-    ckl::zero_loss_kernel<<<1, 1, 0, st>>>(loss);
-  } else {
-    ckl::prep_kernel<<<static_cast<unsigned>(cdiv(T, ckl::PREP_WARPS)), ckl::PREP_WARPS * 32, 0,
-                       st>>>(topk_idx, topk_logp, mask, T, K, V,
-                             reinterpret_cast<int2*>(w8 + o_pairs),
-                             reinterpret_cast<float*>(w8 + o_hp), &hdr->status, &hdr->countN);
-    if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
-    TcParams p;
-    std::memset(&p, 0, sizeof(p));
-    p.T = static_cast<int32_t>(T);
-    p.d = static_cast<int32_t>(d);
-    p.V = static_cast<int32_t>(V);
-    p.K = K;
-    p.n_vt = static_cast<int32_t>(n_vt);
-    p.pairs = reinterpret_cast<const int2*>(w8 + o_pairs);
-    p.partials = reinterpret_cast<float4*>(w8 + o_part);
-    p.mask = mask;
-    p.status = &hdr->status;
-    p.countN = &hdr->countN;
-    p.rows = static_cast<int32_t>(T);
-    p.row0 = 0;
-    p.n_rb = static_cast<int32_t>(n_rb);
-    p.S = S;
-    p.n_units = p.n_rb * S;
-    if (!map2d(&p.tm[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, H, d, T, d * 2, ckl::BK, ckl::BM,
-               CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !map2d(&p.tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, V, d * 2, ckl::BK,
-               ckl::BN_V / kSlotCTAs, CU_TENSOR_MAP_SWIZZLE_128B))
-      return CKL_ERR_CUDA;
-    if (launch_tc<ckl::MODE_FWD>(p, p.n_units, di, st) != CKL_OK) return CKL_ERR_CUDA;
-    ckl::combine_kernel<<<static_cast<unsigned>(cdiv(T, ckl::COMBINE_THREADS)),
-                          ckl::COMBINE_THREADS, 0, st>>>(
-        reinterpret_cast<const float4*>(w8 + o_part), S, reinterpret_cast<const float*>(w8 + o_hp),
-        mask, T, lse, reinterpret_cast<double*>(w8 + o_bs), &hdr->ticket, &hdr->countN, loss);
-  }
-  if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
+  // The buffer still holds the previous call's words: the header is cleared
+  // before the prep, exactly as in ckl_forward, and the GEMM and combine
+  // overwrite every other word they read.
+  int rc = clear_and_prep(topk_idx, topk_logp, mask, T, K, V, w8, L, st, nullptr);
+  if (rc != CKL_OK) return rc;
+  rc = forward_gemm_combine<false>(H, W, mask, T, d, V, K, loss, lse, w8, L, di, st, nullptr);
+  if (rc != CKL_OK) return rc;
   if (device_status) {
+    Header* hdr = reinterpret_cast<Header*>(w8);
     copy_status_kernel<<<1, 1, 0, st>>>(&hdr->status, device_status);
     if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
   }

@@ -209,7 +209,8 @@ constexpr int COMBINE_THREADS = 256;
 __global__ void __launch_bounds__(COMBINE_THREADS)
 combine_kernel(const float4* __restrict__ partials, int S, const float* __restrict__ Hp,
                const uint8_t* __restrict__ mask, int64_t T, float* __restrict__ lse,
-               double* block_sums, unsigned int* ticket, const int* countN, float* loss) {
+               double* block_sums, unsigned int* ticket, const int* countN, float* loss,
+               double* numer) {
   __shared__ double s_w[COMBINE_THREADS / 32];
   __shared__ bool s_last;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * COMBINE_THREADS + threadIdx.x;
@@ -248,6 +249,7 @@ combine_kernel(const float4* __restrict__ partials, int S, const float* __restri
     for (unsigned b = 0; b < gridDim.x; ++b) total += bs[b];
     const int n = *reinterpret_cast<const volatile int*>(countN);
     *loss = (n > 0) ? static_cast<float>(total / static_cast<double>(n)) : 0.f;
+    *numer = total;
   }
 }
 
@@ -276,6 +278,28 @@ transpose_rows_kernel(const E* __restrict__ Hc, int rows, int d, E* __restrict__
 
 // Loss of an empty batch (T = 0).
 __global__ void zero_loss_kernel(float* loss) { *loss = 0.f; }
+
+// Data parallel, after the forward on this rank's rows: (sum of KL over the
+// rank's positions that count, N_r), twice: one copy for the sum over
+// ranks, one kept.
+__global__ void dp_local_stats_kernel(const double* numer, const int* countN, double* stats) {
+  const double n = static_cast<double>(*countN);
+  stats[0] = *numer;
+  stats[1] = n;
+  stats[2] = *numer;
+  stats[3] = n;
+}
+
+// Data parallel, after stats[0..1] were summed over the ranks: the global
+// mean loss, and the upstream gradient this rank's backward takes so that
+// its own 1 / N_r scale becomes g / N (0 when no position counts anywhere).
+__global__ void dp_finish_kernel(const double* stats, const float* grad_loss, float* loss,
+                                 float* grad_local) {
+  const double num = stats[0], n = stats[1], n_r = stats[3];
+  const double g = (grad_loss != nullptr) ? static_cast<double>(*grad_loss) : 1.0;
+  *loss = (n > 0.0) ? static_cast<float>(num / n) : 0.f;
+  *grad_local = (n > 0.0) ? static_cast<float>(g * n_r / n) : 0.f;
+}
 
 // Self-test of the bounded waits: one CTA waits, with the kernels' own wait,
 // on an mbarrier that nothing arrives on.  The wait runs out after limit_ns,
@@ -390,7 +414,8 @@ dh_convert_kernel(const float4* __restrict__ src, int64_t n4, uint2* __restrict_
 constexpr int ROWSUM_THREADS = 1024;
 
 __global__ void __launch_bounds__(ROWSUM_THREADS)
-rowsum_loss_kernel(const float* __restrict__ rowloss, int64_t T, const int* countN, float* loss) {
+rowsum_loss_kernel(const float* __restrict__ rowloss, int64_t T, const int* countN, float* loss,
+                   double* numer) {
   __shared__ double s[ROWSUM_THREADS];
   double v = 0.0;
   for (int64_t t = threadIdx.x; t < T; t += ROWSUM_THREADS) v += static_cast<double>(rowloss[t]);
@@ -403,6 +428,7 @@ rowsum_loss_kernel(const float* __restrict__ rowloss, int64_t T, const int* coun
   if (threadIdx.x == 0) {
     const int n = *countN;
     *loss = (n > 0) ? static_cast<float>(s[0] / static_cast<double>(n)) : 0.f;
+    *numer = s[0];
   }
 }
 

@@ -131,7 +131,12 @@ CKL_API int ckl_backward_plan(int64_t T, int64_t d, int64_t V, int32_t K, int64_
 
 /*
  * Forward: the mean KL over the positions that count, and lse for EVERY row
- * (masked rows too).
+ * (masked rows too).  The pages' forward pass: hidden states are projected
+ * to logits a piece at a time and each piece is folded into the running
+ * loss and dropped ("Дистилляция LLM на одной GPU: offline-кэш и chunked KL
+ * loss", section «Два приёма»); here the pieces are 128 x 256 tensor-core
+ * tiles whose epilogue keeps an online log-sum-exp and gathers the teacher
+ * ids, so no logit is ever stored.
  *   H          [T, d] bf16  student hidden states
  *   W          [V, d] bf16  output head
  *   topk_idx   [T, K] int32 cached teacher token ids (repeats allowed; each
@@ -153,8 +158,12 @@ CKL_API int ckl_forward(const uint16_t* H, const uint16_t* W, const int32_t* top
                 size_t workspace_bytes, void* stream, ckl_trace* trace);
 
 /*
- * Backward by recomputation, one block at a time: each block's logits are
- * rebuilt from H and W, turned into the unscaled logit gradient
+ * Backward by recomputation: the backward rebuilds each chunk's logits
+ * instead of keeping them ("LLMのための効率的な知識蒸留...", section
+ * "2つのシステム変更"), and the logit gradient is the closed form the paper
+ * mentions ("Tối ưu hóa chi phí chưng cất tri thức ...", closing paragraph,
+ * after "Mô hình học sinh thu được").  One block at a time, each block's
+ * logits are rebuilt from H and W, turned into the unscaled logit gradient
  * dZ = exp(z - lse) - scatter(p) (0 on rows that do not count), stored as
  * bf16 in the workspace (at most chunk x V entries), then fed to two
  * tensor-core GEMMs: dH_c = s dZ_c W and dW (+)= s dZ_c^T H_c, with
@@ -264,6 +273,31 @@ CKL_API int ckl_selftest_wait_timeout(int64_t limit_ns, void* workspace, size_t 
                                       void* stream);
 
 /*
+ * Data-parallel training over T (no counterpart in the pages, which run on
+ * one GPU): each rank holds its own rows of the batch and all of W, and the
+ * loss is the mean over the positions that count on every rank.
+ *
+ * ckl_dp_local_stats: after ckl_forward on this rank's rows with
+ * `workspace`, writes (device memory, 8-byte aligned, fp64)
+ *   stats[0] = stats[2] = sum over this rank's counted positions of KL_t,
+ *   stats[1] = stats[3] = N_r, the number of those positions.
+ * The step then sums stats[0..1] over the ranks (an all-reduce of two
+ * doubles) and keeps stats[2..3] as they are.
+ *
+ * ckl_dp_finish: from the summed stats[0..1] and this rank's N_r (stats[3]),
+ * writes loss = stats[0] / stats[1] (0 when no position counts on any rank)
+ * and grad_local = g N_r / N (fp32, device; g = *grad_loss, NULL = 1; 0 when
+ * N = 0).  ckl_backward on this rank with grad_loss = grad_local scales by
+ * g / N, so its dH rows are final and its dW is this rank's share of the
+ * gradient; summing dW over the ranks gives the global dW.
+ * Both enqueue one tiny kernel on `stream` and return CKL_ERR_INVALID_ARG for
+ * null or misaligned pointers.
+ */
+CKL_API int ckl_dp_local_stats(const void* workspace, double* stats, void* stream);
+CKL_API int ckl_dp_finish(const double* stats, const float* grad_loss, float* loss,
+                          float* grad_local, void* stream);
+
+/*
  * Reads the device status word of the last call that used `workspace`:
  * synchronises `stream`, copies the word to *device_status (a host pointer)
  * and returns the matching ckl_status (CKL_OK when the word is 0).
@@ -311,18 +345,22 @@ CKL_API int32_t ckl_version(void);
  * Same inputs and outputs as ckl_forward (there is no `chunk`: the forward
  * never holds per-chunk logits).  The scratch lives in one library-owned
  * static device buffer of CKL_STATIC_SCRATCH_BYTES, present on every GPU
- * that loads the library until the process exits.  It must hold
- * 256 + T*K*8 + T*4 + T*S*16 + ceil(T/256)*8 bytes (each term rounded up to
- * 256), where S <= 64 is the number of vocabulary splits the forward picks
- * for this GPU (37 for T = 8192 on a 148-SM B200): about 23 000 tokens at
- * K = 100.  Larger problems return CKL_ERR_WORKSPACE before anything is
- * enqueued.  Nothing is allocated: no cudaMalloc, no cudaFree.
+ * that loads the library until the process exits.  A problem fits when
+ *   256 + r(8 K T) + r(4 T) + r(1024 T) + r(8 ceil(T / 256))
+ *       <= CKL_STATIC_SCRATCH_BYTES,   r(x) = x rounded up to a multiple of 256
+ * (the sorted teacher pairs, sum p log p, the vocabulary-split partials and
+ * the loss's block sums), whatever the GPU: T <= 18 355 at K = 100.  Larger
+ * problems return CKL_ERR_WORKSPACE before anything is enqueued, and before
+ * any CUDA call.  Nothing is allocated: no cudaMalloc, no cudaFree.  The
+ * results are those of ckl_forward on the same inputs (the same launches).
  *
- * The first call on each device looks up the buffer's device address
- * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture begins.  Every call on a device shares the one
- * buffer, which keeps the previous call's contents (the call clears what
- * must start at zero): calls that overlap on the GPU -- on different
+ * On each device, the first call looks up the buffer's device address
+ * (cudaGetSymbolAddress) with that device current, and keeps it with the
+ * CUDA context it was looked up in; a call in another context of that device
+ * (after cudaDeviceReset) looks it up again.  Make the first call on a
+ * device before any stream capture begins.  Every call on a device shares
+ * the one buffer, which keeps the previous call's contents (the call clears
+ * what must start at zero): calls that overlap on the GPU -- on different
  * streams, or from different host threads -- race and give wrong results.
  *
  *   device_status  [1] int32, device memory, may be NULL: receives the

@@ -23,7 +23,8 @@ def ckl():
 
 def test_header_declares_the_entry_points():
     assert _declared() == ["ckl_backward", "ckl_backward_ex", "ckl_backward_f32",
-                           "ckl_backward_plan", "ckl_forward", "ckl_forward_backward",
+                           "ckl_backward_plan", "ckl_dp_finish", "ckl_dp_local_stats",
+                           "ckl_forward", "ckl_forward_backward",
                            "ckl_forward_f32", "ckl_forward_static_scratch",
                            "ckl_read_device_status", "ckl_selftest_wait_timeout",
                            "ckl_single_pass_workspace_bytes",
@@ -163,3 +164,25 @@ def test_host_checks_return_before_any_device_work(ckl):
     assert L.ckl_topk_cache(fake, 4, 100, 0, fake, fake, nul, nul) == 1
     assert L.ckl_topk_cache(fake, 4, 100, 101, fake, fake, nul, nul) == 1
     assert L.ckl_topk_cache(fake, 4, 5000, 3000, fake, fake, nul, nul) == 2
+    # data-parallel stats: null or misaligned buffers
+    L.ckl_dp_local_stats.argtypes = [ctypes.c_void_p] * 3
+    L.ckl_dp_finish.argtypes = [ctypes.c_void_p] * 5
+    assert L.ckl_dp_local_stats(nul, fake, nul) == 1
+    assert L.ckl_dp_local_stats(fake, ctypes.c_void_p(4100), nul) == 1
+    assert L.ckl_dp_finish(nul, nul, fake, fake, nul) == 1
+    assert L.ckl_dp_finish(fake, nul, fake, ctypes.c_void_p(4097), nul) == 1
+
+
+def test_static_scratch_limit_is_checked_on_the_host(ckl):
+    """ckl_forward_static_scratch rejects a problem one token past the limit
+    ckl.h states (T = 18 355 at K = 100) before any CUDA call.  Without a
+    device, a problem at the limit gets as far as the device query."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is visible: the GPU test checks the limit with real buffers")
+    vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+    f = ctypes.CDLL(ckl.LIB_PATH).ckl_forward_static_scratch
+    f.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, vp, vp, vp, vp]
+    fake = ctypes.c_void_p(1 << 20)
+    assert f(fake, fake, fake, fake, None, 18356, 64, 1000, 100, fake, fake, None, None) == 3
+    assert f(fake, fake, fake, fake, None, 18355, 64, 1000, 100, fake, fake, None, None) == 4

@@ -44,3 +44,22 @@ def test_rank_seeds_differ_and_warmup_contract():
     assert len({bench.rank_seed(0, r) for r in range(8)}) == 8
     with pytest.raises(SystemExit):
         bench.main(["--warmup", "2"])
+
+
+def test_clock_summary_keeps_only_samples_inside_the_timed_region():
+    # idle samples before and after the window (1965 MHz) must not enter the
+    # median; the loaded ones inside it (1300-1400 MHz, power cap) do
+    samples = [(0.0, 1965.0, 1965.0, 150.0, set()), (0.1, 1965.0, 1965.0, 150.0, set())]
+    samples += [(1.0 + 0.02 * i, 1300.0 + 5 * i, 1965.0, 990.0, {"sw_power_cap"})
+                for i in range(21)]
+    samples += [(2.0, 1965.0, 1965.0, 200.0, set())]
+    s = bench.summarise_clocks(samples, 0.9, 1.5, "test")
+    assert s["samples"] == 21 and s["sm_mhz"] == 1350.0 and s["sm_min_mhz"] == 1300.0
+    assert s["sm_max_mhz"] == 1965.0 and s["reasons"] == ["sw_power_cap"]
+    assert s["power_w"] == 990.0
+    assert bench.summarise_clocks(samples, 5.0, 6.0) is None
+
+
+def test_cpu_description_names_the_host():
+    model, n = bench.cpu_description()
+    assert n >= 1 and (model is None or isinstance(model, str))

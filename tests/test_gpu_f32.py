@@ -36,18 +36,23 @@ def _dev(c, mask="config"):
 def run_f32(ckl, c, chunk=None, g=None, dW0=None):
     H, W, idx, logp, m = _dev(c)
     chunk = chunk or c["chunk"]
-    loss, lse = ckl.forward_f32(H, W, idx, logp, m, chunk)
+    T, d, V, K = c["T"], c["d"], c["V"], c["K"]
+    ws = torch.empty(ckl.lib.ckl_workspace_bytes_f32(T, d, V, K, chunk), dtype=torch.uint8,
+                     device="cuda")
+    loss, lse = ckl.forward_f32(H, W, idx, logp, m, chunk, workspace=ws)
+    st_f = ckl.read_device_status(ws)
     gl = None if g is None else torch.tensor([g], dtype=torch.float32, device="cuda")
     dW = None
     if dW0 is not None:
         dW = torch.from_numpy(np.ascontiguousarray(dW0, dtype=np.float32)).cuda()
     dH, dW = ckl.backward_f32(H, W, idx, logp, m, lse, grad_loss=gl, chunk=chunk, dW=dW,
-                              accumulate_dW=dW0 is not None)
+                              accumulate_dW=dW0 is not None, workspace=ws)
+    st_b = ckl.read_device_status(ws)
     torch.cuda.synchronize()
-    st = (0, 0)
+    assert st_f[0] == 0 and st_b[0] == 0, (st_f, st_b)
     return dict(loss=float(loss.item()), lse=lse.cpu().numpy().astype(np.float64),
                 dH=dH.cpu().numpy().astype(np.float64), dW=dW.cpu().numpy().astype(np.float64),
-                status_f=st, status_b=st)
+                status_f=st_f, status_b=st_b)
 
 
 def _ref(c, g=1.0):
@@ -73,9 +78,15 @@ def assert_parity_tf32(out, ref, c, tag=""):
 
 
 def test_tiny_fp32_config(gpu_lib):
+    # the tiny workload is an fp32 case: besides the tf32-derived bounds, its
+    # results meet the contract tolerances themselves (loss 1e-3 relative,
+    # lse 2e-3 absolute, dH and dW 1e-2 relative Frobenius)
+    from gpu_util import assert_parity
     c = make_config("tiny", fp32=True)
     assert c["H"].dtype == np.float32
-    assert_parity_tf32(run_f32(gpu_lib, c), _ref(c), c, "fp32 tiny")
+    out, ref = run_f32(gpu_lib, c), _ref(c)
+    assert_parity_tf32(out, ref, c, "fp32 tiny")
+    assert_parity(out, ref, "fp32 tiny, contract tolerances")
 
 
 @pytest.mark.parametrize("chunk", [100, 300])

@@ -79,6 +79,34 @@ def test_too_many_ties_is_reported_and_other_rows_are_right(gpu_lib):
     assert np.abs(logp[rows] - ref_logp).max() <= LOGP_ATOL
 
 
+@pytest.mark.parametrize("V", [1001, 1024])
+def test_many_rows_per_cta_heavy_ties_every_row(gpu_lib, V):
+    # far more rows than the launch has CTAs, so every CTA handles many rows
+    # in turn (state left from a previous row would show); logits on a 0.25
+    # grid tie often, also at the K-th value; V = 1001 takes the scalar loads
+    rng = np.random.default_rng(7)
+    z = np.round(rng.normal(0, 2, (1500, V)) * 4) / 4
+    z[1400] = 0.5                                   # a row of equal logits, late
+    z[1401, ::3] = 3.0                              # many ties above the K-th value
+    _check(gpu_lib, f32_to_bf16_bits(z.astype(np.float32)), 16)
+
+
+def test_teacher_sized_many_rows_sampled(gpu_lib):
+    # 1500 teacher-sized rows (several per CTA); ids checked exactly on a
+    # seeded sample of 160 rows, most of them past the first row of each CTA,
+    # plus a late row whose top values tie heavily
+    rng = np.random.default_rng(8)
+    T, V, K = 1500, 128256, 100
+    z = rng.normal(0, 2, (T, V)).astype(np.float32)
+    z[1333, rng.choice(V, 400, replace=False)] = 7.5      # 400 equal top logits
+    bits = f32_to_bf16_bits(z)
+    del z
+    sample = np.unique(np.concatenate([rng.choice(296, 32, replace=False),
+                                       296 + rng.choice(T - 296, 128, replace=False),
+                                       [1333, T - 1]]))
+    _check(gpu_lib, bits, K, rows=sample)
+
+
 def test_cache_feeds_the_loss(gpu_lib):
     # The producer's output is a valid teacher cache for the fused loss.
     from ckl_synth import make_inputs

@@ -77,17 +77,35 @@ def test_two_gloo_ranks(tmp_path):
 class _OracleOps:
     """Stands in for the CUDA library on CPU: the oracle's dense forward and
     backward of the rank's own rows, with the library's interface (fp32/bf16
-    outputs, dW written range by range with on_dw_ready after each range)."""
+    outputs, the fp64 (sum of KL, N_r) stats, dW written range by range with
+    on_dw_ready after each range)."""
 
     def __init__(self, c):
         self.c = c
+        self.fwd = None
+
+    def new_workspace(self, T, d, V, K, chunk, device=None):
+        return torch.zeros(1, dtype=torch.uint8)
 
     def forward(self, H, W, idx, logp, mask, chunk, workspace=None):
         import oracle
         c = self.c
         r = oracle.dense(c["H"], c["W"], c["idx"], c["logp"], c["mask"], g=1.0)
+        self.fwd = r
         return (torch.tensor([r["loss"]], dtype=torch.float32),
                 torch.from_numpy(r["lse"].astype(np.float32)))
+
+    def dp_local_stats(self, workspace):
+        r = self.fwd
+        num = r["loss"] * r["N"]
+        return torch.tensor([num, r["N"], num, r["N"]], dtype=torch.float64)
+
+    def dp_finish(self, stats, grad_loss=None):
+        num, n, n_r = float(stats[0]), float(stats[1]), float(stats[3])
+        g = 1.0 if grad_loss is None else float(grad_loss.item())
+        loss = num / n if n > 0 else 0.0
+        return (torch.tensor([loss], dtype=torch.float32),
+                torch.tensor([g * n_r / n if n > 0 else 0.0], dtype=torch.float32))
 
     def backward(self, H, W, idx, logp, mask, lse, grad_loss=None, chunk=1024, dW=None,
                  workspace=None, on_dw_ready=None):
@@ -120,7 +138,9 @@ def _dp_worker(rank, world, port, out_dir):
         Wt = torch.zeros(60, 16)
         g = torch.tensor([0.7], dtype=torch.float32)
         mt = torch.from_numpy(np.ascontiguousarray(part["mask"], dtype=np.uint8))
-        loss, lse, dH, dW = dp_forward_backward(Ht, Wt, None, None, mask=mt, chunk=8,
+        it = torch.from_numpy(part["idx"])
+        lt = torch.from_numpy(part["logp"])
+        loss, lse, dH, dW = dp_forward_backward(Ht, Wt, it, lt, mask=mt, chunk=8,
                                                 grad_loss=g, ops=ops)
         np.savez(os.path.join(out_dir, f"dp{rank}.npz"), loss=loss.numpy(), dH=dH.numpy(),
                  dW=dW.numpy(), lo=lo, hi=hi)

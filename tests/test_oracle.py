@@ -28,6 +28,25 @@ def _values(c):
     return oracle.widen_bf16(c["H"]), oracle.widen_bf16(c["W"])
 
 
+# --- the input widening -------------------------------------------------------
+
+def test_widen_bf16_every_bit_pattern_matches_torch():
+    # All 65 536 bf16 patterns, against torch's own bf16 -> fp64 conversion:
+    # finite values equal (signed zeros and subnormals included), infinities
+    # with their sign, NaN patterns NaN.
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    got = oracle.widen_bf16(bits)
+    ref = torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).double().numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert np.array_equal(np.signbit(got[~nan]), np.signbit(ref[~nan]))
+    assert got.dtype == np.float64 and got.shape == bits.shape
+    # a few by hand: 1.0, -2.0, the smallest subnormal, the largest finite
+    assert oracle.widen_bf16(np.array([0x3F80, 0xC000, 0x0001, 0x7F7F], np.uint16)).tolist() == [
+        1.0, -2.0, 2.0 ** -133, (2 - 2 ** -7) * 2.0 ** 127]
+
+
 # --- Gibbs' inequality and the zero case -----------------------------------
 
 def test_kl_nonnegative_per_row():
