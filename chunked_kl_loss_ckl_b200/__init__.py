@@ -24,7 +24,8 @@ __all__ = [
     "forward", "backward", "read_device_status", "status_string", "chunked_kl_loss",
     "topk_cache", "single_pass_workspace_bytes", "forward_backward", "backward_plan",
     "DW_READY_FN", "forward_f32", "backward_f32", "selftest_wait_timeout", "dp_local_stats",
-    "dp_finish",
+    "dp_finish", "forward_vocab_shard", "combine_vocab_shards", "backward_vocab_shard",
+    "dh_to_bf16",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libckl.so")
@@ -96,6 +97,16 @@ def _load() -> ctypes.CDLL:
     L.ckl_topk_cache.restype = ctypes.c_int
     L.ckl_selftest_wait_timeout.argtypes = [i64, vp, sz, vp]
     L.ckl_selftest_wait_timeout.restype = ctypes.c_int
+    L.ckl_forward_vocab_shard.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i32, i64,
+                                          vp, vp, sz, vp, tr]
+    L.ckl_forward_vocab_shard.restype = ctypes.c_int
+    L.ckl_combine_vocab_shards.argtypes = [vp, i32, vp, i64, i32, vp, vp, vp, sz, vp, tr]
+    L.ckl_combine_vocab_shards.restype = ctypes.c_int
+    L.ckl_backward_vocab_shard.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i32, i64,
+                                           vp, vp, vp, vp, i32, vp, sz, vp, tr]
+    L.ckl_backward_vocab_shard.restype = ctypes.c_int
+    L.ckl_dh_to_bf16.argtypes = [vp, vp, i64, vp]
+    L.ckl_dh_to_bf16.restype = ctypes.c_int
     L.ckl_dp_local_stats.argtypes = [vp, vp, vp]
     L.ckl_dp_local_stats.restype = ctypes.c_int
     L.ckl_dp_finish.argtypes = [vp, vp, vp, vp, vp]
@@ -382,6 +393,82 @@ def selftest_wait_timeout(limit_s: float, workspace, stream=None) -> None:
                                        _stream_handle(stream))
     if rc != CKL_OK:
         raise CklError(rc, "ckl_selftest_wait_timeout")
+
+
+def _check_shard(H, W_shard, idx, logp, mask, V, v_begin, v_end):
+    T, d, Vs, K = _check_inputs(H, W_shard, idx, logp, mask)
+    if not (0 <= v_begin < v_end <= V) or Vs != v_end - v_begin:
+        raise ValueError("W_shard must hold rows [v_begin, v_end) of a V-row head")
+    return T, d, Vs, K
+
+
+def forward_vocab_shard(H, W_shard, idx, logp, mask, V: int, v_begin: int, v_end: int,
+                        chunk: int = 1024, workspace=None, stream=None,
+                        trace: Trace | None = None):
+    """This vocabulary shard's per-row partials [T, 4] (ckl_forward_vocab_shard)
+    and the workspace that ``combine_vocab_shards`` then reads."""
+    T, d, Vs, K = _check_shard(H, W_shard, idx, logp, mask, V, v_begin, v_end)
+    if workspace is None:
+        workspace = new_workspace(T, d, Vs, K, chunk, H.device)
+    part = torch.empty(T, 4, dtype=torch.float32, device=H.device)
+    rc = lib.ckl_forward_vocab_shard(_ptr(H), _ptr(W_shard), _ptr(idx), _ptr(logp), _ptr(mask),
+                                     T, d, V, v_begin, v_end, K, chunk, _ptr(part),
+                                     _ptr(workspace), workspace.numel(), _stream_handle(stream),
+                                     _trace_ptr(trace))
+    if rc != CKL_OK:
+        raise CklError(rc, "ckl_forward_vocab_shard")
+    return part, workspace
+
+
+def combine_vocab_shards(gathered, mask, K: int, workspace, stream=None,
+                         trace: Trace | None = None):
+    """(loss [1], lse [T]) from every shard's partials, gathered [g, T, 4]."""
+    g, T, four = gathered.shape
+    if four != 4 or gathered.dtype != torch.float32 or not gathered.is_contiguous():
+        raise ValueError("gathered must be a contiguous float32 [g, T, 4] tensor")
+    loss = torch.empty(1, dtype=torch.float32, device=gathered.device)
+    lse = torch.empty(T, dtype=torch.float32, device=gathered.device)
+    rc = lib.ckl_combine_vocab_shards(_ptr(gathered), g, _ptr(mask), T, K, _ptr(loss), _ptr(lse),
+                                      _ptr(workspace), workspace.numel(), _stream_handle(stream),
+                                      _trace_ptr(trace))
+    if rc != CKL_OK:
+        raise CklError(rc, "ckl_combine_vocab_shards")
+    return loss, lse
+
+
+def backward_vocab_shard(H, W_shard, idx, logp, mask, V: int, v_begin: int, v_end: int, lse,
+                         grad_loss=None, chunk: int = 1024, dW=None, accumulate_dW: bool = False,
+                         workspace=None, stream=None, trace: Trace | None = None):
+    """(this shard's fp32 share of dH [T, d], dW of the shard's rows [Vs, d])."""
+    T, d, Vs, K = _check_shard(H, W_shard, idx, logp, mask, V, v_begin, v_end)
+    if workspace is None:
+        workspace = new_workspace(T, d, Vs, K, chunk, H.device)
+    if grad_loss is not None and (grad_loss.dtype != torch.float32 or not grad_loss.is_cuda):
+        raise TypeError("grad_loss must be a CUDA float32 tensor")
+    dHp = torch.empty(T, d, dtype=torch.float32, device=H.device)
+    if dW is None:
+        dW = torch.empty(Vs, d, dtype=torch.float32, device=H.device)
+        accumulate_dW = False
+    rc = lib.ckl_backward_vocab_shard(_ptr(H), _ptr(W_shard), _ptr(idx), _ptr(logp), _ptr(mask),
+                                      T, d, V, v_begin, v_end, K, chunk, _ptr(lse),
+                                      _ptr(grad_loss), _ptr(dHp), _ptr(dW),
+                                      int(bool(accumulate_dW)), _ptr(workspace),
+                                      workspace.numel(), _stream_handle(stream),
+                                      _trace_ptr(trace))
+    if rc != CKL_OK:
+        raise CklError(rc, "ckl_backward_vocab_shard")
+    return dHp, dW
+
+
+def dh_to_bf16(src, stream=None):
+    """bf16 copy (round to nearest even) of an fp32 CUDA tensor (ckl_dh_to_bf16)."""
+    if src.dtype != torch.float32 or not src.is_cuda or not src.is_contiguous():
+        raise ValueError("src must be a contiguous float32 CUDA tensor")
+    dst = torch.empty(src.shape, dtype=torch.bfloat16, device=src.device)
+    rc = lib.ckl_dh_to_bf16(_ptr(src), _ptr(dst), src.numel(), _stream_handle(stream))
+    if rc != CKL_OK:
+        raise CklError(rc, "ckl_dh_to_bf16")
+    return dst
 
 
 def dp_local_stats(workspace, stream=None):

@@ -274,12 +274,26 @@ bool setup_mode(DevInfo& di) {
   return true;
 }
 
+// L2 cache policies of each GEMM's operand loads (TcParams::l2hint codes).
+#ifndef CKL_L2HINT_FWD
+#define CKL_L2HINT_FWD 0
+#endif
+#ifndef CKL_L2HINT_DZ
+#define CKL_L2HINT_DZ 0
+#endif
+#ifndef CKL_L2HINT_DHDW
+#define CKL_L2HINT_DHDW 0
+#endif
+constexpr int32_t kL2Hint[4] = {CKL_L2HINT_FWD, CKL_L2HINT_DZ, CKL_L2HINT_DHDW, CKL_L2HINT_FWD};
+
 // Launches one persistent GEMM on min(co-resident slots, units) CTA pairs.
 template <int MODE, bool F32 = false>
-int launch_tc(const TcParams& p, int64_t units, const DevInfo& di, cudaStream_t st) {
+int launch_tc(const TcParams& p0, int64_t units, const DevInfo& di, cudaStream_t st) {
   const int slots = static_cast<int>(std::min<int64_t>(di.slots[MODE], units));
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = tc_config<MODE>(slots, st, attr);
+  TcParams p = p0;
+  p.l2hint = kL2Hint[MODE];
   return cudaLaunchKernelEx(&cfg, ckl::tc_kernel<MODE, kPair, F32>, p) == cudaSuccess
              ? CKL_OK
              : CKL_ERR_CUDA;
@@ -413,7 +427,7 @@ int clear_and_prep(const int32_t* idx, const float* logp, const uint8_t* mask, i
 int common_prep(const void* H, const void* W, const int32_t* idx, const float* logp,
                 const uint8_t* mask, int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk,
                 void* ws, size_t ws_bytes, cudaStream_t st, ckl_trace* trace, DevInfo& di,
-                Layout& L, bool single_pass = false, int eb = 2) {
+                Layout& L, bool single_pass = false, int eb = 2, int64_t v_valid = -1) {
   if (!sizes_ok(T, d, V, K, chunk)) return CKL_ERR_INVALID_ARG;
   // H, topk_idx and topk_logp may be NULL only for an empty batch.
   if (!W || !ws || (T > 0 && (!H || !idx || !logp))) return CKL_ERR_INVALID_ARG;
@@ -425,7 +439,8 @@ int common_prep(const void* H, const void* W, const int32_t* idx, const float* l
   if (!device_info(di)) return CKL_ERR_CUDA;
   if (di.major != 10) return CKL_ERR_UNSUPPORTED;
   if (!encode_fn()) return CKL_ERR_CUDA;
-  return clear_and_prep(idx, logp, mask, T, K, V, static_cast<uint8_t*>(ws), L, st, trace);
+  return clear_and_prep(idx, logp, mask, T, K, v_valid < 0 ? V : v_valid,
+                        static_cast<uint8_t*>(ws), L, st, trace);
 }
 
 void fill_common(TcParams& p, uint8_t* w8, const Layout& L, int64_t T, int64_t d, int64_t V,
@@ -464,7 +479,7 @@ template <bool F32>
 int dz_block(const void* H, const void* W, const uint8_t* mask, const float* lse, int64_t T,
              int64_t d, int64_t V, int32_t K, int64_t r0, int64_t rows, int64_t prow,
              int64_t v_lo, int64_t cols, uint8_t* w8, const Layout& L, const DevInfo& di,
-             cudaStream_t st, ckl_trace* trace) {
+             cudaStream_t st, ckl_trace* trace, int64_t v_off = 0) {
   constexpr int eb = F32 ? 4 : 2;
   constexpr uint32_t PW = kKE<F32>;
   TcParams p;
@@ -478,6 +493,7 @@ int dz_block(const void* H, const void* W, const uint8_t* mask, const float* lse
   p.S = 1;
   p.n_units = p.n_rb * p.n_vt;  // tiles, dealt out round-robin
   p.lse = lse;
+  p.v_off = static_cast<int32_t>(v_off);
   const uint8_t* Hr = static_cast<const uint8_t*>(H) + r0 * d * eb;
   if (!map2d(&p.tm[0], kDT<F32>, Hr, d, rows, d * eb, kKE<F32>, ckl::BM,
              CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -626,7 +642,7 @@ int forward_gemm_combine(const void* H, const void* W, const uint8_t* mask, int6
     TraceScope ts(trace, st, CKL_KERNEL_FWD_COMBINE);
     const unsigned grid = static_cast<unsigned>(cdiv(T, ckl::COMBINE_THREADS));
     ckl::combine_kernel<<<grid, ckl::COMBINE_THREADS, 0, st>>>(
-        reinterpret_cast<const float4*>(w8 + L.partials), p.S,
+        reinterpret_cast<const float4*>(w8 + L.partials), p.S, p.S, 1,
         reinterpret_cast<const float*>(w8 + L.hp), mask, T, lse,
         reinterpret_cast<double*>(w8 + L.blocksums), &hdr->ticket, &hdr->countN, loss,
         &hdr->numer);
@@ -653,13 +669,16 @@ int forward_impl(const void* H, const void* W, const int32_t* topk_idx, const fl
 }
 
 // The blocked backward (S0, S1, S5-S7) on bf16 or fp32 H and W; dH is bf16
-// or fp32 like H.
+// or fp32 like H.  For a vocabulary shard (W = rows [v_off, v_off + V) of a
+// head of v_valid rows), dH_f32 = true: dH is this shard's fp32 share, summed
+// over the shards by the caller.
 template <bool F32>
 int backward_impl(const void* H, const void* W, const int32_t* topk_idx, const float* topk_logp,
                   const uint8_t* mask, int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk,
                   const float* lse, const float* grad_loss, void* dH, float* dW,
                   int32_t accumulate_dW, void* workspace, size_t workspace_bytes, void* stream,
-                  ckl_trace* trace, ckl_dw_ready_fn on_dw_ready, void* user) {
+                  ckl_trace* trace, ckl_dw_ready_fn on_dw_ready, void* user,
+                  int64_t v_valid = -1, int64_t v_off = 0, bool dh_f32 = F32) {
   constexpr int eb = F32 ? 4 : 2;
   if (!dW || !aligned16(dW)) return CKL_ERR_INVALID_ARG;
   if (T > 0 && (!lse || !aligned4(lse) || !dH || !aligned16(dH))) return CKL_ERR_INVALID_ARG;
@@ -668,7 +687,7 @@ int backward_impl(const void* H, const void* W, const int32_t* topk_idx, const f
   DevInfo di;
   Layout L;
   int rc = common_prep(H, W, topk_idx, topk_logp, mask, T, d, V, K, chunk, workspace,
-                       workspace_bytes, st, trace, di, L, false, eb);
+                       workspace_bytes, st, trace, di, L, false, eb, v_valid);
   if (rc != CKL_OK) return rc;
   if (T == 0) {
     if (!accumulate_dW &&
@@ -689,13 +708,13 @@ int backward_impl(const void* H, const void* W, const int32_t* topk_idx, const f
       const int64_t v_lo = s * P.Sv;
       const int64_t cols = std::min(P.Sv, V - v_lo);
       rc = dz_block<F32>(H, W, mask, lse, T, d, V, K, r0, rows, P.Cr, v_lo, cols, w8, L, di,
-                         st, trace);
+                         st, trace, v_off);
       if (rc != CKL_OK) return rc;
       // bf16 dH: one slab writes it, several sum into the fp32 partial first;
       // fp32 dH: the slabs store / add into the output itself
       int dh_mode;
       void* dh_out;
-      if (F32) {
+      if (dh_f32) {
         dh_mode = (s == 0) ? 1 : 2;
         dh_out = static_cast<uint8_t*>(dH) + r0 * d * 4;
       } else {
@@ -709,7 +728,7 @@ int backward_impl(const void* H, const void* W, const int32_t* topk_idx, const f
       // the last row chunk's launch is the last to write these dW rows
       if (on_dw_ready && r0 + rows == T) on_dw_ready(v_lo, v_lo + cols, user);
     }
-    if (!F32 && P.n > 1) {
+    if (!dh_f32 && P.n > 1) {
       // dH rows of this chunk: the fp32 sum over its slabs, rounded once
       TraceScope ts(trace, st, CKL_KERNEL_OTHER);
       const int64_t n4 = rows * d / 4;
@@ -914,6 +933,104 @@ int ckl_selftest_wait_timeout(int64_t limit_ns, void* workspace, size_t workspac
   Header* hdr = static_cast<Header*>(workspace);
   ckl::wait_timeout_selftest_kernel<<<1, 32, 0, st>>>(&hdr->status,
                                                       static_cast<uint64_t>(limit_ns));
+  return cudaGetLastError() == cudaSuccess ? CKL_OK : CKL_ERR_CUDA;
+}
+
+int ckl_forward_vocab_shard(const uint16_t* H, const uint16_t* W_shard, const int32_t* topk_idx,
+                            const float* topk_logp, const uint8_t* mask, int64_t T, int64_t d,
+                            int64_t V, int64_t v_begin, int64_t v_end, int32_t K, int64_t chunk,
+                            float* row_partials, void* workspace, size_t workspace_bytes,
+                            void* stream, ckl_trace* trace) {
+  if (v_begin < 0 || v_end <= v_begin || v_end > V || !sizes_ok(T, d, V, K, chunk))
+    return CKL_ERR_INVALID_ARG;
+  if (T > 0 && (!row_partials || !aligned16(row_partials))) return CKL_ERR_INVALID_ARG;
+  const int64_t Vs = v_end - v_begin;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DevInfo di;
+  Layout L;
+  int rc = common_prep(H, W_shard, topk_idx, topk_logp, mask, T, d, Vs, K, chunk, workspace,
+                       workspace_bytes, st, trace, di, L, false, 2, V);
+  if (rc != CKL_OK || T == 0) return rc;
+  uint8_t* w8 = static_cast<uint8_t*>(workspace);
+  TcParams p;
+  std::memset(&p, 0, sizeof(p));
+  fill_common(p, w8, L, T, d, Vs, K, mask);
+  p.rows = static_cast<int32_t>(T);
+  p.n_rb = static_cast<int32_t>(cdiv(T, kMB));
+  p.v_off = static_cast<int32_t>(v_begin);
+  forward_schedule(p, d, 2, di.slots[ckl::MODE_FWD]);
+  if (!map2d(&p.tm[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, H, d, T, d * 2, ckl::BK, ckl::BM,
+             CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map2d(&p.tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W_shard, d, Vs, d * 2, ckl::BK,
+             ckl::BN_V / kSlotCTAs, CU_TENSOR_MAP_SWIZZLE_128B))
+    return CKL_ERR_CUDA;
+  {
+    TraceScope ts(trace, st, CKL_KERNEL_FWD_GEMM);
+    if (launch_tc<ckl::MODE_FWD>(p, p.n_units, di, st) != CKL_OK) return CKL_ERR_CUDA;
+  }
+  TraceScope ts(trace, st, CKL_KERNEL_FWD_COMBINE);
+  ckl::merge_splits_kernel<<<static_cast<unsigned>(cdiv(T, ckl::COMBINE_THREADS)),
+                             ckl::COMBINE_THREADS, 0, st>>>(
+      reinterpret_cast<const float4*>(w8 + L.partials), p.S, T,
+      reinterpret_cast<float4*>(row_partials));
+  return cudaGetLastError() == cudaSuccess ? CKL_OK : CKL_ERR_CUDA;
+}
+
+int ckl_combine_vocab_shards(const float* gathered, int32_t g, const uint8_t* mask, int64_t T,
+                             int32_t K, float* loss, float* lse, void* workspace,
+                             size_t workspace_bytes, void* stream, ckl_trace* trace) {
+  if (g < 1 || T < 0 || K < 1 || !loss || !aligned4(loss) || !workspace ||
+      !aligned16(workspace) || (T > 0 && (!gathered || !aligned16(gathered) || !lse ||
+                                          !aligned4(lse))))
+    return CKL_ERR_INVALID_ARG;
+  const Layout L = forward_layout(T, K);
+  if (workspace_bytes < L.total) return CKL_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* w8 = static_cast<uint8_t*>(workspace);
+  Header* hdr = reinterpret_cast<Header*>(w8);
+  if (T == 0) {
+    TraceScope ts(trace, st, CKL_KERNEL_OTHER);
+    ckl::zero_loss_kernel<<<1, 1, 0, st>>>(loss);
+    return cudaGetLastError() == cudaSuccess ? CKL_OK : CKL_ERR_CUDA;
+  }
+  if (cudaMemsetAsync(&hdr->ticket, 0, sizeof(hdr->ticket), st) != cudaSuccess)
+    return CKL_ERR_CUDA;
+  TraceScope ts(trace, st, CKL_KERNEL_FWD_COMBINE);
+  ckl::combine_kernel<<<static_cast<unsigned>(cdiv(T, ckl::COMBINE_THREADS)),
+                        ckl::COMBINE_THREADS, 0, st>>>(
+      reinterpret_cast<const float4*>(gathered), g, 1, T,
+      reinterpret_cast<const float*>(w8 + L.hp), mask, T, lse,
+      reinterpret_cast<double*>(w8 + L.blocksums), &hdr->ticket, &hdr->countN, loss,
+      &hdr->numer);
+  return cudaGetLastError() == cudaSuccess ? CKL_OK : CKL_ERR_CUDA;
+}
+
+int ckl_backward_vocab_shard(const uint16_t* H, const uint16_t* W_shard,
+                             const int32_t* topk_idx, const float* topk_logp,
+                             const uint8_t* mask, int64_t T, int64_t d, int64_t V,
+                             int64_t v_begin, int64_t v_end, int32_t K, int64_t chunk,
+                             const float* lse, const float* grad_loss, float* dH_partial,
+                             float* dW_shard, int32_t accumulate_dW, void* workspace,
+                             size_t workspace_bytes, void* stream, ckl_trace* trace) {
+  if (v_begin < 0 || v_end <= v_begin || v_end > V || !sizes_ok(T, d, V, K, chunk))
+    return CKL_ERR_INVALID_ARG;
+  return backward_impl<false>(H, W_shard, topk_idx, topk_logp, mask, T, d, v_end - v_begin, K,
+                              chunk, lse, grad_loss, dH_partial, dW_shard, accumulate_dW,
+                              workspace, workspace_bytes, stream, trace, nullptr, nullptr, V,
+                              v_begin, true);
+}
+
+int ckl_dh_to_bf16(const float* src, uint16_t* dst, int64_t n, void* stream) {
+  if (n < 0 || n % 4 != 0 || (n > 0 && (!src || !dst || !aligned16(src) ||
+                                        (reinterpret_cast<uintptr_t>(dst) & 7u))))
+    return CKL_ERR_INVALID_ARG;
+  if (n == 0) return CKL_OK;
+  DevInfo di;
+  if (!device_info(di)) return CKL_ERR_CUDA;
+  const int64_t n4 = n / 4;
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(cdiv(n4, 256), 4 * di.sms));
+  ckl::dh_convert_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const float4*>(src), n4, reinterpret_cast<uint2*>(dst));
   return cudaGetLastError() == cudaSuccess ? CKL_OK : CKL_ERR_CUDA;
 }
 

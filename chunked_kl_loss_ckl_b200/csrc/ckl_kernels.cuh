@@ -95,6 +95,11 @@ struct alignas(64) TcParams {
   int32_t dw_mode;  // DHDW: 0 = contiguous dW ranges per slot, 1 = dW tiles dealt in rounds
   int32_t split_fast;  // FWD: units numbered split-fastest (see JobIter)
   int32_t dw_Ql, dw_El, dw_Qh, dw_Eh;  // DHDW rounds: quotas, see JobIter
+  // L2 cache policy of the operand loads, 2 bits each (0 = none, 1 =
+  // evict_last, 2 = evict_first): bits 0-1 A, 2-3 B (FWD / DZ / dH units),
+  // bits 4-5 A, 6-7 B (dW tiles)
+  int32_t l2hint;
+  int32_t v_off;    // FWD / DZ: teacher id of local vocabulary column 0 (a vocabulary shard)
   const int2* pairs;      // [T, K] (id, p as bits), sorted by id per row
   float4* partials;       // FWD: [T, S] (max of z log2e, sum 2^(..), sum p z, 0)
   const float* lse;       // DZ: [T]
@@ -206,8 +211,12 @@ prep_kernel(const int32_t* __restrict__ idx, const float* __restrict__ logp,
 // ------------------------------------------------------------------ combine
 constexpr int COMBINE_THREADS = 256;
 
+// Partial s of row t is partials[t * row_stride + s * split_stride]: the
+// forward's vocabulary splits ([T][S]: S, 1) or the vocabulary shards of
+// several GPUs gathered as [g][T] (1, T).
 __global__ void __launch_bounds__(COMBINE_THREADS)
-combine_kernel(const float4* __restrict__ partials, int S, const float* __restrict__ Hp,
+combine_kernel(const float4* __restrict__ partials, int S, int64_t row_stride,
+               int64_t split_stride, const float* __restrict__ Hp,
                const uint8_t* __restrict__ mask, int64_t T, float* __restrict__ lse,
                double* block_sums, unsigned int* ticket, const int* countN, float* loss,
                double* numer) {
@@ -216,12 +225,12 @@ combine_kernel(const float4* __restrict__ partials, int S, const float* __restri
   const int64_t t = static_cast<int64_t>(blockIdx.x) * COMBINE_THREADS + threadIdx.x;
   float contrib = 0.f;
   if (t < T) {
-    const float4* pr = partials + t * S;
+    const float4* pr = partials + t * row_stride;
     float M = -INFINITY;
-    for (int s = 0; s < S; ++s) M = fmaxf(M, pr[s].x);
+    for (int s = 0; s < S; ++s) M = fmaxf(M, pr[s * split_stride].x);
     float se = 0.f, pz = 0.f;
     for (int s = 0; s < S; ++s) {
-      const float4 q = pr[s];
+      const float4 q = pr[s * split_stride];
       se += q.y * exp2f(q.x - M);
       pz += q.z;
     }
@@ -251,6 +260,26 @@ combine_kernel(const float4* __restrict__ partials, int S, const float* __restri
     *loss = (n > 0) ? static_cast<float>(total / static_cast<double>(n)) : 0.f;
     *numer = total;
   }
+}
+
+// One vocabulary shard's row partials: the forward's S splits of row t merged
+// into (max of z log2e, sum of 2^(z log2e - max), sum of p z over the shard's
+// teacher ids, 0), for the combine across shards.
+__global__ void __launch_bounds__(COMBINE_THREADS)
+merge_splits_kernel(const float4* __restrict__ partials, int S, int64_t T,
+                    float4* __restrict__ out) {
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * COMBINE_THREADS + threadIdx.x;
+  if (t >= T) return;
+  const float4* pr = partials + t * S;
+  float M = -INFINITY;
+  for (int s = 0; s < S; ++s) M = fmaxf(M, pr[s].x);
+  float se = 0.f, pz = 0.f;
+  for (int s = 0; s < S; ++s) {
+    const float4 q = pr[s];
+    se += q.y * exp2f(q.x - M);
+    pz += q.z;
+  }
+  out[t] = make_float4(M, se, pz, 0.f);
 }
 
 // H_c^T for the dW GEMM: Hc [rows, d] (pitch d) -> HcT [d, pitch_t] (rows
@@ -670,6 +699,26 @@ tc_kernel(const __grid_constant__ TcParams p) {
       uint32_t phase = 0;
       uint32_t issued = 0;
       bool ok = true;
+      const uint64_t pol_last = l2_policy_evict_last();
+      const uint64_t pol_first = l2_policy_evict_first();
+      // one operand load; a pair's may carry an L2 policy (code h, see l2hint)
+      auto load2 = [&](uint32_t dst, const CUtensorMap* m, uint32_t bar, int x, int y, int h) {
+        if (PAIR) {
+          if (h == 0) tma_load_2d_pair(dst, m, bar, x, y);
+          else tma_load_2d_pair_hint(dst, m, bar, x, y, h == 1 ? pol_last : pol_first);
+        } else {
+          tma_load_2d(dst, m, bar, x, y);
+        }
+      };
+      auto load3 = [&](uint32_t dst, const CUtensorMap* m, uint32_t bar, int x, int y, int z,
+                       int h) {
+        if (PAIR) {
+          if (h == 0) tma_load_3d_pair(dst, m, bar, x, y, z);
+          else tma_load_3d_pair_hint(dst, m, bar, x, y, z, h == 1 ? pol_last : pol_first);
+        } else {
+          tma_load_3d(dst, m, bar, x, y, z);
+        }
+      };
       JobIter it;
       it.init(p, MODE, PAIR ? 2 : 1);
       for (; ok && it.valid(p); it.next(p)) {
@@ -706,37 +755,23 @@ tc_kernel(const __grid_constant__ TcParams p) {
           }
           const uint32_t sa = sbase + C::A_OFF + stage * A_BYTES;
           const uint32_t sb = sbase + C::B_OFF + stage * B_STAGE;
+          const int ha = (kind == 6) ? (p.l2hint >> 4) & 3 : p.l2hint & 3;
+          const int hb = (kind == 6) ? (p.l2hint >> 6) & 3 : (p.l2hint >> 2) & 3;
           if (MODE != MODE_DHDW) {
-            if (PAIR) {
-              tma_load_2d_pair(sa, &p.tm[0], fb, kb * KE, a_y);
-              tma_load_2d_pair(sb, &p.tm[1], fb, kb * KE, b_y);
-            } else {
-              tma_load_2d(sa, &p.tm[0], fb, kb * KE, a_y);
-              tma_load_2d(sb, &p.tm[1], fb, kb * KE, b_y);
-            }
+            load2(sa, &p.tm[0], fb, kb * KE, a_y, ha);
+            load2(sb, &p.tm[1], fb, kb * KE, b_y, hb);
           } else if (kind == 5) {
             // dZ is stored as 64-column panels: k-block kb is panel kb.  W is
             // MN-major here: one 64-column atom per box.
-            if (PAIR) {
-              tma_load_3d_pair(sa, &p.tm[0], fb, 0, a_y, kb);
-              for (int j = 0; j < half_n / KE; ++j)
-                tma_load_2d_pair(sb + j * ATOM_B, &p.tm[1], fb, b_x + KE * j, p.v_lo + kb * KE);
-            } else {
-              tma_load_3d(sa, &p.tm[0], fb, 0, a_y, kb);
-              for (int j = 0; j < half_n / KE; ++j)
-                tma_load_2d(sb + j * ATOM_B, &p.tm[1], fb, b_x + KE * j, p.v_lo + kb * KE);
-            }
+            load3(sa, &p.tm[0], fb, 0, a_y, kb, ha);
+            for (int j = 0; j < half_n / KE; ++j)
+              load2(sb + j * ATOM_B, &p.tm[1], fb, b_x + KE * j, p.v_lo + kb * KE, hb);
           } else {
             // A = dZ^T: one box holding the two 64-column panels of this
             // vocabulary row block (8 KB each, one MN-major atom column each).
             // B = H_c^T (d rows x chunk rows, chunk rows contiguous): K-major.
-            if (PAIR) {
-              tma_load_3d_pair(sa, &p.tm[2], fb, 0, kb * KE, a_x / KE);
-              tma_load_2d_pair(sb, &p.tm[3], fb, kb * KE, b_x);
-            } else {
-              tma_load_3d(sa, &p.tm[2], fb, 0, kb * KE, a_x / KE);
-              tma_load_2d(sb, &p.tm[3], fb, kb * KE, b_x);
-            }
+            load3(sa, &p.tm[2], fb, 0, kb * KE, a_x / KE, ha);
+            load2(sb, &p.tm[3], fb, kb * KE, b_x, hb);
           }
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -915,7 +950,7 @@ tc_kernel(const __grid_constant__ TcParams p) {
         const bool want_ids = (MODE == MODE_DZ) ? counts : row_ok;
         if (want_ids) {
           const int2* pr = p.pairs + t * p.K;
-          const int v_lo = (p.vt0 + it.vt) * BN_V;
+          const int v_lo = p.v_off + (p.vt0 + it.vt) * BN_V;
           int lo = 0, hi = p.K;
           while (lo < hi) {
             const int mid = (lo + hi) >> 1;
@@ -961,8 +996,10 @@ tc_kernel(const __grid_constant__ TcParams p) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) se += ex2_approx(fmaf(x[j], LOG2E, -run_m));
           run_s += se;
-          while (nidx < v0 + 32) {
-            const int off = nidx - v0;
+          // ids past this launch's last column (another vocabulary shard's) stop the walk
+          const int v_hi = p.v_off + min(v0 + 32, p.V);
+          while (nidx < v_hi) {
+            const int off = nidx - p.v_off - v0;
             float val = x[0];
 #pragma unroll
             for (int j = 1; j < 32; ++j) val = (off == j) ? x[j] : val;
@@ -984,8 +1021,9 @@ tc_kernel(const __grid_constant__ TcParams p) {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
             x[j] = counts ? ex2_approx(fmaf(x[j], LOG2E, -lse2)) : 0.f;
-          while (nidx < v0 + 32) {
-            const int off = nidx - v0;
+          const int v_hi = p.v_off + min(v0 + 32, p.V);
+          while (nidx < v_hi) {
+            const int off = nidx - p.v_off - v0;
 #pragma unroll
             for (int j = 0; j < 32; ++j) x[j] -= (off == j) ? np_ : 0.f;
             ++cur;

@@ -273,6 +273,54 @@ CKL_API int ckl_selftest_wait_timeout(int64_t limit_ns, void* workspace, size_t 
                                       void* stream);
 
 /*
+ * Vocabulary-parallel loss: the head is split by rows over g GPUs, rank r
+ * holding W_shard = W[v_begin, v_end) (the output projection of a model
+ * whose vocabulary is sharded, so that no GPU holds all of W or dW).  The
+ * pages run one GPU and say that the fused loss let a GPT-OSS-20B
+ * distillation shrink from four nodes to one ("Tối ưu hóa chi phí chưng cất
+ * tri thức ...", section "Mở rộng quy mô đến độ dài ngữ cảnh dài"); this is
+ * the split a larger head takes when it does not fit one GPU.  Every rank
+ * holds all T rows of H and of the teacher cache; ids are global, in [0, V).
+ *
+ * ckl_forward_vocab_shard: prep + logit GEMM over this shard's columns;
+ *   writes row_partials [T, 4] fp32 (16-byte aligned): per row, (m, s, pz, 0)
+ *   with m = max over the shard of z log2(e), s = sum over the shard of
+ *   2^(z log2(e) - m), pz = sum of p_k z over the teacher ids inside the
+ *   shard.  Workspace: ckl_workspace_bytes(T, d, v_end - v_begin, K, chunk).
+ * ckl_combine_vocab_shards: gathered [g, T, 4] = every rank's row_partials
+ *   in rank order (an all-gather); writes lse [T] and the loss, exactly as
+ *   ckl_forward does from its vocabulary splits.  Uses the sum p log p and N
+ *   that ckl_forward_vocab_shard left in `workspace` (same T, K).
+ * ckl_backward_vocab_shard: recomputes this shard's logits with the global
+ *   lse; writes dH_partial [T, d] fp32 = this shard's share of dH (sum it
+ *   over the ranks, then round with ckl_dh_to_bf16) and dW_shard
+ *   [v_end - v_begin, d] fp32 (store, or add when accumulate_dW), which is
+ *   final: it needs no exchange.
+ * ckl_dh_to_bf16: dst[i] = bf16(src[i]), round to nearest even, n % 4 == 0,
+ *   src 16-byte and dst 8-byte aligned.
+ * Sizes, alignment and errors as in ckl_forward / ckl_backward, plus
+ * CKL_ERR_INVALID_ARG unless 0 <= v_begin < v_end <= V.
+ */
+CKL_API int ckl_forward_vocab_shard(const uint16_t* H, const uint16_t* W_shard,
+                                    const int32_t* topk_idx, const float* topk_logp,
+                                    const uint8_t* mask, int64_t T, int64_t d, int64_t V,
+                                    int64_t v_begin, int64_t v_end, int32_t K, int64_t chunk,
+                                    float* row_partials, void* workspace, size_t workspace_bytes,
+                                    void* stream, ckl_trace* trace);
+CKL_API int ckl_combine_vocab_shards(const float* gathered, int32_t g, const uint8_t* mask,
+                                     int64_t T, int32_t K, float* loss, float* lse,
+                                     void* workspace, size_t workspace_bytes, void* stream,
+                                     ckl_trace* trace);
+CKL_API int ckl_backward_vocab_shard(const uint16_t* H, const uint16_t* W_shard,
+                                     const int32_t* topk_idx, const float* topk_logp,
+                                     const uint8_t* mask, int64_t T, int64_t d, int64_t V,
+                                     int64_t v_begin, int64_t v_end, int32_t K, int64_t chunk,
+                                     const float* lse, const float* grad_loss, float* dH_partial,
+                                     float* dW_shard, int32_t accumulate_dW, void* workspace,
+                                     size_t workspace_bytes, void* stream, ckl_trace* trace);
+CKL_API int ckl_dh_to_bf16(const float* src, uint16_t* dst, int64_t n, void* stream);
+
+/*
  * Data-parallel training over T (no counterpart in the pages, which run on
  * one GPU): each rank holds its own rows of the batch and all of W, and the
  * loss is the mean over the positions that count on every rank.

@@ -23,9 +23,11 @@ def ckl():
 
 def test_header_declares_the_entry_points():
     assert _declared() == ["ckl_backward", "ckl_backward_ex", "ckl_backward_f32",
-                           "ckl_backward_plan", "ckl_dp_finish", "ckl_dp_local_stats",
-                           "ckl_forward", "ckl_forward_backward",
+                           "ckl_backward_plan", "ckl_backward_vocab_shard",
+                           "ckl_combine_vocab_shards", "ckl_dh_to_bf16", "ckl_dp_finish",
+                           "ckl_dp_local_stats", "ckl_forward", "ckl_forward_backward",
                            "ckl_forward_f32", "ckl_forward_static_scratch",
+                           "ckl_forward_vocab_shard",
                            "ckl_read_device_status", "ckl_selftest_wait_timeout",
                            "ckl_single_pass_workspace_bytes",
                            "ckl_status_string", "ckl_topk_cache", "ckl_version",
@@ -171,6 +173,17 @@ def test_host_checks_return_before_any_device_work(ckl):
     assert L.ckl_dp_local_stats(fake, ctypes.c_void_p(4100), nul) == 1
     assert L.ckl_dp_finish(nul, nul, fake, fake, nul) == 1
     assert L.ckl_dp_finish(fake, nul, fake, ctypes.c_void_p(4097), nul) == 1
+    # vocabulary shards: the shard must lie inside [0, V) and be non-empty
+    for vb, ve in ((-1, 10), (10, 10), (50, 101)):
+        assert L.ckl_forward_vocab_shard(fake, fake, fake, fake, nul, 4, 64, 100, vb, ve, 4, 8,
+                                         fake, fake, 1 << 20, nul, nul) == 1
+        assert L.ckl_backward_vocab_shard(fake, fake, fake, fake, nul, 4, 64, 100, vb, ve, 4, 8,
+                                          fake, nul, fake, fake, 0, fake, 1 << 20, nul, nul) == 1
+    assert L.ckl_combine_vocab_shards(fake, 0, nul, 4, 4, fake, fake, fake, 1 << 20, nul,
+                                      nul) == 1
+    assert L.ckl_combine_vocab_shards(fake, 2, nul, 4, 4, fake, fake, fake, 16, nul, nul) == 3
+    assert L.ckl_dh_to_bf16(fake, fake, 6, nul) == 1
+    assert L.ckl_dh_to_bf16(ctypes.c_void_p(4100), fake, 8, nul) == 1
 
 
 def test_static_scratch_limit_is_checked_on_the_host(ckl):

@@ -165,3 +165,111 @@ def test_data_parallel_step_two_gloo_ranks(tmp_path):
         np.testing.assert_allclose(x["dW"], full["dW"], rtol=1e-5, atol=1e-7)
         lo, hi = int(x["lo"]), int(x["hi"])
         np.testing.assert_allclose(x["dH"], full["dH"][lo:hi], rtol=1e-5, atol=1e-7)
+
+
+# ---------------------------------------------------------------- vocabulary parallel
+class _OracleVPOps:
+    """Stands in for the CUDA library's vocabulary-shard entry points on CPU:
+    per-row (max z log2 e, sum of 2^(z log2 e - max), sum of p z over the
+    shard's teacher ids) from the oracle's logits of the shard, their merge,
+    and the shard's share of the closed-form gradient."""
+
+    LOG2E = 1.0 / np.log(2.0)
+
+    def __init__(self, c):
+        import oracle
+        self.c = c
+        self.H = oracle.widen_bf16(c["H"])
+        self.W = oracle.widen_bf16(c["W"])
+        self.p, self.logp_n = oracle.renormalise_topk(c["logp"])
+        m = np.ones(c["T"]) if c["mask"] is None else (c["mask"] != 0).astype(float)
+        self.m, self.N = m, m.sum()
+
+    def _shard_logits(self, vb, ve):
+        import oracle
+        return oracle.logits(self.H, self.W[vb:ve])
+
+    def forward_vocab_shard(self, H, W_shard, idx, logp, mask, V, vb, ve, chunk):
+        Z = self._shard_logits(vb, ve)
+        y = Z * self.LOG2E
+        mx = y.max(axis=1)
+        s = np.exp2(y - mx[:, None]).sum(axis=1)
+        ids = self.c["idx"].astype(np.int64)
+        inside = (ids >= vb) & (ids < ve)
+        zg = np.take_along_axis(Z, np.clip(ids - vb, 0, ve - vb - 1), axis=1)
+        pz = np.where(inside, self.p * zg, 0.0).sum(axis=1)
+        part = np.stack([mx, s, pz, np.zeros_like(mx)], axis=1)
+        return torch.from_numpy(part.astype(np.float32)), torch.zeros(1)
+
+    def combine_vocab_shards(self, gathered, mask, K, ws):
+        g = gathered.double().numpy()
+        M = g[:, :, 0].max(axis=0)
+        S = (g[:, :, 1] * np.exp2(g[:, :, 0] - M[None, :])).sum(axis=0)
+        pz = g[:, :, 2].sum(axis=0)
+        lse = (M + np.log2(S)) * np.log(2.0)
+        hp = np.where(self.p > 0, self.p * np.where(self.p > 0, self.logp_n, 0.0), 0.0).sum(1)
+        kl = hp - pz + lse
+        loss = (self.m * kl).sum() / self.N if self.N > 0 else 0.0
+        self.lse = lse
+        return torch.tensor([loss], dtype=torch.float32), torch.from_numpy(lse.astype(np.float32))
+
+    def backward_vocab_shard(self, H, W_shard, idx, logp, mask, V, vb, ve, lse, grad_loss=None,
+                             chunk=1024, workspace=None):
+        g = 1.0 if grad_loss is None else float(grad_loss.item())
+        Z = self._shard_logits(vb, ve)
+        G = np.exp(Z - self.lse[:, None])
+        ids = self.c["idx"].astype(np.int64)
+        for t in range(Z.shape[0]):
+            for k in range(ids.shape[1]):
+                if vb <= ids[t, k] < ve:
+                    G[t, ids[t, k] - vb] -= self.p[t, k]
+        G *= (g * self.m / self.N)[:, None] if self.N > 0 else 0.0
+        return torch.from_numpy(G @ self.W[vb:ve]), torch.from_numpy(G.T @ self.H)
+
+    def dh_to_bf16(self, x):
+        return x.to(torch.bfloat16)
+
+
+def _vp_worker(rank, world, port, out_dir):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        from chunked_kl_loss_ckl_b200.vp import vp_forward_backward
+        from ckl_synth import make_inputs
+        c = make_inputs(40, 16, 60, 5, seed=5, w_std=0.4, mask=("bernoulli", 0.2))
+        vb, ve = (0, 23) if rank == 0 else (23, 60)          # uneven, unaligned
+        ops = _OracleVPOps(c)
+        g = torch.tensor([0.7], dtype=torch.float32)
+        loss, lse, dH, dW = vp_forward_backward(
+            torch.zeros(40, 16), torch.zeros(ve - vb, 16), 60, vb, ve,
+            torch.from_numpy(c["idx"]), torch.from_numpy(c["logp"]),
+            torch.from_numpy(c["mask"]), chunk=8, grad_loss=g, ops=ops)
+        np.savez(os.path.join(out_dir, f"vp{rank}.npz"), loss=loss.numpy(), lse=lse.numpy(),
+                 dH=dH.float().numpy(), dW=dW.numpy(), vb=vb, ve=ve)
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def test_vocab_parallel_step_two_gloo_ranks(tmp_path):
+    """vp_forward_backward on two ranks holding uneven vocabulary shards of
+    the head equals the unsharded loss, lse, dH and (concatenated) dW: the
+    per-row (max, sum of exp, sum of p z) partials merge exactly."""
+    world = 2
+    mp.spawn(_vp_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True)
+    r = [np.load(tmp_path / f"vp{i}.npz") for i in range(world)]
+    import oracle
+    from ckl_synth import make_inputs
+    c = make_inputs(40, 16, 60, 5, seed=5, w_std=0.4, mask=("bernoulli", 0.2))
+    full = oracle.dense(c["H"], c["W"], c["idx"], c["logp"], c["mask"], g=0.7)
+    for x in r:
+        assert abs(float(x["loss"][0]) - full["loss"]) <= 1e-6 * full["loss"]
+        np.testing.assert_allclose(x["lse"], full["lse"], rtol=1e-6, atol=1e-6)
+        # dH is rounded to bf16 once, after the sum over the shards
+        np.testing.assert_allclose(x["dH"], full["dH"], rtol=1e-2, atol=1e-4)
+        np.testing.assert_allclose(x["dW"], full["dW"][int(x["vb"]):int(x["ve"])], rtol=1e-5,
+                                   atol=1e-7)
+    assert np.array_equal(r[0]["dH"], r[1]["dH"])
