@@ -274,26 +274,12 @@ bool setup_mode(DevInfo& di) {
   return true;
 }
 
-// L2 cache policies of each GEMM's operand loads (TcParams::l2hint codes).
-#ifndef CKL_L2HINT_FWD
-#define CKL_L2HINT_FWD 0
-#endif
-#ifndef CKL_L2HINT_DZ
-#define CKL_L2HINT_DZ 0
-#endif
-#ifndef CKL_L2HINT_DHDW
-#define CKL_L2HINT_DHDW 0
-#endif
-constexpr int32_t kL2Hint[4] = {CKL_L2HINT_FWD, CKL_L2HINT_DZ, CKL_L2HINT_DHDW, CKL_L2HINT_FWD};
-
 // Launches one persistent GEMM on min(co-resident slots, units) CTA pairs.
 template <int MODE, bool F32 = false>
-int launch_tc(const TcParams& p0, int64_t units, const DevInfo& di, cudaStream_t st) {
+int launch_tc(const TcParams& p, int64_t units, const DevInfo& di, cudaStream_t st) {
   const int slots = static_cast<int>(std::min<int64_t>(di.slots[MODE], units));
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = tc_config<MODE>(slots, st, attr);
-  TcParams p = p0;
-  p.l2hint = kL2Hint[MODE];
   return cudaLaunchKernelEx(&cfg, ckl::tc_kernel<MODE, kPair, F32>, p) == cudaSuccess
              ? CKL_OK
              : CKL_ERR_CUDA;
@@ -914,9 +900,15 @@ int ckl_topk_cache(const uint16_t* teacher_logits, int64_t T, int64_t V, int32_t
   if (T == 0) return CKL_OK;
   const int vec8 = (V % 8 == 0 && aligned16(teacher_logits)) ? 1 : 0;
   const int grid = static_cast<int>(std::min<int64_t>(T, static_cast<int64_t>(di.sms) * 2));
-  ckl::topk_cache_kernel<<<grid, ckl::TK_THREADS, 0, st>>>(teacher_logits, T, static_cast<int>(V),
-                                                           K, vec8, topk_idx, topk_logp,
-                                                           device_status);
+  if (K <= ckl::TK_THREADS) {
+    ckl::topk_stream_kernel<<<grid, ckl::TK_THREADS, 0, st>>>(
+        teacher_logits, T, static_cast<int>(V), K, vec8, topk_idx, topk_logp, device_status);
+    if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
+    ckl::topk_fallback_kernel<<<grid, ckl::TK_THREADS, 0, st>>>(
+        teacher_logits, T, static_cast<int>(V), K, vec8, topk_idx, topk_logp, device_status);
+  } else
+    ckl::topk_cache_kernel<<<grid, ckl::TK_THREADS, 0, st>>>(
+        teacher_logits, T, static_cast<int>(V), K, vec8, topk_idx, topk_logp, device_status);
   return cudaGetLastError() == cudaSuccess ? CKL_OK : CKL_ERR_CUDA;
 }
 

@@ -95,10 +95,6 @@ struct alignas(64) TcParams {
   int32_t dw_mode;  // DHDW: 0 = contiguous dW ranges per slot, 1 = dW tiles dealt in rounds
   int32_t split_fast;  // FWD: units numbered split-fastest (see JobIter)
   int32_t dw_Ql, dw_El, dw_Qh, dw_Eh;  // DHDW rounds: quotas, see JobIter
-  // L2 cache policy of the operand loads, 2 bits each (0 = none, 1 =
-  // evict_last, 2 = evict_first): bits 0-1 A, 2-3 B (FWD / DZ / dH units),
-  // bits 4-5 A, 6-7 B (dW tiles)
-  int32_t l2hint;
   int32_t v_off;    // FWD / DZ: teacher id of local vocabulary column 0 (a vocabulary shard)
   const int2* pairs;      // [T, K] (id, p as bits), sorted by id per row
   float4* partials;       // FWD: [T, S] (max of z log2e, sum 2^(..), sum p z, 0)
@@ -699,26 +695,6 @@ tc_kernel(const __grid_constant__ TcParams p) {
       uint32_t phase = 0;
       uint32_t issued = 0;
       bool ok = true;
-      const uint64_t pol_last = l2_policy_evict_last();
-      const uint64_t pol_first = l2_policy_evict_first();
-      // one operand load; a pair's may carry an L2 policy (code h, see l2hint)
-      auto load2 = [&](uint32_t dst, const CUtensorMap* m, uint32_t bar, int x, int y, int h) {
-        if (PAIR) {
-          if (h == 0) tma_load_2d_pair(dst, m, bar, x, y);
-          else tma_load_2d_pair_hint(dst, m, bar, x, y, h == 1 ? pol_last : pol_first);
-        } else {
-          tma_load_2d(dst, m, bar, x, y);
-        }
-      };
-      auto load3 = [&](uint32_t dst, const CUtensorMap* m, uint32_t bar, int x, int y, int z,
-                       int h) {
-        if (PAIR) {
-          if (h == 0) tma_load_3d_pair(dst, m, bar, x, y, z);
-          else tma_load_3d_pair_hint(dst, m, bar, x, y, z, h == 1 ? pol_last : pol_first);
-        } else {
-          tma_load_3d(dst, m, bar, x, y, z);
-        }
-      };
       JobIter it;
       it.init(p, MODE, PAIR ? 2 : 1);
       for (; ok && it.valid(p); it.next(p)) {
@@ -755,23 +731,37 @@ tc_kernel(const __grid_constant__ TcParams p) {
           }
           const uint32_t sa = sbase + C::A_OFF + stage * A_BYTES;
           const uint32_t sb = sbase + C::B_OFF + stage * B_STAGE;
-          const int ha = (kind == 6) ? (p.l2hint >> 4) & 3 : p.l2hint & 3;
-          const int hb = (kind == 6) ? (p.l2hint >> 6) & 3 : (p.l2hint >> 2) & 3;
           if (MODE != MODE_DHDW) {
-            load2(sa, &p.tm[0], fb, kb * KE, a_y, ha);
-            load2(sb, &p.tm[1], fb, kb * KE, b_y, hb);
+            if (PAIR) {
+              tma_load_2d_pair(sa, &p.tm[0], fb, kb * KE, a_y);
+              tma_load_2d_pair(sb, &p.tm[1], fb, kb * KE, b_y);
+            } else {
+              tma_load_2d(sa, &p.tm[0], fb, kb * KE, a_y);
+              tma_load_2d(sb, &p.tm[1], fb, kb * KE, b_y);
+            }
           } else if (kind == 5) {
             // dZ is stored as 64-column panels: k-block kb is panel kb.  W is
             // MN-major here: one 64-column atom per box.
-            load3(sa, &p.tm[0], fb, 0, a_y, kb, ha);
-            for (int j = 0; j < half_n / KE; ++j)
-              load2(sb + j * ATOM_B, &p.tm[1], fb, b_x + KE * j, p.v_lo + kb * KE, hb);
+            if (PAIR) {
+              tma_load_3d_pair(sa, &p.tm[0], fb, 0, a_y, kb);
+              for (int j = 0; j < half_n / KE; ++j)
+                tma_load_2d_pair(sb + j * ATOM_B, &p.tm[1], fb, b_x + KE * j, p.v_lo + kb * KE);
+            } else {
+              tma_load_3d(sa, &p.tm[0], fb, 0, a_y, kb);
+              for (int j = 0; j < half_n / KE; ++j)
+                tma_load_2d(sb + j * ATOM_B, &p.tm[1], fb, b_x + KE * j, p.v_lo + kb * KE);
+            }
           } else {
             // A = dZ^T: one box holding the two 64-column panels of this
             // vocabulary row block (8 KB each, one MN-major atom column each).
             // B = H_c^T (d rows x chunk rows, chunk rows contiguous): K-major.
-            load3(sa, &p.tm[2], fb, 0, kb * KE, a_x / KE, ha);
-            load2(sb, &p.tm[3], fb, kb * KE, b_x, hb);
+            if (PAIR) {
+              tma_load_3d_pair(sa, &p.tm[2], fb, 0, kb * KE, a_x / KE);
+              tma_load_2d_pair(sb, &p.tm[3], fb, kb * KE, b_x);
+            } else {
+              tma_load_3d(sa, &p.tm[2], fb, 0, kb * KE, a_x / KE);
+              tma_load_2d(sb, &p.tm[3], fb, kb * KE, b_x);
+            }
           }
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }

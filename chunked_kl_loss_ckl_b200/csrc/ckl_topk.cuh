@@ -6,8 +6,11 @@
 // position are kept, and training reads that cache.  This is the step that
 // writes it, given the teacher's logits.
 //
-// One CTA per row (persistent over rows), three passes over the row (the
-// first from HBM, the others mostly from L2):
+// One CTA per row (persistent over rows).  The streaming form (below, K up
+// to the CTA's 512 threads) reads each row once from HBM and once more from
+// L2.  The histogram form, used for larger K and for rows the streaming form
+// cannot settle, makes three passes over the row (the first from HBM, the
+// others mostly from L2):
 //   1. the largest logit (packed bf16 maxima, two per instruction);
 //   2. the row's sum of exp(z - max) (log-sum-exp = max + log of it), and a
 //      histogram of the 128 keys just below the largest (one bucket per bf16
@@ -55,6 +58,7 @@ __device__ __forceinline__ uint32_t bf16_key2(uint32_t w) {
 }
 
 constexpr int TK_UNROLL = 2;  // independent 16-byte loads in flight per thread
+constexpr int TS_UNROLL = 4;  // the same, in the streaming form's pass from HBM
 
 __device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
   uint32_t r;
@@ -126,142 +130,353 @@ __device__ __forceinline__ void tk_for_row(const uint16_t* z, int V, bool vec8, 
   }
 }
 
+// Shared memory of one row's selection.
+struct TkShared {
+  uint32_t hist[TK_WIN];
+  unsigned long long cand[TK_CAP];
+  float s_s[TK_THREADS / 32];
+  float s_c[TK_THREADS / 32];
+  uint32_t s_part[TK_THREADS / 32];
+  uint32_t s_thr, s_ncand, s_found, s_total;
+  float s_lse;
+};
+
+// Sorts the row's n candidates (key << 32 | ~id) in shared memory, descending
+// (equal keys: smaller id first), and writes the first K: ids and z - lse.
+__device__ __forceinline__ void tk_sort_and_write(TkShared& sm, uint32_t n, int K, float lse,
+                                                  int64_t row, int32_t* idx_out,
+                                                  float* logp_out) {
+  const int tid = threadIdx.x;
+  uint32_t P = 1;
+  while (P < n) P <<= 1;
+  for (uint32_t i = n + tid; i < P; i += TK_THREADS) sm.cand[i] = 0ull;
+  __syncthreads();
+  for (uint32_t k = 2; k <= P; k <<= 1) {
+    for (uint32_t j = k >> 1; j > 0; j >>= 1) {
+      for (uint32_t i = tid; i < P; i += TK_THREADS) {
+        const uint32_t ixj = i ^ j;
+        if (ixj > i) {
+          const unsigned long long a = sm.cand[i], b = sm.cand[ixj];
+          const bool up = (i & k) == 0;
+          if (up ? (a < b) : (a > b)) { sm.cand[i] = b; sm.cand[ixj] = a; }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int k = tid; k < K; k += TK_THREADS) {
+    const unsigned long long e = sm.cand[k];
+    const uint32_t key = static_cast<uint32_t>(e >> 32);
+    idx_out[row * K + k] = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(e));
+    logp_out[row * K + k] = key_value(key) - lse;
+  }
+  __syncthreads();
+}
+
+// Gathers every element of the row whose value is >= v_thr into the
+// candidates; returns their count (the array holds at most TK_CAP).
+__device__ __forceinline__ uint32_t tk_gather(TkShared& sm, const uint16_t* z, int V, bool vec8,
+                                              float v_thr) {
+  if (threadIdx.x == 0) sm.s_ncand = 0;
+  __syncthreads();
+  auto put = [&](float v, uint32_t raw, int i) {
+    if (v >= v_thr) {
+      const uint32_t slot = atomicAdd(&sm.s_ncand, 1u);
+      if (slot < TK_CAP)
+        sm.cand[slot] = (static_cast<unsigned long long>(bf16_key(raw)) << 32) |
+                        (0xFFFFFFFFu - static_cast<uint32_t>(i));
+    }
+  };
+  if (vec8) {
+    // a whole 8-element vector below the threshold is skipped on its maximum
+    const uint4* z4 = reinterpret_cast<const uint4*>(z);
+    const int n8 = V / 8;
+    for (int base = threadIdx.x; base < n8; base += TK_THREADS * TK_UNROLL) {
+      uint4 v[TK_UNROLL];
+#pragma unroll
+      for (int u = 0; u < TK_UNROLL; ++u) {
+        const int i = base + u * TK_THREADS;
+        if (i < n8) v[u] = z4[i];
+      }
+#pragma unroll
+      for (int u = 0; u < TK_UNROLL; ++u) {
+        const int i = base + u * TK_THREADS;
+        if (i >= n8) continue;
+        const uint32_t m2 = bf16x2_max(bf16x2_max(v[u].x, v[u].y), bf16x2_max(v[u].z, v[u].w));
+        if (fmaxf(bf16_lo(m2), bf16_hi(m2)) < v_thr) continue;
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          put(bf16_lo(w[j]), w[j] & 0xFFFFu, 8 * i + 2 * j);
+          put(bf16_hi(w[j]), w[j] >> 16, 8 * i + 2 * j + 1);
+        }
+      }
+    }
+  } else {
+    for (int i = threadIdx.x; i < V; i += TK_THREADS) {
+      const uint32_t b = z[i];
+      put(__uint_as_float(b << 16), b, i);
+    }
+  }
+  __syncthreads();
+  return sm.s_ncand;
+}
+
+// One row by histogram windows (exact for any data with at most TK_CAP
+// elements at or above the K-th largest value): the largest logit; the sum of
+// exp against it and the histogram of the 128 keys just below it, sliding
+// down 4096 keys at a time until K elements are covered; the gather; the sort.
+__device__ void tk_row_hist(TkShared& sm, const uint16_t* z, int V, bool vec8, int K,
+                            int64_t row, int32_t* idx_out, float* logp_out, int* status) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // ---- pass 1: the largest logit
+  float zm = tk_row_max(z, V, vec8);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) zm = fmaxf(zm, __shfl_xor_sync(0xffffffffu, zm, o));
+  if (lane == 0) sm.s_s[warp] = zm;
+  for (int j = tid; j < TK_WIN; j += TK_THREADS) sm.hist[j] = 0;
+  if (tid == 0) { sm.s_found = 0; sm.s_thr = 0; }
+  __syncthreads();
+  float zmax = -INFINITY;
+  for (int w = 0; w < TK_THREADS / 32; ++w) zmax = fmaxf(zmax, sm.s_s[w]);
+  __syncthreads();  // s_s is reused below
+  // its key (bf16 bits of the value; -0 counts as +0)
+  const uint32_t kmax = bf16_key(__float_as_uint(zmax) >> 16);
+
+  // ---- pass 2: sum of exp against the maximum, and the first window's
+  // histogram; further windows (4096 keys each) only when needed
+  uint32_t above = 0;         // elements with a key above the window
+  int top = static_cast<int>(kmax);
+  float lse = 0.f;
+  for (int win = 0;; ++win) {
+    const int lo = top - (win == 0 ? TK_WIN0 : TK_WIN) + 1;
+    // the window's bounds as values: key order is value order
+    const float v_lo = lo > 0 ? key_value(static_cast<uint32_t>(lo)) : -INFINITY;
+    const float v_top = key_value(static_cast<uint32_t>(top));
+    if (win == 0) {
+      float s = 0.f;
+      tk_for_row(z, V, vec8, [&](float v, uint32_t raw, int) {
+        s += ex2_approx((v - zmax) * LOG2E);  // v - zmax is exact near the max
+        if (v >= v_lo) atomicAdd(&sm.hist[top - static_cast<int>(bf16_key(raw))], 1u);
+      });
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (lane == 0) sm.s_s[warp] = s;
+    } else {
+      for (int j = tid; j < TK_WIN; j += TK_THREADS) sm.hist[j] = 0;
+      __syncthreads();
+      tk_for_row(z, V, vec8, [&](float v, uint32_t raw, int) {
+        if (v <= v_top && v >= v_lo) atomicAdd(&sm.hist[top - static_cast<int>(bf16_key(raw))], 1u);
+      });
+    }
+    __syncthreads();
+    if (win == 0) {
+      float S = 0.f;
+      for (int w = 0; w < TK_THREADS / 32; ++w) S += sm.s_s[w];
+      lse = zmax + logf(S);
+    }
+    // block scan over the window: thread tid owns buckets [8 tid, 8 tid + 8)
+    uint32_t own = 0;
+#pragma unroll
+    for (int j = 0; j < TK_WIN / TK_THREADS; ++j) own += sm.hist[tid * (TK_WIN / TK_THREADS) + j];
+    uint32_t incl = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) sm.s_part[warp] = incl;
+    __syncthreads();
+    uint32_t before = 0;
+    for (int w = 0; w < warp; ++w) before += sm.s_part[w];
+    before += incl - own;  // elements in buckets before this thread's (higher keys)
+    if (tid == TK_THREADS - 1) sm.s_total = before + own;
+    if (above + before < static_cast<uint32_t>(K) &&
+        above + before + own >= static_cast<uint32_t>(K)) {
+      uint32_t c = above + before;
+      for (int j = 0; j < TK_WIN / TK_THREADS; ++j) {
+        c += sm.hist[tid * (TK_WIN / TK_THREADS) + j];
+        if (c >= static_cast<uint32_t>(K)) {
+          sm.s_thr = static_cast<uint32_t>(top - (tid * (TK_WIN / TK_THREADS) + j));
+          sm.s_found = 1;
+          break;
+        }
+      }
+    }
+    __syncthreads();
+    if (sm.s_found || lo <= 0) break;
+    above += sm.s_total;
+    top = lo - 1;
+    __syncthreads();
+  }
+  const float v_thr = key_value(sm.s_thr);
+
+  // ---- pass 3: gather every element at or above the threshold, sort
+  const uint32_t ncand = tk_gather(sm, z, V, vec8, v_thr);
+  if (tid == 0 && ncand > static_cast<uint32_t>(TK_CAP) && status != nullptr)
+    atomicOr(status, CKL_DEV_TOPK_TIES);
+  tk_sort_and_write(sm, min(ncand, static_cast<uint32_t>(TK_CAP)), K, lse, row, idx_out,
+                    logp_out);
+}
+
 __global__ void __launch_bounds__(TK_THREADS, 2)
 topk_cache_kernel(const uint16_t* __restrict__ logits, int64_t T, int V, int K, int vec8,
                   int32_t* __restrict__ idx_out, float* __restrict__ logp_out, int* status) {
-  __shared__ uint32_t hist[TK_WIN];
-  __shared__ unsigned long long cand[TK_CAP];
-  __shared__ float s_s[TK_THREADS / 32];
-  __shared__ uint32_t s_part[TK_THREADS / 32];
-  __shared__ uint32_t s_thr, s_ncand, s_found, s_total;
+  __shared__ TkShared sm;
+  for (int64_t row = blockIdx.x; row < T; row += gridDim.x)
+    tk_row_hist(sm, logits + row * static_cast<int64_t>(V), V, vec8 != 0, K, row, idx_out,
+                logp_out, status);
+}
+
+// ------------------------------------------------------------ streaming form
+// Two passes per row.  Pass 1 (the only one from HBM): every thread keeps
+// its running maximum c and the sum of 2^((z - c) log2 e) over its own
+// elements, rescaled when c grows (at most once per 8-element vector); the
+// block merges the (c, sum) pairs into the row's log-sum-exp.  The K-th
+// largest of the threads' maxima is at most the row's K-th largest value
+// (those K maxima are K elements of the row), so it is a valid threshold:
+// pass 2 (from L2) gathers every element at or above it, vectors whose
+// maximum is below it skipped whole, and the sort keeps the first K.  With
+// the row's top K spread over the threads, the threshold sits just below the
+// K-th value and a few more than K elements are gathered.  When more than
+// TK_CAP would be (the row's large values crowded into few threads), the
+// row is marked and done again by histogram windows in topk_fallback_kernel.
+// Needs K <= TK_THREADS.
+__device__ __forceinline__ uint32_t tk_kth_largest_key(TkShared& sm, uint32_t key, int K) {
+  // two 256-bucket rounds (high byte, then low byte) over the threads' keys
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-
-  for (int64_t row = blockIdx.x; row < T; row += gridDim.x) {
-    const uint16_t* z = logits + row * static_cast<int64_t>(V);
-
-    // ---- pass 1: the largest logit
-    float zm = tk_row_max(z, V, vec8 != 0);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) zm = fmaxf(zm, __shfl_xor_sync(0xffffffffu, zm, o));
-    if (lane == 0) s_s[warp] = zm;
-    for (int j = tid; j < TK_WIN; j += TK_THREADS) hist[j] = 0;
-    if (tid == 0) { s_found = 0; s_thr = 0; }
+  uint32_t prefix = 0, need = static_cast<uint32_t>(K);
+  for (int round = 0; round < 2; ++round) {
+    for (int j = tid; j < 256; j += TK_THREADS) sm.hist[j] = 0;
     __syncthreads();
-    float zmax = -INFINITY;
-    for (int w = 0; w < TK_THREADS / 32; ++w) zmax = fmaxf(zmax, s_s[w]);
-    __syncthreads();  // s_s is reused below
-    // its key (bf16 bits of the value; -0 counts as +0)
-    const uint32_t kmax = bf16_key(__float_as_uint(zmax) >> 16);
-
-    // ---- pass 2: sum of exp against the maximum, and the first window's
-    // histogram; further windows (4096 keys each) only when needed
-    uint32_t above = 0;         // elements with a key above the window
-    int top = static_cast<int>(kmax);
-    float lse = 0.f;
-    for (int win = 0;; ++win) {
-      const int lo = top - (win == 0 ? TK_WIN0 : TK_WIN) + 1;
-      // the window's bounds as values: key order is value order
-      const float v_lo = lo > 0 ? key_value(static_cast<uint32_t>(lo)) : -INFINITY;
-      const float v_top = key_value(static_cast<uint32_t>(top));
-      if (win == 0) {
-        float s = 0.f;
-        tk_for_row(z, V, vec8 != 0, [&](float v, uint32_t raw, int) {
-          s += ex2_approx((v - zmax) * LOG2E);  // v - zmax is exact near the max
-          if (v >= v_lo) atomicAdd(&hist[top - static_cast<int>(bf16_key(raw))], 1u);
-        });
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (lane == 0) s_s[warp] = s;
-      } else {
-        for (int j = tid; j < TK_WIN; j += TK_THREADS) hist[j] = 0;
-        __syncthreads();
-        tk_for_row(z, V, vec8 != 0, [&](float v, uint32_t raw, int) {
-          if (v <= v_top && v >= v_lo) atomicAdd(&hist[top - static_cast<int>(bf16_key(raw))], 1u);
-        });
-      }
-      __syncthreads();
-      if (win == 0) {
-        float S = 0.f;
-        for (int w = 0; w < TK_THREADS / 32; ++w) S += s_s[w];
-        lse = zmax + logf(S);
-      }
-      // block scan over the window: thread tid owns buckets [8 tid, 8 tid + 8)
-      uint32_t own = 0;
-#pragma unroll
-      for (int j = 0; j < TK_WIN / TK_THREADS; ++j) own += hist[tid * (TK_WIN / TK_THREADS) + j];
-      uint32_t incl = own;
+    const bool in = (round == 0) || ((key >> 8) == prefix);
+    if (in) atomicAdd(&sm.hist[(round == 0) ? (key >> 8) : (key & 0xFFu)], 1u);
+    __syncthreads();
+    // suffix counts: warps 0..7 scan buckets 255..0, 32 each
+    uint32_t c = 0, incl = 0;
+    if (warp < 8) {
+      c = sm.hist[255 - (warp * 32 + lane)];
+      incl = c;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += v;
       }
-      if (lane == 31) s_part[warp] = incl;
-      __syncthreads();
-      uint32_t before = 0;
-      for (int w = 0; w < warp; ++w) before += s_part[w];
-      before += incl - own;  // elements in buckets before this thread's (higher keys)
-      if (tid == TK_THREADS - 1) s_total = before + own;
-      if (above + before < static_cast<uint32_t>(K) &&
-          above + before + own >= static_cast<uint32_t>(K)) {
-        uint32_t c = above + before;
-        for (int j = 0; j < TK_WIN / TK_THREADS; ++j) {
-          c += hist[tid * (TK_WIN / TK_THREADS) + j];
-          if (c >= static_cast<uint32_t>(K)) {
-            s_thr = static_cast<uint32_t>(top - (tid * (TK_WIN / TK_THREADS) + j));
-            s_found = 1;
-            break;
-          }
-        }
-      }
-      __syncthreads();
-      if (s_found || lo <= 0) break;
-      above += s_total;
-      top = lo - 1;
-      __syncthreads();
+      if (lane == 31) sm.s_part[warp] = incl;
     }
-    const uint32_t thr = s_thr;
-    const float v_thr = key_value(thr);
+    __syncthreads();
+    if (warp < 8) {
+      uint32_t before = incl - c;
+      for (int w = 0; w < warp; ++w) before += sm.s_part[w];
+      if (before < need && before + c >= need) {
+        const uint32_t b = 255u - static_cast<uint32_t>(warp * 32 + lane);
+        sm.s_thr = (round == 0) ? b : ((prefix << 8) | b);
+        sm.s_total = before;  // keys above this bucket
+      }
+    }
+    __syncthreads();
+    if (round == 0) {
+      prefix = sm.s_thr;
+      need -= sm.s_total;
+    }
+    __syncthreads();
+  }
+  return sm.s_thr;
+}
 
-    // ---- pass 3: gather every element at or above the threshold
-    if (tid == 0) s_ncand = 0;
-    __syncthreads();
-    tk_for_row(z, V, vec8 != 0, [&](float v, uint32_t raw, int i) {
-      if (v >= v_thr) {
-        const uint32_t slot = atomicAdd(&s_ncand, 1u);
-        if (slot < TK_CAP)
-          cand[slot] = (static_cast<unsigned long long>(bf16_key(raw)) << 32) |
-                       (0xFFFFFFFFu - static_cast<uint32_t>(i));
+__global__ void __launch_bounds__(TK_THREADS, 2)
+topk_stream_kernel(const uint16_t* __restrict__ logits, int64_t T, int V, int K, int vec8,
+                   int32_t* __restrict__ idx_out, float* __restrict__ logp_out, int* status) {
+  __shared__ TkShared sm;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int64_t row = blockIdx.x; row < T; row += gridDim.x) {
+    const uint16_t* z = logits + row * static_cast<int64_t>(V);
+    // ---- pass 1: per-thread maximum and sum of exp against it
+    float cmax = -INFINITY;  // this thread's largest value so far
+    float cl = -INFINITY;    // cmax * log2 e
+    float s = 0.f;
+    auto rescale = [&](float vm) {
+      if (vm > cmax) {
+        const float nl = vm * LOG2E;
+        s *= ex2_approx(cl - nl);  // 0 while nothing was summed
+        cmax = vm;
+        cl = nl;
       }
-    });
-    __syncthreads();
-    const uint32_t n = min(s_ncand, static_cast<uint32_t>(TK_CAP));
-    if (tid == 0 && s_ncand > static_cast<uint32_t>(TK_CAP) && status != nullptr)
-      atomicOr(status, CKL_DEV_TOPK_TIES);
-    uint32_t P = 1;
-    while (P < n) P <<= 1;
-    for (uint32_t i = n + tid; i < P; i += TK_THREADS) cand[i] = 0ull;
-    __syncthreads();
-    // bitonic sort, descending
-    for (uint32_t k = 2; k <= P; k <<= 1) {
-      for (uint32_t j = k >> 1; j > 0; j >>= 1) {
-        for (uint32_t i = tid; i < P; i += TK_THREADS) {
-          const uint32_t ixj = i ^ j;
-          if (ixj > i) {
-            const unsigned long long a = cand[i], b = cand[ixj];
-            const bool up = (i & k) == 0;
-            if (up ? (a < b) : (a > b)) { cand[i] = b; cand[ixj] = a; }
-          }
+    };
+    if (vec8) {
+      const uint4* z4 = reinterpret_cast<const uint4*>(z);
+      const int n8 = V / 8;
+      for (int base = tid; base < n8; base += TK_THREADS * TS_UNROLL) {
+        uint4 v[TS_UNROLL];
+#pragma unroll
+        for (int u = 0; u < TS_UNROLL; ++u) {
+          const int i = base + u * TK_THREADS;
+          if (i < n8) v[u] = z4[i];
         }
-        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < TS_UNROLL; ++u) {
+          const int i = base + u * TK_THREADS;
+          if (i >= n8) continue;
+          const uint32_t m2 = bf16x2_max(bf16x2_max(v[u].x, v[u].y), bf16x2_max(v[u].z, v[u].w));
+          rescale(fmaxf(bf16_lo(m2), bf16_hi(m2)));
+          const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+          float a = 0.f, b = 0.f;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            a += ex2_approx(fmaf(bf16_lo(w[j]), LOG2E, -cl));
+            b += ex2_approx(fmaf(bf16_hi(w[j]), LOG2E, -cl));
+          }
+          s += a + b;
+        }
+      }
+    } else {
+      for (int i = tid; i < V; i += TK_THREADS) {
+        const float v = __uint_as_float(static_cast<uint32_t>(z[i]) << 16);
+        rescale(v);
+        s += ex2_approx(fmaf(v, LOG2E, -cl));
       }
     }
-    for (int k = tid; k < K; k += TK_THREADS) {
-      const unsigned long long e = cand[k];
-      const uint32_t key = static_cast<uint32_t>(e >> 32);
-      idx_out[row * K + k] = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(e));
-      logp_out[row * K + k] = key_value(key) - lse;
+    // ---- the row's log-sum-exp from the threads' (c, s) pairs
+    float wc = cl, ws = s;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float oc = __shfl_xor_sync(0xffffffffu, wc, o);
+      const float os = __shfl_xor_sync(0xffffffffu, ws, o);
+      const float nc = fmaxf(wc, oc);
+      ws = (nc == -INFINITY) ? 0.f : ws * ex2_approx(wc - nc) + os * ex2_approx(oc - nc);
+      wc = nc;
     }
-    __syncthreads();
+    if (lane == 0) { sm.s_c[warp] = wc; sm.s_s[warp] = ws; }
+    // ---- threshold: the K-th largest of the threads' maxima
+    const uint32_t my_key = (cmax == -INFINITY) ? 0u : bf16_key(__float_as_uint(cmax) >> 16);
+    const uint32_t thr = tk_kth_largest_key(sm, my_key, K);  // synchronises the block
+    float C = -INFINITY;
+    for (int w = 0; w < TK_THREADS / 32; ++w) C = fmaxf(C, sm.s_c[w]);
+    float S = 0.f;
+    for (int w = 0; w < TK_THREADS / 32; ++w) S += sm.s_s[w] * ex2_approx(sm.s_c[w] - C);
+    const float lse = (C + log2f(S)) * LN2;
+    const float v_thr = (thr == 0u) ? -INFINITY : key_value(thr);
+    // ---- pass 2: gather, sort, write
+    const uint32_t ncand = tk_gather(sm, z, V, vec8 != 0, v_thr);
+    if (ncand <= static_cast<uint32_t>(TK_CAP)) {
+      tk_sort_and_write(sm, ncand, K, lse, row, idx_out, logp_out);
+    } else if (tid == 0) {
+      idx_out[row * K] = -1;  // left to topk_fallback_kernel
+    }
+  }
+}
+
+// The rows topk_stream_kernel left (first id -1), by histogram windows.  A
+// kernel of its own, so that the streaming kernel's registers are not shaped
+// by a path it rarely takes.
+__global__ void __launch_bounds__(TK_THREADS, 2)
+topk_fallback_kernel(const uint16_t* __restrict__ logits, int64_t T, int V, int K, int vec8,
+                     int32_t* __restrict__ idx_out, float* __restrict__ logp_out, int* status) {
+  __shared__ TkShared sm;
+  for (int64_t row = blockIdx.x; row < T; row += gridDim.x) {
+    if (idx_out[row * K] != -1) continue;  // uniform over the block
+    tk_row_hist(sm, logits + row * static_cast<int64_t>(V), V, vec8 != 0, K, row, idx_out,
+                logp_out, status);
   }
 }
 

@@ -14,8 +14,12 @@ count on ALL ranks, so:
 * dW is summed over ranks with all-reduces issued while the backward is still
   running: the library reports each range of dW rows as soon as the launches
   that last write them are enqueued (``on_dw_ready``, one range per
-  vocabulary slab when the backward is sliced), and the all-reduce of that
-  range is queued right then, behind them, on the collective's stream.
+  vocabulary slab when the backward is sliced).  The ranges depend on the
+  rank's own row count (the blocking of its backward), but collectives must
+  be issued in the same order with the same sizes on every rank, so dW is
+  exchanged in fixed pieces that are the same on every rank: a piece's
+  all-reduce is queued, behind the launches that finish it, as soon as the
+  reported ranges cover it.
 
 The pages run on one GPU (their multi-node setup is the one the loss lets
 them leave); this is the exchange a data-parallel training step adds around
@@ -28,7 +32,7 @@ from __future__ import annotations
 import torch
 import torch.distributed as dist
 
-__all__ = ["dp_forward_backward"]
+__all__ = ["dp_forward_backward", "dw_pieces"]
 
 
 def dp_forward_backward(H, W, idx, logp, mask=None, chunk: int = 1024, grad_loss=None,
@@ -56,12 +60,30 @@ def dp_forward_backward(H, W, idx, logp, mask=None, chunk: int = 1024, grad_loss
     works = []
     if dW is None:
         dW = torch.empty(V, d, dtype=torch.float32, device=H.device)
+    bounds = dw_pieces(V)
+    state = {"next": 0}
 
     def ready(v0: int, v1: int):
-        works.append(dist.all_reduce(dW[v0:v1], group=group, async_op=True))
+        # ranges arrive in increasing order and partition [0, V): rows below
+        # v1 are final; exchange every piece that lies below it
+        while state["next"] < len(bounds) and bounds[state["next"]][1] <= v1:
+            b, e = bounds[state["next"]]
+            works.append(dist.all_reduce(dW[b:e], group=group, async_op=True))
+            state["next"] += 1
 
     dH, dW = ops.backward(H, W, idx, logp, mask, lse, grad_loss=g_local, chunk=chunk, dW=dW,
                           workspace=workspace, on_dw_ready=ready)
+    if state["next"] != len(bounds):
+        raise RuntimeError("the backward did not report every dW row as final")
     for w in works:
         w.wait()
     return loss, lse, dH, dW
+
+
+def dw_pieces(V: int, pieces: int = 8, align: int = 256):
+    """The fixed pieces [begin, end) of dW's rows exchanged one all-reduce
+    each: the same on every rank, since they depend on V alone."""
+    step = -(-V // pieces)
+    if V >= pieces * align:
+        step = -(-step // align) * align
+    return [(b, min(V, b + step)) for b in range(0, V, step)]
