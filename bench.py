@@ -310,9 +310,12 @@ def bench_ours(args):
                                 device_id=dev)
 
     import chunked_kl_loss_ckl_b200 as ckl
-    from ckl_synth import make_config
+    from ckl_synth import CONFIGS, make_config, student_topk_torch
 
-    c = make_config(args.config, seed=rank_seed(args.seed, rank))
+    # the GPT-OSS-shaped teacher ids come from the student's own top-200
+    # logits: input preparation, done with torch on the GPU before timing
+    topk = student_topk_torch if CONFIGS[args.config].get("neighbourhood") else None
+    c = make_config(args.config, seed=rank_seed(args.seed, rank), student_topk=topk)
     T, d, V, K, chunk = c["T"], c["d"], c["V"], c["K"], c["chunk"]
     to = lambda a, dt: torch.from_numpy(a).to(dev)
     H = to(c["H"].view(np.int16), None).view(torch.bfloat16)

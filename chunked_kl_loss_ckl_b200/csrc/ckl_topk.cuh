@@ -143,17 +143,19 @@ struct TkShared {
 
 // Sorts the row's n candidates (key << 32 | ~id) in shared memory, descending
 // (equal keys: smaller id first), and writes the first K: ids and z - lse.
-__device__ __forceinline__ void tk_sort_and_write(TkShared& sm, uint32_t n, int K, float lse,
+// NT = threads of the block.
+template <int NT = TK_THREADS, typename SM>
+__device__ __forceinline__ void tk_sort_and_write(SM& sm, uint32_t n, int K, float lse,
                                                   int64_t row, int32_t* idx_out,
                                                   float* logp_out) {
   const int tid = threadIdx.x;
   uint32_t P = 1;
   while (P < n) P <<= 1;
-  for (uint32_t i = n + tid; i < P; i += TK_THREADS) sm.cand[i] = 0ull;
+  for (uint32_t i = n + tid; i < P; i += NT) sm.cand[i] = 0ull;
   __syncthreads();
   for (uint32_t k = 2; k <= P; k <<= 1) {
     for (uint32_t j = k >> 1; j > 0; j >>= 1) {
-      for (uint32_t i = tid; i < P; i += TK_THREADS) {
+      for (uint32_t i = tid; i < P; i += NT) {
         const uint32_t ixj = i ^ j;
         if (ixj > i) {
           const unsigned long long a = sm.cand[i], b = sm.cand[ixj];
@@ -164,7 +166,7 @@ __device__ __forceinline__ void tk_sort_and_write(TkShared& sm, uint32_t n, int 
       __syncthreads();
     }
   }
-  for (int k = tid; k < K; k += TK_THREADS) {
+  for (int k = tid; k < K; k += NT) {
     const unsigned long long e = sm.cand[k];
     const uint32_t key = static_cast<uint32_t>(e >> 32);
     idx_out[row * K + k] = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(e));
@@ -175,7 +177,8 @@ __device__ __forceinline__ void tk_sort_and_write(TkShared& sm, uint32_t n, int 
 
 // Gathers every element of the row whose value is >= v_thr into the
 // candidates; returns their count (the array holds at most TK_CAP).
-__device__ __forceinline__ uint32_t tk_gather(TkShared& sm, const uint16_t* z, int V, bool vec8,
+template <int NT = TK_THREADS, int UNROLL = TK_UNROLL, typename SM>
+__device__ __forceinline__ uint32_t tk_gather(SM& sm, const uint16_t* z, int V, bool vec8,
                                               float v_thr) {
   if (threadIdx.x == 0) sm.s_ncand = 0;
   __syncthreads();
@@ -191,16 +194,16 @@ __device__ __forceinline__ uint32_t tk_gather(TkShared& sm, const uint16_t* z, i
     // a whole 8-element vector below the threshold is skipped on its maximum
     const uint4* z4 = reinterpret_cast<const uint4*>(z);
     const int n8 = V / 8;
-    for (int base = threadIdx.x; base < n8; base += TK_THREADS * TK_UNROLL) {
-      uint4 v[TK_UNROLL];
+    for (int base = threadIdx.x; base < n8; base += NT * UNROLL) {
+      uint4 v[UNROLL];
 #pragma unroll
-      for (int u = 0; u < TK_UNROLL; ++u) {
-        const int i = base + u * TK_THREADS;
+      for (int u = 0; u < UNROLL; ++u) {
+        const int i = base + u * NT;
         if (i < n8) v[u] = z4[i];
       }
 #pragma unroll
-      for (int u = 0; u < TK_UNROLL; ++u) {
-        const int i = base + u * TK_THREADS;
+      for (int u = 0; u < UNROLL; ++u) {
+        const int i = base + u * NT;
         if (i >= n8) continue;
         const uint32_t m2 = bf16x2_max(bf16x2_max(v[u].x, v[u].y), bf16x2_max(v[u].z, v[u].w));
         if (fmaxf(bf16_lo(m2), bf16_hi(m2)) < v_thr) continue;
@@ -213,7 +216,7 @@ __device__ __forceinline__ uint32_t tk_gather(TkShared& sm, const uint16_t* z, i
       }
     }
   } else {
-    for (int i = threadIdx.x; i < V; i += TK_THREADS) {
+    for (int i = threadIdx.x; i < V; i += NT) {
       const uint32_t b = z[i];
       put(__uint_as_float(b << 16), b, i);
     }
@@ -341,37 +344,58 @@ topk_cache_kernel(const uint16_t* __restrict__ logits, int64_t T, int V, int K, 
 // K-th value and a few more than K elements are gathered.  When more than
 // TK_CAP would be (the row's large values crowded into few threads), the
 // row is marked and done again by histogram windows in topk_fallback_kernel.
-// Needs K <= TK_THREADS.
-__device__ __forceinline__ uint32_t tk_kth_largest_key(TkShared& sm, uint32_t key, int K) {
-  // two 256-bucket rounds (high byte, then low byte) over the threads' keys
+// Blocks of TS_THREADS threads, four per SM, so that one block's HBM pass
+// overlaps another's selection; needs K <= TS_THREADS.
+constexpr int TS_THREADS = 256;
+
+struct TsShared {
+  unsigned long long cand[TK_CAP];
+  uint32_t hist[256];
+  float s_c[TS_THREADS / 32];
+  float s_s[TS_THREADS / 32];
+  uint32_t s_part[TS_THREADS / 32];
+  uint32_t s_thr, s_total, s_ncand;
+};
+
+// The K-th largest of the block's keys (one per thread; 0 = no element),
+// by two 256-bucket rounds: high byte, then low byte.
+__device__ __forceinline__ uint32_t ts_kth_largest_key(TsShared& sm, uint32_t key, int K) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int NW = TS_THREADS / 32;
+  constexpr int PER = 256 / TS_THREADS > 0 ? 256 / TS_THREADS : 1;  // buckets per thread
+  static_assert(TS_THREADS * PER == 256, "one or more whole buckets per thread");
   uint32_t prefix = 0, need = static_cast<uint32_t>(K);
   for (int round = 0; round < 2; ++round) {
-    for (int j = tid; j < 256; j += TK_THREADS) sm.hist[j] = 0;
+    for (int j = tid; j < 256; j += TS_THREADS) sm.hist[j] = 0;
     __syncthreads();
-    const bool in = (round == 0) || ((key >> 8) == prefix);
-    if (in) atomicAdd(&sm.hist[(round == 0) ? (key >> 8) : (key & 0xFFu)], 1u);
+    if (round == 0 || (key >> 8) == prefix)
+      atomicAdd(&sm.hist[(round == 0) ? (key >> 8) : (key & 0xFFu)], 1u);
     __syncthreads();
-    // suffix counts: warps 0..7 scan buckets 255..0, 32 each
-    uint32_t c = 0, incl = 0;
-    if (warp < 8) {
-      c = sm.hist[255 - (warp * 32 + lane)];
-      incl = c;
+    // thread tid owns buckets 255 - PER tid - j, j < PER (descending keys)
+    uint32_t own = 0;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      if (lane == 31) sm.s_part[warp] = incl;
+    for (int j = 0; j < PER; ++j) own += sm.hist[255 - (PER * tid + j)];
+    uint32_t incl = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
     }
+    if (lane == 31) sm.s_part[warp] = incl;
     __syncthreads();
-    if (warp < 8) {
-      uint32_t before = incl - c;
-      for (int w = 0; w < warp; ++w) before += sm.s_part[w];
-      if (before < need && before + c >= need) {
-        const uint32_t b = 255u - static_cast<uint32_t>(warp * 32 + lane);
-        sm.s_thr = (round == 0) ? b : ((prefix << 8) | b);
-        sm.s_total = before;  // keys above this bucket
+    uint32_t before = incl - own;
+    for (int w = 0; w < warp && w < NW; ++w) before += sm.s_part[w];
+    if (before < need && before + own >= need) {
+      uint32_t c = before;
+      for (int j = 0; j < PER; ++j) {
+        const uint32_t b = 255u - static_cast<uint32_t>(PER * tid + j);
+        const uint32_t h = sm.hist[b];
+        if (c + h >= need) {
+          sm.s_thr = (round == 0) ? b : ((prefix << 8) | b);
+          sm.s_total = c;  // keys above this bucket
+          break;
+        }
+        c += h;
       }
     }
     __syncthreads();
@@ -384,82 +408,81 @@ __device__ __forceinline__ uint32_t tk_kth_largest_key(TkShared& sm, uint32_t ke
   return sm.s_thr;
 }
 
-__global__ void __launch_bounds__(TK_THREADS, 2)
+__global__ void __launch_bounds__(TS_THREADS, 4)
 topk_stream_kernel(const uint16_t* __restrict__ logits, int64_t T, int V, int K, int vec8,
                    int32_t* __restrict__ idx_out, float* __restrict__ logp_out, int* status) {
-  __shared__ TkShared sm;
+  __shared__ TsShared sm;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int64_t row = blockIdx.x; row < T; row += gridDim.x) {
     const uint16_t* z = logits + row * static_cast<int64_t>(V);
     // ---- pass 1: per-thread maximum and sum of exp against it
     float cmax = -INFINITY;  // this thread's largest value so far
-    float cl = -INFINITY;    // cmax * log2 e
-    float s = 0.f;
+    float s = 0.f;           // sum of 2^((z - cmax) log2 e)
     auto rescale = [&](float vm) {
       if (vm > cmax) {
-        const float nl = vm * LOG2E;
-        s *= ex2_approx(cl - nl);  // 0 while nothing was summed
+        s *= ex2_approx((cmax - vm) * LOG2E);  // 0 while nothing was summed
         cmax = vm;
-        cl = nl;
       }
     };
     if (vec8) {
       const uint4* z4 = reinterpret_cast<const uint4*>(z);
       const int n8 = V / 8;
-      for (int base = tid; base < n8; base += TK_THREADS * TS_UNROLL) {
+      for (int base = tid; base < n8; base += TS_THREADS * TS_UNROLL) {
         uint4 v[TS_UNROLL];
 #pragma unroll
         for (int u = 0; u < TS_UNROLL; ++u) {
-          const int i = base + u * TK_THREADS;
+          const int i = base + u * TS_THREADS;
           if (i < n8) v[u] = z4[i];
         }
 #pragma unroll
         for (int u = 0; u < TS_UNROLL; ++u) {
-          const int i = base + u * TK_THREADS;
+          const int i = base + u * TS_THREADS;
           if (i >= n8) continue;
           const uint32_t m2 = bf16x2_max(bf16x2_max(v[u].x, v[u].y), bf16x2_max(v[u].z, v[u].w));
           rescale(fmaxf(bf16_lo(m2), bf16_hi(m2)));
           const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
           float a = 0.f, b = 0.f;
+          // z - cmax is exact for the values that matter (near the maximum)
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            a += ex2_approx(fmaf(bf16_lo(w[j]), LOG2E, -cl));
-            b += ex2_approx(fmaf(bf16_hi(w[j]), LOG2E, -cl));
+            a += ex2_approx((bf16_lo(w[j]) - cmax) * LOG2E);
+            b += ex2_approx((bf16_hi(w[j]) - cmax) * LOG2E);
           }
           s += a + b;
         }
       }
     } else {
-      for (int i = tid; i < V; i += TK_THREADS) {
+      for (int i = tid; i < V; i += TS_THREADS) {
         const float v = __uint_as_float(static_cast<uint32_t>(z[i]) << 16);
         rescale(v);
-        s += ex2_approx(fmaf(v, LOG2E, -cl));
+        s += ex2_approx((v - cmax) * LOG2E);
       }
     }
-    // ---- the row's log-sum-exp from the threads' (c, s) pairs
-    float wc = cl, ws = s;
+    // ---- the row's log-sum-exp from the threads' (cmax, s) pairs
+    float wc = cmax, ws = s;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       const float oc = __shfl_xor_sync(0xffffffffu, wc, o);
       const float os = __shfl_xor_sync(0xffffffffu, ws, o);
       const float nc = fmaxf(wc, oc);
-      ws = (nc == -INFINITY) ? 0.f : ws * ex2_approx(wc - nc) + os * ex2_approx(oc - nc);
+      ws = (nc == -INFINITY) ? 0.f
+                             : ws * ex2_approx((wc - nc) * LOG2E) + os * ex2_approx((oc - nc) * LOG2E);
       wc = nc;
     }
     if (lane == 0) { sm.s_c[warp] = wc; sm.s_s[warp] = ws; }
     // ---- threshold: the K-th largest of the threads' maxima
     const uint32_t my_key = (cmax == -INFINITY) ? 0u : bf16_key(__float_as_uint(cmax) >> 16);
-    const uint32_t thr = tk_kth_largest_key(sm, my_key, K);  // synchronises the block
+    const uint32_t thr = ts_kth_largest_key(sm, my_key, K);  // synchronises the block
     float C = -INFINITY;
-    for (int w = 0; w < TK_THREADS / 32; ++w) C = fmaxf(C, sm.s_c[w]);
+    for (int w = 0; w < TS_THREADS / 32; ++w) C = fmaxf(C, sm.s_c[w]);
     float S = 0.f;
-    for (int w = 0; w < TK_THREADS / 32; ++w) S += sm.s_s[w] * ex2_approx(sm.s_c[w] - C);
-    const float lse = (C + log2f(S)) * LN2;
+    for (int w = 0; w < TS_THREADS / 32; ++w) S += sm.s_s[w] * ex2_approx((sm.s_c[w] - C) * LOG2E);
+    const float lse = C + logf(S);
     const float v_thr = (thr == 0u) ? -INFINITY : key_value(thr);
     // ---- pass 2: gather, sort, write
-    const uint32_t ncand = tk_gather(sm, z, V, vec8 != 0, v_thr);
+    const uint32_t ncand = tk_gather<TS_THREADS, TS_UNROLL>(sm, z, V, vec8 != 0, v_thr);
     if (ncand <= static_cast<uint32_t>(TK_CAP)) {
-      tk_sort_and_write(sm, ncand, K, lse, row, idx_out, logp_out);
+      tk_sort_and_write<TS_THREADS>(sm, ncand, K, lse, row, idx_out, logp_out);
     } else if (tid == 0) {
       idx_out[row * K] = -1;  // left to topk_fallback_kernel
     }

@@ -13,4 +13,5 @@ from .inputs import (  # noqa: F401
     make_config,
     make_inputs,
     student_topk_numpy,
+    student_topk_torch,
 )

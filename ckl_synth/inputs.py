@@ -38,6 +38,7 @@ __all__ = [
     "make_inputs",
     "make_config",
     "student_topk_numpy",
+    "student_topk_torch",
 ]
 
 # The five workloads, with the pages' shapes (T tokens, d hidden, V vocab,
@@ -164,6 +165,27 @@ def student_topk_numpy(H_bits: np.ndarray, W_bits: np.ndarray, n: int,
         o = np.argsort(-zp, axis=1, kind="stable")
         out[r0:r1] = np.take_along_axis(part, o, axis=1)
     return out
+
+
+def student_topk_torch(H_bits: np.ndarray, W_bits: np.ndarray, n: int,
+                       block_rows: int = 1024) -> np.ndarray:
+    """``student_topk_numpy`` on the GPU (torch, fp32 products, no TF32):
+    the input recipe of the GPT-OSS-shaped teacher cache at full size."""
+    import torch
+    prev = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = False
+    try:
+        Wf = torch.from_numpy(W_bits.view(np.int16)).cuda().view(torch.bfloat16).float()
+        out = np.empty((H_bits.shape[0], n), dtype=np.int64)
+        for r0 in range(0, H_bits.shape[0], block_rows):
+            r1 = min(H_bits.shape[0], r0 + block_rows)
+            Hf = torch.from_numpy(H_bits[r0:r1].view(np.int16)).cuda().view(torch.bfloat16).float()
+            z = Hf @ Wf.T
+            out[r0:r1] = torch.topk(z, n, dim=1, sorted=True).indices.cpu().numpy()
+            del z
+        return out
+    finally:
+        torch.backends.cuda.matmul.allow_tf32 = prev
 
 
 def _teacher_logp(rng: np.random.Generator, n: int, k: int, std: float) -> np.ndarray:

@@ -74,20 +74,4 @@ def assert_parity(out, ref, tag=""):
     return e
 
 
-def student_topk_torch(H_bits, W_bits, n, block_rows: int = 1024):
-    """Top-n student logits per row (ids, descending) from fp32 W . h on the
-    GPU: the input recipe of the GPT-OSS-shaped teacher cache at full size."""
-    prev = torch.backends.cuda.matmul.allow_tf32
-    torch.backends.cuda.matmul.allow_tf32 = False
-    try:
-        Wf = torch.from_numpy(W_bits.view(np.int16)).cuda().view(torch.bfloat16).float()
-        out = np.empty((H_bits.shape[0], n), dtype=np.int64)
-        for r0 in range(0, H_bits.shape[0], block_rows):
-            r1 = min(H_bits.shape[0], r0 + block_rows)
-            Hf = torch.from_numpy(H_bits[r0:r1].view(np.int16)).cuda().view(torch.bfloat16).float()
-            z = Hf @ Wf.T
-            out[r0:r1] = torch.topk(z, n, dim=1, sorted=True).indices.cpu().numpy()
-            del z
-        return out
-    finally:
-        torch.backends.cuda.matmul.allow_tf32 = prev
+from ckl_synth import student_topk_torch  # noqa: E402,F401  (re-exported for the tests)

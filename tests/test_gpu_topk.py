@@ -108,16 +108,16 @@ def test_teacher_sized_many_rows_sampled(gpu_lib):
 
 
 def test_rows_whose_large_values_crowd_into_few_threads(gpu_lib):
-    # The streaming pass thresholds at the K-th largest of its 512 threads'
-    # maxima; thread t reads the 8-element vectors t, t + 512, ...  Giving
-    # every element of threads 0-11 a large value (about 3000 elements) puts
+    # The streaming pass thresholds at the K-th largest of its 256 threads'
+    # maxima; thread t reads the 8-element vectors t, t + 256, ...  Giving
+    # every element of threads 0-11 a large value (about 6000 elements) puts
     # far more than 2048 of them above that threshold, so the row is handed
     # to the histogram kernel, which must still return the exact top K.
     rng = np.random.default_rng(9)
     T, V, K = 6, 128256, 100
     z = rng.normal(0, 2, (T, V)).astype(np.float32)
     vec = np.arange(V // 8)
-    crowd = np.concatenate([8 * vec[vec % 512 == t][:, None] + np.arange(8)[None, :]
+    crowd = np.concatenate([8 * vec[vec % 256 == t][:, None] + np.arange(8)[None, :]
                             for t in range(12)]).ravel()
     assert crowd.size > 2048 + K
     for r in (1, 4):
