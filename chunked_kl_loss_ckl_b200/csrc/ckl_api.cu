@@ -47,6 +47,7 @@ struct Layout {
   int64_t cr_alloc; // rows the sliced schedule may hold (0 = never sliced)
   int64_t pitch_t;  // H_c^T row pitch (elements): max(cap, cr_alloc) rounded up to 8
   int64_t zpitch;   // single pass: fp32 logit row pitch (elements), V rounded up to 4
+  int64_t sp_rows;  // single pass: dZ rows held (the chunks of one dH/dW launch)
   int eb;           // bytes per H / W / dZ element: 2 (bf16) or 4 (fp32, tf32 MMAs)
 };
 
@@ -105,7 +106,12 @@ Layout forward_layout(int64_t T, int32_t K) {
   return L;
 }
 
-// single_pass adds the chunk's fp32 logits [cap][zpitch] and the rows' loss terms [T].
+// Chunks whose dZ the single pass gathers before one dH / dW launch: dW is
+// read-modify-written once per group instead of once per chunk.
+constexpr int64_t kSpGroup = 4;
+
+// single_pass adds the chunk's fp32 logits [cap][zpitch] and the rows' loss
+// terms [T], and holds the dZ of up to kSpGroup chunks.
 // eb = 4: the fp32 entry points (dZ and H_c^T in fp32; dH accumulates in the
 // caller's fp32 output, so no partial-dH buffer).
 Layout layout(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk, bool single_pass,
@@ -117,11 +123,13 @@ Layout layout(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk, bool si
   // largest chunk (a sliced block uses the same bytes as [Sv/64][Cr][64]).
   L.npanels = cdiv(V, 64);
   L.cap = std::min(chunk, std::max<int64_t>(T, 1));
+  L.sp_rows = single_pass ? std::min(kSpGroup, cdiv(std::max<int64_t>(T, 1), L.cap)) * L.cap
+                          : L.cap;
   L.dz = off;
-  off += align256(static_cast<size_t>(L.npanels) * L.cap * 64 * eb);
+  off += align256(static_cast<size_t>(L.npanels) * L.sp_rows * 64 * eb);
   // H_c^T for the dW GEMM: [d][pitch_t] bf16.
   L.cr_alloc = sliced_rows(T, d, V, L.cap, eb);
-  L.pitch_t = cdiv(std::max(L.cap, L.cr_alloc), 8) * 8;
+  L.pitch_t = cdiv(std::max(L.sp_rows, L.cr_alloc), 8) * 8;
   L.hct = off;
   off += align256(static_cast<size_t>(d) * L.pitch_t * eb);
   // fp32 dH of a sliced row chunk, summed over its vocabulary slabs.
@@ -578,9 +586,16 @@ int dhdw_block(const void* W, const uint8_t* mask, int64_t T, int64_t d, int64_t
   // swizzle with 32-byte chunks, the only MN-major layout of kind::tf32
   constexpr CUtensorMapSwizzle mn_sw =
       F32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B;
+  // W as the dH GEMM's MN-major B operand: viewed as [d / KE][V][KE] when d
+  // is a multiple of KE, so that one box carries a CTA's half_n columns per
+  // stage (half_n / KE atoms, ATOM_B apart); otherwise one 2-D box per atom
+  p.w3d = (d % KE == 0 &&
+           map3d2(&p.tm[1], kDT<F32>, W, KE, V, d / KE, d * eb, KE * eb, KE, KE,
+                  static_cast<uint32_t>(bn / kSlotCTAs / KE), mn_sw))
+              ? 1 : 0;
+  if (!p.w3d && !map2d(&p.tm[1], kDT<F32>, W, d, V, d * eb, KE, KE, mn_sw)) return CKL_ERR_CUDA;
   if (!map3d(&p.tm[0], kDT<F32>, dz, KE, rows, npan, 128, prow * 128, KE, ckl::BM,
              CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !map2d(&p.tm[1], kDT<F32>, W, d, V, d * eb, KE, KE, mn_sw) ||
       !map3d2(&p.tm[2], kDT<F32>, dz, KE, rows, npan, 128, prow * 128, KE, KE,
               static_cast<uint32_t>(ckl::BM / KE), mn_sw) ||
       !map2d(&p.tm[3], kDT<F32>, w8 + L.hct, rows, d, L.pitch_t * eb, KE, bn / kSlotCTAs,
@@ -833,8 +848,10 @@ int ckl_forward_backward(const uint16_t* H, const uint16_t* W, const int32_t* to
   Header* hdr = reinterpret_cast<Header*>(w8);
   float* z = reinterpret_cast<float*>(w8 + L.z);
   float* rowloss = reinterpret_cast<float*>(w8 + L.rowloss);
+  const int64_t grp = L.sp_rows;  // rows of one dH / dW launch: kSpGroup chunks
   for (int64_t c0 = 0; c0 < T; c0 += chunk) {
     const int64_t rows = std::min<int64_t>(chunk, T - c0);
+    const int64_t g0 = c0 / grp * grp;  // first row of this chunk's group
     const uint16_t* Hc = H + c0 * d;
     // ---- logits of this chunk, once: online log-sum-exp + gather partials and fp32 z
     TcParams p;
@@ -861,16 +878,20 @@ int ckl_forward_backward(const uint16_t* H, const uint16_t* W, const int32_t* to
       ckl::zrow_kernel<<<static_cast<unsigned>(rows), ckl::ZROW_THREADS, 0, st>>>(
           z, L.zpitch, reinterpret_cast<const float4*>(w8 + L.partials), p.S,
           reinterpret_cast<const float*>(w8 + L.hp), mask,
-          reinterpret_cast<const int2*>(w8 + L.pairs), K, static_cast<int>(V), c0, L.cap, lse,
-          rowloss, reinterpret_cast<uint16_t*>(w8 + L.dz));
+          reinterpret_cast<const int2*>(w8 + L.pairs), K, static_cast<int>(V), c0, grp, c0 - g0,
+          lse, rowloss, reinterpret_cast<uint16_t*>(w8 + L.dz));
       if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
     }
-    rc = transpose_rows<false>(H, d, c0, rows, w8, L, st, trace);
-    if (rc != CKL_OK) return rc;
-    rc = dhdw_block<false>(W, mask, T, d, V, K, c0, rows, L.cap, 0, V, 0,
-                    (c0 == 0 && !accumulate_dW) ? 1 : 0, grad_loss, dH + c0 * d, dW, w8, L, di,
-                    st, trace);
-    if (rc != CKL_OK) return rc;
+    // ---- dH and dW once the group's dZ is complete
+    if (c0 + rows == T || c0 + rows == g0 + grp) {
+      const int64_t grows = c0 + rows - g0;
+      rc = transpose_rows<false>(H, d, g0, grows, w8, L, st, trace);
+      if (rc != CKL_OK) return rc;
+      rc = dhdw_block<false>(W, mask, T, d, V, K, g0, grows, grp, 0, V, 0,
+                             (g0 == 0 && !accumulate_dW) ? 1 : 0, grad_loss, dH + g0 * d, dW,
+                             w8, L, di, st, trace);
+      if (rc != CKL_OK) return rc;
+    }
   }
   {
     TraceScope ts(trace, st, CKL_KERNEL_FWD_COMBINE);

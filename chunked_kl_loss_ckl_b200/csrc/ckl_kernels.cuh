@@ -96,6 +96,7 @@ struct alignas(64) TcParams {
   int32_t split_fast;  // FWD: units numbered split-fastest (see JobIter)
   int32_t dw_Ql, dw_El, dw_Qh, dw_Eh;  // DHDW rounds: quotas, see JobIter
   int32_t v_off;    // FWD / DZ: teacher id of local vocabulary column 0 (a vocabulary shard)
+  int32_t w3d;      // DHDW: tm[1] is the 3-D view of W (one box per stage for the dH B operand)
   const int2* pairs;      // [T, K] (id, p as bits), sorted by id per row
   float4* partials;       // FWD: [T, S] (max of z log2e, sum 2^(..), sum p z, 0)
   const float* lse;       // DZ: [T]
@@ -347,7 +348,9 @@ __global__ void wait_timeout_selftest_kernel(int* status, uint64_t limit_ns) {
 // splits into lse_t and its loss term m_t (Hp_t - pz_t + lse_t), then turn the
 // stored fp32 logits into dZ_t = m_t (exp(z - lse_t) - scatter p_t) as bf16 in
 // the 64-column panel layout the dH/dW GEMM reads (columns V .. round_up(V, 64)
-// are written 0).  Same arithmetic as the recompute path's dZ epilogue.
+// are written 0): panel rows of pitch `cap`, this chunk's rows from `drow0`
+// (several chunks share one dH/dW launch).  Same arithmetic as the recompute
+// path's dZ epilogue.
 constexpr int ZROW_THREADS = 512;
 constexpr int ZROW_UNROLL = 4;
 
@@ -355,11 +358,13 @@ __global__ void __launch_bounds__(ZROW_THREADS)
 zrow_kernel(const float* __restrict__ Z, int64_t zpitch, const float4* __restrict__ partials,
             int S, const float* __restrict__ Hp, const uint8_t* __restrict__ mask,
             const int2* __restrict__ pairs, int K, int V, int64_t row0, int64_t cap,
-            float* __restrict__ lse, float* __restrict__ rowloss, uint16_t* __restrict__ dz) {
+            int64_t drow0, float* __restrict__ lse, float* __restrict__ rowloss,
+            uint16_t* __restrict__ dz) {
   __shared__ float s_lse2;
   __shared__ int s_counts;
   const int r = blockIdx.x;
   const int64_t t = row0 + r;
+  const int64_t dr = drow0 + r;  // row within the dZ panels
   if (threadIdx.x == 0) {
     const float4* pr = partials + t * S;
     float M = -INFINITY;
@@ -406,7 +411,7 @@ zrow_kernel(const float* __restrict__ Z, int64_t zpitch, const float4* __restric
       uint2 o;
       o.x = pack_bf16x2(q[0], q[1]);
       o.y = pack_bf16x2(q[2], q[3]);
-      *reinterpret_cast<uint2*>(dz + ((static_cast<int64_t>(v >> 6) * cap + r) << 6) + (v & 63)) = o;
+      *reinterpret_cast<uint2*>(dz + ((static_cast<int64_t>(v >> 6) * cap + dr) << 6) + (v & 63)) = o;
     }
   }
   __syncthreads();
@@ -420,7 +425,7 @@ zrow_kernel(const float* __restrict__ Z, int64_t zpitch, const float4* __restric
       float x = ex2_approx(fmaf(zr[id], LOG2E, -lse2));
       for (int j = k; j < K && pr[j].x == id; ++j) x -= __int_as_float(pr[j].y);
       const uint32_t b = pack_bf16x2(x, 0.f);
-      dz[((static_cast<int64_t>(id >> 6) * cap + r) << 6) + (id & 63)] = static_cast<uint16_t>(b & 0xFFFFu);
+      dz[((static_cast<int64_t>(id >> 6) * cap + dr) << 6) + (id & 63)] = static_cast<uint16_t>(b & 0xFFFFu);
     }
   }
 }
@@ -744,8 +749,15 @@ tc_kernel(const __grid_constant__ TcParams p) {
             // MN-major here: one 64-column atom per box.
             if (PAIR) {
               tma_load_3d_pair(sa, &p.tm[0], fb, 0, a_y, kb);
-              for (int j = 0; j < half_n / KE; ++j)
-                tma_load_2d_pair(sb + j * ATOM_B, &p.tm[1], fb, b_x + KE * j, p.v_lo + kb * KE);
+              if (p.w3d) {
+                // W viewed as [d / KE][V][KE]: this CTA's half_n columns are
+                // half_n / KE atoms, one box, landing ATOM_B apart
+                tma_load_3d_pair(sb, &p.tm[1], fb, 0, p.v_lo + kb * KE, b_x / KE);
+              } else {
+                for (int j = 0; j < half_n / KE; ++j)
+                  tma_load_2d_pair(sb + j * ATOM_B, &p.tm[1], fb, b_x + KE * j,
+                                   p.v_lo + kb * KE);
+              }
             } else {
               tma_load_3d(sa, &p.tm[0], fb, 0, a_y, kb);
               for (int j = 0; j < half_n / KE; ++j)
@@ -813,18 +825,23 @@ tc_kernel(const __grid_constant__ TcParams p) {
         if (!mbar_wait(bar_tempty + 8 * acc, acc_phase ^ 1u, p.status)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc) * ACC_COLS;
+        // descriptors of stage 0's operands for this job (a_mn / b_mn: that
+        // operand is MN-major, dH's W or dW's dZ^T); a stage, or a K step
+        // within it, only moves the start address, the low 14 bits in
+        // 16-byte units, which stay below 2^14 for any shared-memory address
+        const uint64_t ad0 = (F32 && a_mn) ? sdesc_sw128_b32(sbase + C::A_OFF, a_lbo, MN_SBO)
+                                           : sdesc_sw128(sbase + C::A_OFF, a_lbo, 1024);
+        const uint64_t bd0 = (F32 && b_mn) ? sdesc_sw128_b32(sbase + C::B_OFF, b_lbo, MN_SBO)
+                                           : sdesc_sw128(sbase + C::B_OFF, b_lbo, 1024);
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(bar_full + 8 * stage, phase, p.status)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sa = sbase + C::A_OFF + stage * A_BYTES;
-          const uint32_t sb = sbase + C::B_OFF + stage * B_STAGE;
+          const uint64_t ads = ad0 + static_cast<uint64_t>((stage * A_BYTES) >> 4);
+          const uint64_t bds = bd0 + static_cast<uint64_t>((stage * B_STAGE) >> 4);
 #pragma unroll
           for (int kk = 0; kk < KE / KI; ++kk) {
-            // a_mn / b_mn: that operand is MN-major (dH's W, dW's dZ^T)
-            const uint64_t ad = (F32 && a_mn) ? sdesc_sw128_b32(sa + kk * a_step, a_lbo, MN_SBO)
-                                              : sdesc_sw128(sa + kk * a_step, a_lbo, 1024);
-            const uint64_t bd = (F32 && b_mn) ? sdesc_sw128_b32(sb + kk * b_step, b_lbo, MN_SBO)
-                                              : sdesc_sw128(sb + kk * b_step, b_lbo, 1024);
+            const uint64_t ad = ads + static_cast<uint64_t>((kk * a_step) >> 4);
+            const uint64_t bd = bds + static_cast<uint64_t>((kk * b_step) >> 4);
             const uint32_t acc_in = (kb | kk) != 0 ? 1u : 0u;
             if constexpr (F32) {
               if (PAIR) umma_tf32_pair(d_tmem, ad, bd, idesc, acc_in);

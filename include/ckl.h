@@ -196,8 +196,10 @@ CKL_API int ckl_backward(const uint16_t* H, const uint16_t* W, const int32_t* to
  * forward-chunked).  This entry point drops the recompute: per chunk of rows
  * it runs the logit GEMM once, storing the chunk's fp32 logits (chunk x V)
  * beside the online log-sum-exp, turns them into dZ once lse is known, and
- * feeds dZ to the same dH / dW GEMMs as ckl_backward.  6 d V FLOP per token
- * instead of 8 d V, for chunk x V x 4 more workspace bytes.  Results equal
+ * feeds dZ to the same dH / dW GEMMs as ckl_backward, once per group of up
+ * to four chunks (so dW is read and written once per group).  6 d V FLOP per
+ * token instead of 8 d V, for chunk x V x 4 more workspace bytes (the fp32
+ * logits) and a dZ buffer of up to 4 chunks x V bf16.  Results equal
  * ckl_forward followed by ckl_backward up to rounding (lse may differ in the
  * last bits: the vocabulary is split differently per chunk).
  *   grad_loss  [1]    fp32  upstream gradient g (device); NULL = 1

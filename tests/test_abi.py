@@ -60,13 +60,16 @@ def test_workspace_is_linear_in_T(ckl):
 
 
 def test_single_pass_workspace_adds_the_chunk_logits(ckl):
+    # fp32 logits of one chunk, the rows' loss terms, and dZ for up to four
+    # chunks (one dH / dW launch per four chunks) instead of one
     d, V, K, chunk = 3072, 128256, 100, 1024
-    for T in (100, 8192, 32768):
+    for T in (100, 2500, 8192, 32768):
         base = ckl.lib.ckl_workspace_bytes(T, d, V, K, chunk)
         sp = ckl.lib.ckl_single_pass_workspace_bytes(T, d, V, K, chunk)
         rows = min(chunk, T)
-        extra = rows * ((V + 3) // 4 * 4) * 4 + T * 4  # fp32 logits + per-row loss terms
-        assert extra <= sp - base <= extra + 512
+        group = min(4, -(-T // rows))
+        extra = rows * ((V + 3) // 4 * 4) * 4 + T * 4 + (group - 1) * rows * (-(-V // 64) * 64) * 2
+        assert extra <= sp - base <= extra + 1024 + d * group * rows * 2, T
     assert ckl.lib.ckl_single_pass_workspace_bytes(10, 60, 100, 4, 8) == 0
 
 
