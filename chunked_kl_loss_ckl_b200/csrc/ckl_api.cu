@@ -922,7 +922,7 @@ int ckl_topk_cache(const uint16_t* teacher_logits, int64_t T, int64_t V, int32_t
   const int vec8 = (V % 8 == 0 && aligned16(teacher_logits)) ? 1 : 0;
   const int grid = static_cast<int>(std::min<int64_t>(T, static_cast<int64_t>(di.sms) * 2));
   if (K <= ckl::TS_THREADS) {
-    const int sgrid = static_cast<int>(std::min<int64_t>(T, static_cast<int64_t>(di.sms) * 4));
+    const int sgrid = static_cast<int>(std::min<int64_t>(T, static_cast<int64_t>(di.sms) * 3));
     ckl::topk_stream_kernel<<<sgrid, ckl::TS_THREADS, 0, st>>>(
         teacher_logits, T, static_cast<int>(V), K, vec8, topk_idx, topk_logp, device_status);
     if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
