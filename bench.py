@@ -108,6 +108,37 @@ def flops_per_token(c):
     return 8.0 * c["d"] * c["V"]
 
 
+def backward_blocks(T, V, plan):
+    """(rows, cols) of each block of the backward, in order (row chunks of
+    plan[0] rows, each swept in plan[2] vocabulary slabs of plan[1] columns)."""
+    Cr, Sv, n = plan
+    out = []
+    for r0 in range(0, T, Cr):
+        for s in range(n):
+            out.append((min(Cr, T - r0), min(Sv, V - s * Sv)))
+    return out
+
+
+def backward_launches(T, V, plan):
+    """Tensor-core launches of one backward per kernel: the first block's dZ,
+    then per block its dH and dW together with the next block's dZ (one fused
+    launch), the last block's dH and dW alone."""
+    nb = len(backward_blocks(T, V, plan))
+    return {"fwd_gemm": 1, "bwd_dz": 1, "bwd_fused": nb - 1, "bwd_dhdw": 1}
+
+
+def kernel_flops_per_step(T, d, V, plan):
+    """FLOPs of one forward + backward per tensor-core kernel: the logits 2 T V
+    d, each block's recomputed logits 2 rows cols d and its dH + dW 4 rows cols
+    d (8 d V per token in all)."""
+    blocks = backward_blocks(T, V, plan)
+    dz = [2.0 * r * c * d for r, c in blocks]
+    hw = [4.0 * r * c * d for r, c in blocks]
+    return {"fwd_gemm": 2.0 * T * V * d, "bwd_dz": dz[0],
+            "bwd_fused": sum(hw[b] + dz[b + 1] for b in range(len(blocks) - 1)),
+            "bwd_dhdw": hw[-1]}
+
+
 # ----------------------------------------------------------------- distributed
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
@@ -348,7 +379,7 @@ def bench_ours(args):
     # conversion when sliced; the capacity leaves headroom and a full trace is
     # treated as an error below.
     Cr, Sv, n_slabs = ckl.backward_plan(T, d, V, K, chunk)
-    n_launch = 3 + 1 + -(-T // Cr) * (1 + 2 * n_slabs + (1 if n_slabs > 1 else 0))
+    n_launch = 3 + 2 + -(-T // Cr) * (2 + 2 * n_slabs + (1 if n_slabs > 1 else 0))
     trace = ckl.Trace(capacity=args.steps * (n_launch + 4) + 16)
     uuid = None
     try:
@@ -390,12 +421,12 @@ def bench_ours(args):
     gpu_launches = trace.count
     peaks, peak_src = load_peaks()
     # algorithmic FLOPs per launch of each tensor-core kernel: its FLOPs per
-    # step (forward logits 2 T V d; recompute 2 T V d; dH + dW 4 T V d) over
-    # its launches per step (the backward's blocking sets the count)
+    # step over its launches per step (the backward's blocking sets them)
     chunks = (T + chunk - 1) // chunk
-    per_step = {"fwd_gemm": 2.0 * T * V * d, "bwd_dz": 2.0 * T * V * d,
-                "bwd_dhdw": 4.0 * T * V * d}
-    alg = {k: v / (per[k][0] / args.steps) for k, v in per_step.items() if k in per}
+    per_step = kernel_flops_per_step(T, d, V, (Cr, Sv, n_slabs))
+    alg = {k: v / (per[k][0] / args.steps) for k, v in per_step.items()
+           if k in per and v > 0 and per[k][0] == args.steps * backward_launches(
+               T, V, (Cr, Sv, n_slabs)).get(k, 1)}
     dom = max(per, key=lambda k: per[k][1])
     dom_avg_ms = per[dom][1] / per[dom][0]
     roofline = None

@@ -58,7 +58,10 @@ __device__ __forceinline__ uint32_t bf16_key2(uint32_t w) {
 }
 
 constexpr int TK_UNROLL = 2;  // independent 16-byte loads in flight per thread
-constexpr int TS_UNROLL = 4;  // the same, in the streaming form's pass
+#ifndef CKL_TS_UNROLL
+#define CKL_TS_UNROLL 8
+#endif
+constexpr int TS_UNROLL = CKL_TS_UNROLL;  // the same, in the streaming form's pass
 
 __device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
   uint32_t r;
@@ -332,26 +335,26 @@ topk_cache_kernel(const uint16_t* __restrict__ logits, int64_t T, int V, int K, 
 }
 
 // ------------------------------------------------------------ streaming form
-// One pass over each row from HBM.  Every thread keeps, in registers, the
-// TS_KEEP best elements it has read (by value, equal values: smaller id
-// first) and its running maximum c with the sum of 2^((z - c) log2 e) over
-// its elements, rescaled when c grows; an element is compared with the
-// thread's TS_KEEP-th best only when its 8-element vector's maximum beats it.
-// The block then
-//   - merges the (c, sum) pairs into the row's log-sum-exp;
-//   - finds tau, the K-th largest key among all kept elements (a lower bound
-//     of the row's K-th largest, since those K are elements of the row);
-//   - keeps the result exact by construction: a thread whose list is full
-//     may have dropped elements no better than its last kept one, so if every
-//     such last key is below tau, every element at or above tau was kept.
-// Then the kept elements at or above tau are sorted and the first K written.
-// A row where some thread's last kept key reaches tau (its large values
-// crowded into one thread) is read again from memory and every element at or
-// above tau gathered; if more than TK_CAP are, the row is marked and done by
-// histogram windows in topk_fallback_kernel.  Blocks of TS_THREADS threads,
-// three per SM; needs K <= TS_THREADS * TS_KEEP.
+// Two passes per row.  Pass 1 (the only one from HBM): every thread keeps
+// its running maximum c and the sum of 2^((z - c) log2 e) over its own
+// elements, rescaled when c grows (at most once per 8-element vector); the
+// block merges the (c, sum) pairs into the row's log-sum-exp.  The K-th
+// largest of the threads' maxima is at most the row's K-th largest value
+// (those K maxima are K elements of the row), so it is a valid threshold:
+// pass 2 (from L2) gathers every element at or above it, vectors whose
+// maximum is below it skipped whole, and the sort keeps the first K.  With
+// the row's top K spread over the threads, the threshold sits just below the
+// K-th value and a few more than K elements are gathered.  When more than
+// TK_CAP would be (the row's large values crowded into few threads), the
+// row is marked and done again by histogram windows in topk_fallback_kernel.
+// Blocks of TS_THREADS threads, TS_BLOCKS per SM: enough rows in flight to
+// keep HBM busy, few enough (TS_BLOCKS x SMs x 256 KB at V = 128 256) that
+// pass 2 finds its row still in L2; needs K <= TS_THREADS.
 constexpr int TS_THREADS = 256;
-constexpr int TS_KEEP = 8;
+#ifndef CKL_TS_BLOCKS
+#define CKL_TS_BLOCKS 2
+#endif
+constexpr int TS_BLOCKS = CKL_TS_BLOCKS;  // blocks per SM
 
 struct TsShared {
   unsigned long long cand[TK_CAP];
@@ -362,29 +365,24 @@ struct TsShared {
   uint32_t s_thr, s_total, s_ncand;
 };
 
-// The K-th largest of the block's kept keys (entries key << 32 | ~id; 0 =
-// empty, never counted), by two 256-bucket rounds: high byte, then low byte.
-// Returns 0 when fewer than K keys are kept.
-__device__ __forceinline__ uint32_t ts_kth_largest_key(TsShared& sm,
-                                                       const unsigned long long (&e)[TS_KEEP],
-                                                       int K) {
+// The K-th largest of the block's keys (one per thread; 0 = no element),
+// by two 256-bucket rounds: high byte, then low byte.
+__device__ __forceinline__ uint32_t ts_kth_largest_key(TsShared& sm, uint32_t key, int K) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  static_assert(TS_THREADS == 256, "one histogram bucket per thread");
+  constexpr int NW = TS_THREADS / 32;
+  constexpr int PER = 256 / TS_THREADS > 0 ? 256 / TS_THREADS : 1;  // buckets per thread
+  static_assert(TS_THREADS * PER == 256, "one or more whole buckets per thread");
   uint32_t prefix = 0, need = static_cast<uint32_t>(K);
-  if (tid == 0) sm.s_thr = 0;
-  bool few = false;  // fewer than K keys kept: every kept key counts
   for (int round = 0; round < 2; ++round) {
-    sm.hist[tid] = 0;
+    for (int j = tid; j < 256; j += TS_THREADS) sm.hist[j] = 0;
     __syncthreads();
+    if (round == 0 || (key >> 8) == prefix)
+      atomicAdd(&sm.hist[(round == 0) ? (key >> 8) : (key & 0xFFu)], 1u);
+    __syncthreads();
+    // thread tid owns buckets 255 - PER tid - j, j < PER (descending keys)
+    uint32_t own = 0;
 #pragma unroll
-    for (int j = 0; j < TS_KEEP; ++j) {
-      const uint32_t key = static_cast<uint32_t>(e[j] >> 32);
-      if (e[j] != 0ull && (round == 0 || (key >> 8) == prefix))
-        atomicAdd(&sm.hist[(round == 0) ? (key >> 8) : (key & 0xFFu)], 1u);
-    }
-    __syncthreads();
-    // thread tid owns bucket 255 - tid (descending keys)
-    const uint32_t own = sm.hist[255 - tid];
+    for (int j = 0; j < PER; ++j) own += sm.hist[255 - (PER * tid + j)];
     uint32_t incl = own;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -393,19 +391,20 @@ __device__ __forceinline__ uint32_t ts_kth_largest_key(TsShared& sm,
     }
     if (lane == 31) sm.s_part[warp] = incl;
     __syncthreads();
-    uint32_t before = incl - own, total = 0;
-    for (int w = 0; w < TS_THREADS / 32; ++w) {
-      if (w < warp) before += sm.s_part[w];
-      total += sm.s_part[w];
-    }
-    if (round == 0 && total < need) {  // the same on every thread
-      few = true;
-      break;
-    }
+    uint32_t before = incl - own;
+    for (int w = 0; w < warp && w < NW; ++w) before += sm.s_part[w];
     if (before < need && before + own >= need) {
-      const uint32_t b = 255u - static_cast<uint32_t>(tid);
-      sm.s_thr = (round == 0) ? b : ((prefix << 8) | b);
-      sm.s_total = before;  // keys above this bucket
+      uint32_t c = before;
+      for (int j = 0; j < PER; ++j) {
+        const uint32_t b = 255u - static_cast<uint32_t>(PER * tid + j);
+        const uint32_t h = sm.hist[b];
+        if (c + h >= need) {
+          sm.s_thr = (round == 0) ? b : ((prefix << 8) | b);
+          sm.s_total = c;  // keys above this bucket
+          break;
+        }
+        c += h;
+      }
     }
     __syncthreads();
     if (round == 0) {
@@ -414,45 +413,23 @@ __device__ __forceinline__ uint32_t ts_kth_largest_key(TsShared& sm,
     }
     __syncthreads();
   }
-  const uint32_t r = few ? 0u : sm.s_thr;
-  __syncthreads();
-  return r;
+  return sm.s_thr;
 }
 
-__global__ void __launch_bounds__(TS_THREADS, 3)
+__global__ void __launch_bounds__(TS_THREADS, TS_BLOCKS)
 topk_stream_kernel(const uint16_t* __restrict__ logits, int64_t T, int V, int K, int vec8,
                    int32_t* __restrict__ idx_out, float* __restrict__ logp_out, int* status) {
   __shared__ TsShared sm;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int64_t row = blockIdx.x; row < T; row += gridDim.x) {
     const uint16_t* z = logits + row * static_cast<int64_t>(V);
-    // ---- the pass: per-thread maximum, sum of exp against it, best elements
+    // ---- pass 1: per-thread maximum and sum of exp against it
     float cmax = -INFINITY;  // this thread's largest value so far
     float s = 0.f;           // sum of 2^((z - cmax) log2 e)
-    unsigned long long best[TS_KEEP];  // descending; 0 = empty
-#pragma unroll
-    for (int j = 0; j < TS_KEEP; ++j) best[j] = 0ull;
-    float v_last = -INFINITY;  // value of best[TS_KEEP - 1], -inf while the list has room
     auto rescale = [&](float vm) {
       if (vm > cmax) {
         s *= ex2_approx((cmax - vm) * LOG2E);  // 0 while nothing was summed
         cmax = vm;
-      }
-    };
-    auto keep = [&](float v, uint32_t raw, int id) {
-      if (v > v_last) {  // an equal value comes later, so with a larger id: worse
-        unsigned long long x = (static_cast<unsigned long long>(bf16_key(raw)) << 32) |
-                               (0xFFFFFFFFu - static_cast<uint32_t>(id));
-#pragma unroll
-        for (int j = 0; j < TS_KEEP; ++j) {
-          const unsigned long long b = best[j];
-          const bool up = x > b;
-          best[j] = up ? x : b;
-          x = up ? b : x;
-        }
-        v_last = (best[TS_KEEP - 1] == 0ull)
-                     ? -INFINITY
-                     : key_value(static_cast<uint32_t>(best[TS_KEEP - 1] >> 32));
       }
     };
     if (vec8) {
@@ -470,8 +447,7 @@ topk_stream_kernel(const uint16_t* __restrict__ logits, int64_t T, int V, int K,
           const int i = base + u * TS_THREADS;
           if (i >= n8) continue;
           const uint32_t m2 = bf16x2_max(bf16x2_max(v[u].x, v[u].y), bf16x2_max(v[u].z, v[u].w));
-          const float vm = fmaxf(bf16_lo(m2), bf16_hi(m2));
-          rescale(vm);
+          rescale(fmaxf(bf16_lo(m2), bf16_hi(m2)));
           const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
           float a = 0.f, b = 0.f;
           // z - cmax is exact for the values that matter (near the maximum)
@@ -481,22 +457,13 @@ topk_stream_kernel(const uint16_t* __restrict__ logits, int64_t T, int V, int K,
             b += ex2_approx((bf16_hi(w[j]) - cmax) * LOG2E);
           }
           s += a + b;
-          if (vm > v_last) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              keep(bf16_lo(w[j]), w[j] & 0xFFFFu, 8 * i + 2 * j);
-              keep(bf16_hi(w[j]), w[j] >> 16, 8 * i + 2 * j + 1);
-            }
-          }
         }
       }
     } else {
       for (int i = tid; i < V; i += TS_THREADS) {
-        const uint32_t raw = z[i];
-        const float v = __uint_as_float(raw << 16);
+        const float v = __uint_as_float(static_cast<uint32_t>(z[i]) << 16);
         rescale(v);
         s += ex2_approx((v - cmax) * LOG2E);
-        keep(v, raw, i);
       }
     }
     // ---- the row's log-sum-exp from the threads' (cmax, s) pairs
@@ -511,33 +478,17 @@ topk_stream_kernel(const uint16_t* __restrict__ logits, int64_t T, int V, int K,
       wc = nc;
     }
     if (lane == 0) { sm.s_c[warp] = wc; sm.s_s[warp] = ws; }
-    // ---- tau, and whether the kept elements hold everything at or above it
-    const uint32_t tau = ts_kth_largest_key(sm, best, K);  // synchronises the block
+    // ---- threshold: the K-th largest of the threads' maxima
+    const uint32_t my_key = (cmax == -INFINITY) ? 0u : bf16_key(__float_as_uint(cmax) >> 16);
+    const uint32_t thr = ts_kth_largest_key(sm, my_key, K);  // synchronises the block
     float C = -INFINITY;
     for (int w = 0; w < TS_THREADS / 32; ++w) C = fmaxf(C, sm.s_c[w]);
     float S = 0.f;
     for (int w = 0; w < TS_THREADS / 32; ++w) S += sm.s_s[w] * ex2_approx((sm.s_c[w] - C) * LOG2E);
     const float lse = C + logf(S);
-    const bool full = best[TS_KEEP - 1] != 0ull;
-    const bool unsure = full && static_cast<uint32_t>(best[TS_KEEP - 1] >> 32) >= tau;
-    if (tid == 0) sm.s_ncand = 0;
-    const bool again = __syncthreads_or(unsure ? 1 : 0) != 0;
-    uint32_t ncand;
-    if (!again) {
-#pragma unroll
-      for (int j = 0; j < TS_KEEP; ++j) {
-        if (best[j] != 0ull && static_cast<uint32_t>(best[j] >> 32) >= tau) {
-          const uint32_t slot = atomicAdd(&sm.s_ncand, 1u);
-          sm.cand[slot] = best[j];  // at most TS_THREADS * TS_KEEP = TK_CAP entries
-        }
-      }
-      __syncthreads();
-      ncand = sm.s_ncand;
-    } else {
-      // ---- rare: read the row again and gather every element at or above tau
-      ncand = tk_gather<TS_THREADS, TS_UNROLL>(sm, z, V, vec8 != 0,
-                                               tau == 0u ? -INFINITY : key_value(tau));
-    }
+    const float v_thr = (thr == 0u) ? -INFINITY : key_value(thr);
+    // ---- pass 2: gather, sort, write
+    const uint32_t ncand = tk_gather<TS_THREADS, TS_UNROLL>(sm, z, V, vec8 != 0, v_thr);
     if (ncand <= static_cast<uint32_t>(TK_CAP)) {
       tk_sort_and_write<TS_THREADS>(sm, ncand, K, lse, row, idx_out, logp_out);
     } else if (tid == 0) {

@@ -63,3 +63,16 @@ def test_clock_summary_keeps_only_samples_inside_the_timed_region():
 def test_cpu_description_names_the_host():
     model, n = bench.cpu_description()
     assert n >= 1 and (model is None or isinstance(model, str))
+
+
+def test_backward_flops_add_up_to_6dV_per_token():
+    # the per-kernel split of the backward (first block's dZ, fused dH/dW +
+    # next dZ launches, last block's dH/dW) covers 6 d V per token exactly
+    for T, d, V, plan in ((8192, 3072, 128256, (8192, 14336, 9)),
+                          (262144, 4096, 128256, (6144, 64256, 2)),
+                          (1000, 64, 3000, (256, 3008, 1))):
+        f = bench.kernel_flops_per_step(T, d, V, plan)
+        back = f["bwd_dz"] + f["bwd_fused"] + f["bwd_dhdw"]
+        assert abs(back - 6.0 * T * V * d) <= 1e-9 * back
+        n = bench.backward_launches(T, V, plan)
+        assert n["bwd_fused"] == len(bench.backward_blocks(T, V, plan)) - 1
