@@ -120,11 +120,10 @@ def backward_blocks(T, V, plan):
 
 
 def backward_launches(T, V, plan):
-    """Tensor-core launches of one backward per kernel: the first block's dZ,
-    then per block its dH and dW together with the next block's dZ (one fused
-    launch), the last block's dH and dW alone."""
+    """Tensor-core launches of one forward + backward per kernel: the logits
+    once, and per backward block its dZ and its dH + dW."""
     nb = len(backward_blocks(T, V, plan))
-    return {"fwd_gemm": 1, "bwd_dz": 1, "bwd_fused": nb - 1, "bwd_dhdw": 1}
+    return {"fwd_gemm": 1, "bwd_dz": nb, "bwd_dhdw": nb}
 
 
 def kernel_flops_per_step(T, d, V, plan):
@@ -132,11 +131,8 @@ def kernel_flops_per_step(T, d, V, plan):
     d, each block's recomputed logits 2 rows cols d and its dH + dW 4 rows cols
     d (8 d V per token in all)."""
     blocks = backward_blocks(T, V, plan)
-    dz = [2.0 * r * c * d for r, c in blocks]
-    hw = [4.0 * r * c * d for r, c in blocks]
-    return {"fwd_gemm": 2.0 * T * V * d, "bwd_dz": dz[0],
-            "bwd_fused": sum(hw[b] + dz[b + 1] for b in range(len(blocks) - 1)),
-            "bwd_dhdw": hw[-1]}
+    return {"fwd_gemm": 2.0 * T * V * d, "bwd_dz": sum(2.0 * r * c * d for r, c in blocks),
+            "bwd_dhdw": sum(4.0 * r * c * d for r, c in blocks)}
 
 
 # ----------------------------------------------------------------- distributed
@@ -379,7 +375,7 @@ def bench_ours(args):
     # conversion when sliced; the capacity leaves headroom and a full trace is
     # treated as an error below.
     Cr, Sv, n_slabs = ckl.backward_plan(T, d, V, K, chunk)
-    n_launch = 3 + 2 + -(-T // Cr) * (2 + 2 * n_slabs + (1 if n_slabs > 1 else 0))
+    n_launch = 3 + 1 + -(-T // Cr) * (1 + 2 * n_slabs + (1 if n_slabs > 1 else 0))
     trace = ckl.Trace(capacity=args.steps * (n_launch + 4) + 16)
     uuid = None
     try:

@@ -37,7 +37,7 @@ STATUS_NAMES = {
     8: "CKL_ERR_TOPK_TIES",
 }
 KERNEL_NAMES = {1: "prep", 2: "fwd_gemm", 3: "fwd_combine", 4: "bwd_dz", 5: "bwd_dhdw", 6: "other",
-                7: "topk", 8: "sp_gemm", 9: "sp_rows", 10: "bwd_fused"}
+                7: "topk", 8: "sp_gemm", 9: "sp_rows"}
 
 
 class CklError(RuntimeError):

@@ -41,7 +41,7 @@ struct Plan {
 };
 
 struct Layout {
-  size_t pairs, hp, partials, blocksums, dz, hct, dep, dh32, z, rowloss, total;
+  size_t pairs, hp, partials, blocksums, dz, hct, dh32, z, rowloss, total;
   int64_t npanels;  // dZ panels of 64 vocabulary columns (row-chunked schedule)
   int64_t cap;      // rows of one chunk: min(chunk, T)
   int64_t cr_alloc; // rows the sliced schedule may hold (0 = never sliced)
@@ -132,10 +132,6 @@ Layout layout(int64_t T, int64_t d, int64_t V, int32_t K, int64_t chunk, bool si
   L.pitch_t = cdiv(std::max(L.sp_rows, L.cr_alloc), 8) * 8;
   L.hct = off;
   off += align256(static_cast<size_t>(d) * L.pitch_t * eb);
-  // counters ordering the fused dH / dW + next dZ launches (one per dZ
-  // vocabulary block of 256, and one for the dH units)
-  L.dep = off;
-  off += align256(static_cast<size_t>(cdiv(V, 256) + 2) * 4);
   // fp32 dH of a sliced row chunk, summed over its vocabulary slabs.
   L.dh32 = off;
   if (eb == 2) off += align256(static_cast<size_t>(L.cr_alloc) * d * 4);
@@ -233,7 +229,7 @@ struct DevInfo {
   int sms = 0;
   int major = 0;
   bool attrs_set = false;
-  int slots[5] = {0, 0, 0, 0, 0};  // co-resident CTA pairs per GEMM mode
+  int slots[4] = {0, 0, 0, 0};  // co-resident CTA pairs per GEMM mode
 };
 
 // Element type of a launch's operands: bf16 (kind::f16) or fp32 (kind::tf32).
@@ -268,7 +264,7 @@ bool setup_mode(DevInfo& di) {
       cudaSuccess)
     return false;
   // the fp32 form has the same shared memory and threads, so the same occupancy
-  if constexpr (MODE != ckl::MODE_FWDZ && MODE != ckl::MODE_BWD) {
+  if constexpr (MODE != ckl::MODE_FWDZ) {
     if (cudaFuncSetAttribute(ckl::tc_kernel<MODE, kPair, true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) !=
         cudaSuccess)
@@ -312,8 +308,7 @@ bool device_info(DevInfo& out) {
   }
   if (!di.attrs_set && di.major == 10) {
     if (!setup_mode<ckl::MODE_FWD>(di) || !setup_mode<ckl::MODE_DZ>(di) ||
-        !setup_mode<ckl::MODE_DHDW>(di) || !setup_mode<ckl::MODE_FWDZ>(di) ||
-        !setup_mode<ckl::MODE_BWD>(di))
+        !setup_mode<ckl::MODE_DHDW>(di) || !setup_mode<ckl::MODE_FWDZ>(di))
       return false;
     di.attrs_set = true;
   }
@@ -474,13 +469,16 @@ int transpose_rows(const void* H, int64_t d, int64_t r0, int64_t rows, uint8_t* 
 // (v_lo a multiple of 256), recomputed from H and W, into panels
 // [ceil(cols/PW)][prow][PW] at the start of the dZ buffer (PW = 64 bf16 or
 // 32 fp32 columns: 128 bytes).
-// The logit-tile fields of p and its maps tm[zb .. zb + 2] (H rows, W, dZ).
 template <bool F32>
-bool fill_dz(TcParams& p, int zb, const void* H, const void* W, const float* lse, int64_t d,
-             int64_t V, int64_t r0, int64_t rows, int64_t prow, int64_t v_lo, int64_t cols,
-             uint8_t* w8, const Layout& L, int64_t v_off) {
+int dz_block(const void* H, const void* W, const uint8_t* mask, const float* lse, int64_t T,
+             int64_t d, int64_t V, int32_t K, int64_t r0, int64_t rows, int64_t prow,
+             int64_t v_lo, int64_t cols, uint8_t* w8, const Layout& L, const DevInfo& di,
+             cudaStream_t st, ckl_trace* trace, int64_t v_off = 0) {
   constexpr int eb = F32 ? 4 : 2;
   constexpr uint32_t PW = kKE<F32>;
+  TcParams p;
+  std::memset(&p, 0, sizeof(p));
+  fill_common(p, w8, L, T, d, V, K, mask);
   p.rows = static_cast<int32_t>(rows);
   p.row0 = static_cast<int32_t>(r0);
   p.n_rb = static_cast<int32_t>(cdiv(rows, kMB));
@@ -491,23 +489,12 @@ bool fill_dz(TcParams& p, int zb, const void* H, const void* W, const float* lse
   p.lse = lse;
   p.v_off = static_cast<int32_t>(v_off);
   const uint8_t* Hr = static_cast<const uint8_t*>(H) + r0 * d * eb;
-  return map2d(&p.tm[zb], kDT<F32>, Hr, d, rows, d * eb, kKE<F32>, ckl::BM,
-               CU_TENSOR_MAP_SWIZZLE_128B) &&
-         map2d(&p.tm[zb + 1], kDT<F32>, W, d, V, d * eb, kKE<F32>, ckl::BN_V / kSlotCTAs,
-               CU_TENSOR_MAP_SWIZZLE_128B) &&
-         map3d(&p.tm[zb + 2], kDT<F32>, w8 + L.dz, PW, rows, cdiv(cols, PW), 128, prow * 128, 32,
-               ckl::BM, F32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
-}
-
-template <bool F32>
-int dz_block(const void* H, const void* W, const uint8_t* mask, const float* lse, int64_t T,
-             int64_t d, int64_t V, int32_t K, int64_t r0, int64_t rows, int64_t prow,
-             int64_t v_lo, int64_t cols, uint8_t* w8, const Layout& L, const DevInfo& di,
-             cudaStream_t st, ckl_trace* trace, int64_t v_off = 0) {
-  TcParams p;
-  std::memset(&p, 0, sizeof(p));
-  fill_common(p, w8, L, T, d, V, K, mask);
-  if (!fill_dz<F32>(p, 0, H, W, lse, d, V, r0, rows, prow, v_lo, cols, w8, L, v_off))
+  if (!map2d(&p.tm[0], kDT<F32>, Hr, d, rows, d * eb, kKE<F32>, ckl::BM,
+             CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map2d(&p.tm[1], kDT<F32>, W, d, V, d * eb, kKE<F32>, ckl::BN_V / kSlotCTAs,
+             CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map3d(&p.tm[2], kDT<F32>, w8 + L.dz, PW, rows, cdiv(cols, PW), 128, prow * 128, 32,
+             ckl::BM, F32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
     return CKL_ERR_CUDA;
   TraceScope ts(trace, st, CKL_KERNEL_BWD_DZ);
   return launch_tc<ckl::MODE_DZ, F32>(p, p.n_units, di, st);
@@ -563,17 +550,19 @@ void dw_round_quotas(TcParams& p, int64_t G) {
 // 1 stores and 2 adds the block's fp32 share into dh_out (the partial dH of
 // a sliced row chunk, or the fp32 entry points' dH rows).  dw_store 1 stores
 // the block's dW rows, 0 adds.
-// The dH / dW fields of p and its maps tm[0 .. 5], dealt over G slots.
 template <bool F32>
-bool fill_dhdw(TcParams& p, const void* W, int64_t d, int64_t V, int64_t r0, int64_t rows,
-               int64_t prow, int64_t v_lo, int64_t cols, int dh_mode, int dw_store,
-               const float* grad_loss, void* dh_out, float* dW, uint8_t* w8, const Layout& L,
-               int64_t G) {
+int dhdw_block(const void* W, const uint8_t* mask, int64_t T, int64_t d, int64_t V, int32_t K,
+               int64_t r0, int64_t rows, int64_t prow, int64_t v_lo, int64_t cols, int dh_mode,
+               int dw_store, const float* grad_loss, void* dh_out, float* dW, uint8_t* w8,
+               const Layout& L, const DevInfo& di, cudaStream_t st, ckl_trace* trace) {
   constexpr int eb = F32 ? 4 : 2;
   constexpr uint32_t KE = kKE<F32>;  // also the panel width
   void* dz = w8 + L.dz;
   const int bn = pick_bn(d);
   const int64_t npan = cdiv(cols, KE);
+  TcParams p;
+  std::memset(&p, 0, sizeof(p));
+  fill_common(p, w8, L, T, d, V, K, mask);
   p.rows = static_cast<int32_t>(rows);
   p.row0 = static_cast<int32_t>(r0);
   p.bn = bn;
@@ -589,6 +578,7 @@ bool fill_dhdw(TcParams& p, const void* W, int64_t d, int64_t V, int64_t r0, int
   p.grad_loss = grad_loss;
   // dW tiles: contiguous per slot while every slot's dZ panels (kMB x rows
   // per vocabulary block) fit in L2 together, else dealt in rounds
+  const int64_t G = std::min<int64_t>(di.slots[ckl::MODE_DHDW], p.n5 + p.n6);
   p.dw_mode = (kMB * rows * eb * G > (int64_t(48) << 20)) ? 1 : 0;
   if (p.dw_mode == 1) dw_round_quotas(p, G);
   const bool dh_low = (dh_mode == 0);  // bf16 dH
@@ -603,143 +593,21 @@ bool fill_dhdw(TcParams& p, const void* W, int64_t d, int64_t V, int64_t r0, int
            map3d2(&p.tm[1], kDT<F32>, W, KE, V, d / KE, d * eb, KE * eb, KE, KE,
                   static_cast<uint32_t>(bn / kSlotCTAs / KE), mn_sw))
               ? 1 : 0;
-  if (!p.w3d && !map2d(&p.tm[1], kDT<F32>, W, d, V, d * eb, KE, KE, mn_sw)) return false;
-  return map3d(&p.tm[0], kDT<F32>, dz, KE, rows, npan, 128, prow * 128, KE, ckl::BM,
-             CU_TENSOR_MAP_SWIZZLE_128B) &&
-         map3d2(&p.tm[2], kDT<F32>, dz, KE, rows, npan, 128, prow * 128, KE, KE,
-              static_cast<uint32_t>(ckl::BM / KE), mn_sw) &&
-         map2d(&p.tm[3], kDT<F32>, w8 + L.hct, rows, d, L.pitch_t * eb, KE, bn / kSlotCTAs,
-             CU_TENSOR_MAP_SWIZZLE_128B) &&
-         map2d(&p.tm[4], dh_low ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+  if (!p.w3d && !map2d(&p.tm[1], kDT<F32>, W, d, V, d * eb, KE, KE, mn_sw)) return CKL_ERR_CUDA;
+  if (!map3d(&p.tm[0], kDT<F32>, dz, KE, rows, npan, 128, prow * 128, KE, ckl::BM,
+             CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map3d2(&p.tm[2], kDT<F32>, dz, KE, rows, npan, 128, prow * 128, KE, KE,
+              static_cast<uint32_t>(ckl::BM / KE), mn_sw) ||
+      !map2d(&p.tm[3], kDT<F32>, w8 + L.hct, rows, d, L.pitch_t * eb, KE, bn / kSlotCTAs,
+             CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map2d(&p.tm[4], dh_low ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
              dh_out, d, rows, d * (dh_low ? 2 : 4), 32, ckl::BM,
-             dh_low ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B) &&
-         map2d(&p.tm[5], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, dW, d, V, d * 4, 32, ckl::BM,
-             CU_TENSOR_MAP_SWIZZLE_128B);
-}
-
-template <bool F32>
-int dhdw_block(const void* W, const uint8_t* mask, int64_t T, int64_t d, int64_t V, int32_t K,
-               int64_t r0, int64_t rows, int64_t prow, int64_t v_lo, int64_t cols, int dh_mode,
-               int dw_store, const float* grad_loss, void* dh_out, float* dW, uint8_t* w8,
-               const Layout& L, const DevInfo& di, cudaStream_t st, ckl_trace* trace) {
-  TcParams p;
-  std::memset(&p, 0, sizeof(p));
-  fill_common(p, w8, L, T, d, V, K, mask);
-  const int bn = pick_bn(d);
-  const int64_t n_nt = cdiv(d, bn);
-  const int64_t units = cdiv(rows, kMB) * n_nt + cdiv(cols, kMB) * n_nt;
-  const int64_t G = std::min<int64_t>(di.slots[ckl::MODE_DHDW], units);
-  if (!fill_dhdw<F32>(p, W, d, V, r0, rows, prow, v_lo, cols, dh_mode, dw_store, grad_loss,
-                      dh_out, dW, w8, L, G))
+             dh_low ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map2d(&p.tm[5], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, dW, d, V, d * 4, 32, ckl::BM,
+             CU_TENSOR_MAP_SWIZZLE_128B))
     return CKL_ERR_CUDA;
   TraceScope ts(trace, st, CKL_KERNEL_BWD_DHDW);
   return launch_tc<ckl::MODE_DHDW, F32>(p, p.n5 + p.n6, di, st);
-}
-
-// k-blocks (with one more per tile for its epilogue) that the dH / dW part of
-// a launch deals to slot j of G: its round-robin dH units, then its dW tiles
-// (a contiguous range, or its share of the rounds), as JobIter deals them.
-int64_t dhdw_slot_load(const TcParams& p, int64_t G, int64_t j) {
-  const int64_t cnt5 = (p.n5 > j) ? (p.n5 - j + G - 1) / G : 0;
-  int64_t q6 = 0;
-  if (p.dw_mode == 0) {
-    const int64_t c6e = p.c6 + 1;
-    const int64_t total = static_cast<int64_t>(p.n5) * p.c5 + static_cast<int64_t>(p.n6) * c6e;
-    const int64_t target = (total + G - 1) / G;
-    int64_t P = 0, Pc = 0, mine = 0;
-    for (int64_t i = 0; i < G; ++i) {
-      const int64_t c5i = (p.n5 > i) ? (p.n5 - i + G - 1) / G : 0;
-      const int64_t cap = std::max<int64_t>(target - c5i * p.c5, 0);
-      if (i < j) Pc += cap;
-      if (i == j) mine = cap;
-      P += cap;
-    }
-    const int64_t b = (P == 0) ? p.n6 * j / G : p.n6 * Pc / P;
-    const int64_t e = (P == 0) ? p.n6 * (j + 1) / G : p.n6 * (Pc + mine) / P;
-    q6 = e - b;
-  } else {
-    const int64_t r5 = p.n5 % G;
-    q6 = (j < r5) ? p.dw_Qh - 1 + (j < p.dw_Eh ? 1 : 0) : p.dw_Ql - 1 + (j - r5 < p.dw_El ? 1 : 0);
-    q6 = std::max<int64_t>(q6, 0);
-  }
-  return cnt5 * p.c5 + q6 * (p.c6 + 1);
-}
-
-// The next block's dZ tiles per slot (p.zq), cost cz each, filling the slots'
-// dH / dW loads up to an even finish (water-filling, the excess taken from
-// the slots that would finish last).  False when a slot would hold more than
-// the kernel's list does.
-bool dz_quotas(TcParams& p, int64_t G, int64_t nz, int64_t cz) {
-  if (G > ckl::ZQ_SLOTS) return false;
-  int64_t load[ckl::ZQ_SLOTS];
-  int64_t hi = 0;
-  for (int64_t j = 0; j < G; ++j) {
-    load[j] = dhdw_slot_load(p, G, j);
-    hi = std::max(hi, load[j]);
-  }
-  auto fill = [&](int64_t t) {
-    int64_t n = 0;
-    for (int64_t j = 0; j < G; ++j) n += (t > load[j]) ? (t - load[j]) / cz : 0;
-    return n;
-  };
-  int64_t lo = 0, top = hi + (nz + 1) * cz;
-  while (lo < top) {
-    const int64_t mid = (lo + top) / 2;
-    if (fill(mid) >= nz) top = mid;
-    else lo = mid + 1;
-  }
-  int64_t q[ckl::ZQ_SLOTS];
-  int64_t excess = -nz;
-  for (int64_t j = 0; j < G; ++j) {
-    q[j] = (lo > load[j]) ? (lo - load[j]) / cz : 0;
-    excess += q[j];
-  }
-  while (excess > 0) {  // one tile less for the slot that would finish last
-    int64_t w = -1;
-    for (int64_t j = 0; j < G; ++j)
-      if (q[j] > 0 && (w < 0 || load[j] + q[j] * cz >= load[w] + q[w] * cz)) w = j;
-    --q[w];
-    --excess;
-  }
-  for (int64_t j = 0; j < ckl::ZQ_SLOTS; ++j) {
-    const int64_t v = (j < G) ? q[j] : 0;
-    if (v > ckl::ZLIST_MAX) return false;
-    p.zq[j] = static_cast<uint16_t>(v);
-  }
-  return true;
-}
-
-// One launch for the dH / dW of block b and the dZ tiles of the next block
-// (rows [r0n, r0n + rowsn) x columns [v_lon, v_lon + colsn)), which replace
-// block b's dZ in the buffer as its readers finish (MODE_BWD).  *done =
-// false, with nothing enqueued, when the tiles cannot be dealt to the slots;
-// the caller then launches the two separately.
-int bwd_fused_block(const void* H, const void* W, const uint8_t* mask, const float* lse,
-                    int64_t T, int64_t d, int64_t V, int32_t K, int64_t r0, int64_t rows,
-                    int64_t prow, int64_t v_lo, int64_t cols, int dh_mode, int dw_store,
-                    const float* grad_loss, void* dh_out, float* dW, int64_t r0n, int64_t rowsn,
-                    int64_t v_lon, int64_t colsn, int64_t v_off, uint8_t* w8, const Layout& L,
-                    const DevInfo& di, cudaStream_t st, ckl_trace* trace, bool* done) {
-  *done = false;
-  TcParams p;
-  std::memset(&p, 0, sizeof(p));
-  fill_common(p, w8, L, T, d, V, K, mask);
-  const int bn = pick_bn(d);
-  const int64_t n_nt = cdiv(d, bn);
-  const int64_t nz = cdiv(rowsn, kMB) * cdiv(colsn, ckl::BN_V);
-  const int64_t units = cdiv(rows, kMB) * n_nt + cdiv(cols, kMB) * n_nt + nz;
-  const int64_t G = std::min<int64_t>(di.slots[ckl::MODE_BWD], units);
-  if (!fill_dhdw<false>(p, W, d, V, r0, rows, prow, v_lo, cols, dh_mode, dw_store, grad_loss,
-                        dh_out, dW, w8, L, G) ||
-      !fill_dz<false>(p, 6, H, W, lse, d, V, r0n, rowsn, prow, v_lon, colsn, w8, L, v_off))
-    return CKL_ERR_CUDA;
-  if (!dz_quotas(p, G, nz, cdiv(d, ckl::BK) + 1)) return CKL_OK;
-  p.dep = reinterpret_cast<int*>(w8 + L.dep);
-  if (cudaMemsetAsync(p.dep, 0, static_cast<size_t>(p.n_mt + 1) * sizeof(int), st) != cudaSuccess)
-    return CKL_ERR_CUDA;
-  *done = true;
-  TraceScope ts(trace, st, CKL_KERNEL_BWD_FUSED);
-  return launch_tc<ckl::MODE_BWD>(p, units, di, st);
 }
 
 // S2-S4 once the prep has run: the logit GEMM with its online log-sum-exp and
@@ -832,63 +700,36 @@ int backward_impl(const void* H, const void* W, const int32_t* topk_idx, const f
   uint8_t* w8 = static_cast<uint8_t*>(workspace);
   const Plan P = plan_backward(T, d, V, L);
   float* dh32 = reinterpret_cast<float*>(w8 + L.dh32);
-  // The blocks in order: row chunks of P.Cr rows, each swept in P.n slabs.
-  // Block b's dZ is computed before its dH / dW; with bf16 operands the next
-  // block's dZ tiles run in the same launch as block b's dH / dW (MODE_BWD),
-  // each written once the tiles of block b that read its place are done, so
-  // the launch ends on short tiles instead of waiting for its last dW tiles.
-  const int64_t n_rc = cdiv(T, P.Cr);
-  const int64_t nb = n_rc * P.n;
-  auto blk = [&](int64_t b, int64_t& r0, int64_t& rows, int64_t& v_lo, int64_t& cols) {
-    r0 = (b / P.n) * P.Cr;
-    rows = std::min(P.Cr, T - r0);
-    v_lo = (b % P.n) * P.Sv;
-    cols = std::min(P.Sv, V - v_lo);
-  };
-  bool have_dz = false;  // the dZ of block b is already in the buffer
-  for (int64_t b = 0; b < nb; ++b) {
-    int64_t r0, rows, v_lo, cols;
-    blk(b, r0, rows, v_lo, cols);
-    const int64_t s = b % P.n;
-    if (s == 0) {
-      rc = transpose_rows<F32>(H, d, r0, rows, w8, L, st, trace);
-      if (rc != CKL_OK) return rc;
-    }
-    if (!have_dz) {
+  for (int64_t r0 = 0; r0 < T; r0 += P.Cr) {
+    const int64_t rows = std::min(P.Cr, T - r0);
+    rc = transpose_rows<F32>(H, d, r0, rows, w8, L, st, trace);
+    if (rc != CKL_OK) return rc;
+    const int dw_store = (r0 == 0 && !accumulate_dW) ? 1 : 0;
+    for (int64_t s = 0; s < P.n; ++s) {
+      const int64_t v_lo = s * P.Sv;
+      const int64_t cols = std::min(P.Sv, V - v_lo);
       rc = dz_block<F32>(H, W, mask, lse, T, d, V, K, r0, rows, P.Cr, v_lo, cols, w8, L, di,
                          st, trace, v_off);
       if (rc != CKL_OK) return rc;
-    }
-    const int dw_store = (r0 == 0 && !accumulate_dW) ? 1 : 0;
-    // bf16 dH: one slab writes it, several sum into the fp32 partial first;
-    // fp32 dH: the slabs store / add into the output itself
-    int dh_mode;
-    void* dh_out;
-    if (dh_f32) {
-      dh_mode = (s == 0) ? 1 : 2;
-      dh_out = static_cast<uint8_t*>(dH) + r0 * d * 4;
-    } else {
-      dh_mode = (P.n == 1) ? 0 : (s == 0 ? 1 : 2);
-      dh_out = (P.n == 1) ? static_cast<void*>(static_cast<uint8_t*>(dH) + r0 * d * 2)
-                          : static_cast<void*>(dh32);
-    }
-    have_dz = false;
-    if (!F32 && b + 1 < nb) {
-      int64_t r0n, rowsn, v_lon, colsn;
-      blk(b + 1, r0n, rowsn, v_lon, colsn);
-      rc = bwd_fused_block(H, W, mask, lse, T, d, V, K, r0, rows, P.Cr, v_lo, cols, dh_mode,
-                           dw_store, grad_loss, dh_out, dW, r0n, rowsn, v_lon, colsn, v_off, w8,
-                           L, di, st, trace, &have_dz);
-      if (rc != CKL_OK) return rc;
-    }
-    if (!have_dz) {
+      // bf16 dH: one slab writes it, several sum into the fp32 partial first;
+      // fp32 dH: the slabs store / add into the output itself
+      int dh_mode;
+      void* dh_out;
+      if (dh_f32) {
+        dh_mode = (s == 0) ? 1 : 2;
+        dh_out = static_cast<uint8_t*>(dH) + r0 * d * 4;
+      } else {
+        dh_mode = (P.n == 1) ? 0 : (s == 0 ? 1 : 2);
+        dh_out = (P.n == 1) ? static_cast<void*>(static_cast<uint8_t*>(dH) + r0 * d * 2)
+                            : static_cast<void*>(dh32);
+      }
       rc = dhdw_block<F32>(W, mask, T, d, V, K, r0, rows, P.Cr, v_lo, cols, dh_mode, dw_store,
                            grad_loss, dh_out, dW, w8, L, di, st, trace);
       if (rc != CKL_OK) return rc;
+      // the last row chunk's launch is the last to write these dW rows
+      if (on_dw_ready && r0 + rows == T) on_dw_ready(v_lo, v_lo + cols, user);
     }
-    // the last row chunk's launch is the last to write these dW rows
-    if (on_dw_ready && r0 + rows == T) on_dw_ready(v_lo, v_lo + cols, user);
-    if (s == P.n - 1 && !dh_f32 && P.n > 1) {
+    if (!dh_f32 && P.n > 1) {
       // dH rows of this chunk: the fp32 sum over its slabs, rounded once
       TraceScope ts(trace, st, CKL_KERNEL_OTHER);
       const int64_t n4 = rows * d / 4;

@@ -46,13 +46,7 @@ constexpr uint32_t ACC_COLS = 256;          // TMEM columns per accumulator buff
 // FWD: logits + online log-sum-exp + teacher gather; DZ: logit recompute +
 // dZ; DHDW: dH and dW of one chunk; FWDZ: FWD over one chunk that also
 // stores the fp32 logits (the single-pass schedule).
-// BWD: DHDW of one backward block followed, in the same launch, by the DZ
-// tiles of the next block, each written once the tiles of this block that
-// read its place in the dZ buffer are done.
-enum Mode { MODE_FWD = 0, MODE_DZ = 1, MODE_DHDW = 2, MODE_FWDZ = 3, MODE_BWD = 4 };
-
-constexpr int ZQ_SLOTS = 128;    // BWD: scheduling slots a launch may have
-constexpr int ZLIST_MAX = 128;   // BWD: dZ tiles one slot may take
+enum Mode { MODE_FWD = 0, MODE_DZ = 1, MODE_DHDW = 2, MODE_FWDZ = 3 };
 
 // Pipeline depth and epilogue width.  A single CTA holds a 128 x 256 tile:
 // four 48 KB operand stages fill the shared memory beside the epilogue
@@ -72,8 +66,7 @@ struct Cfg {
   static constexpr int B_OFF = STAGES * A_BYTES;
   static constexpr int EPI_OFF = B_OFF + STAGES * B_STAGE;
   static constexpr int BAR_OFF = EPI_OFF + 2 * EPI_STAGE;  // two staging tiles
-  static constexpr int ZLIST_OFF = BAR_OFF + 256;           // BWD: this slot's dZ tiles
-  static constexpr int SMEM_ALLOC = ZLIST_OFF + 4 * ZLIST_MAX + 1024;  // + slack to align to 1 KB
+  static constexpr int SMEM_ALLOC = BAR_OFF + 256 + 1024;  // + slack to align the base to 1 KB
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
   static_assert(8 * (2 * STAGES + 9) + 4 <= 256, "barrier area");
 };
@@ -82,7 +75,7 @@ constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 
 struct alignas(64) TcParams {
-  CUtensorMap tm[9];  // BWD: 0-5 as DHDW, 6-8 as DZ's 0-2 (the next block's H rows, W, dZ)
+  CUtensorMap tm[6];
   int32_t T, d, V, K;
   int32_t rows;     // FWD: T; DZ / DHDW: rows of this chunk
   int32_t row0;     // DZ / DHDW: first row of this chunk
@@ -111,10 +104,6 @@ struct alignas(64) TcParams {
   const float* grad_loss; // DHDW: [1] or null (= 1)
   int* status;            // device status word
   const int* countN;      // N = number of positions that count
-  // BWD: [0] dH units whose dZ reads are done, [1 + vb] dW tiles of vocabulary
-  // block vb whose dZ reads are done (zeroed before the launch)
-  int* dep;
-  uint16_t zq[ZQ_SLOTS];  // BWD: dZ tiles of each slot (the DZ part's units, dealt in rounds)
 };
 
 // ------------------------------------------------------------------ prep
@@ -517,14 +506,10 @@ struct JobIter {
   // Round quotas come in two classes: the r5 = n5 mod G slots with one more
   // dH unit hold Qh tiles (the first Eh of them) or Qh - 1, the others Ql
   // (the first El of them) or Ql - 1; the tile index is then closed-form.
-  // BWD: the DHDW phases, then (phase 2) this slot's dZ tiles of the next
-  // block, zlist[0 .. q7) (tile lin = vt n_rb + rb, as in DZ), then done (3).
   int u, vt, vt_hi;
   int lin;
-  int phase;  // DHDW: 0 = dH units, 1 = dW tiles, 2 = done; BWD: 2 = dZ tiles, 3 = done
+  int phase;  // DHDW: 0 = dH units, 1 = dW tiles, 2 = done
   int k6, e6;
-  int k7, q7;
-  const int* zlist;
   // tiles of a class (n slots, quota Q for the first E, Q - 1 for the rest)
   // dealt in rounds before round k, and those of its first m slots in round k
   __device__ static int cls_before(int k, int n, int Q, int E) {
@@ -535,26 +520,10 @@ struct JobIter {
     if (Q < 1 || k > Q - 1) return 0;
     return (k < Q - 1) ? m : (m < E ? m : E);
   }
-  // BWD: the k7-th dZ tile of this slot
-  __device__ void dz_set(const TcParams& p) {
-    lin = zlist[k7];
-    u = lin % p.n_rb;
-    vt = lin / p.n_rb;
-    vt_hi = vt + 1;
-  }
-  // DHDW: after the last dW tile; BWD: on to the dZ tiles
-  __device__ void dw_done(const TcParams& p) {
-    if (mode != MODE_BWD) { phase = 2; return; }
-    phase = 2;
-    k7 = 0;
-    q7 = p.zq[cta];
-    if (q7 == 0) phase = 3;
-    else dz_set(p);
-  }
-  // DHDW: the next dW tile of this slot (k6 counts them), or the end of them
+  // DHDW: the next dW tile of this slot (k6 counts them), or phase 2
   __device__ void dw_pick(const TcParams& p) {
     if (p.dw_mode == 0) {
-      if (k6 >= e6) { dw_done(p); return; }
+      if (k6 >= e6) { phase = 2; return; }
       u = k6;
       return;
     }
@@ -563,7 +532,7 @@ struct JobIter {
     const bool heavy = cta < r5;
     const int q = heavy ? p.dw_Qh - 1 + (cta < p.dw_Eh ? 1 : 0)
                         : p.dw_Ql - 1 + (cta - r5 < p.dw_El ? 1 : 0);
-    if (k6 >= q) { dw_done(p); return; }
+    if (k6 >= q) { phase = 2; return; }
     u = cls_before(k6, r5, p.dw_Qh, p.dw_Eh) + cls_before(k6, nl, p.dw_Ql, p.dw_El) +
         cls_rank(k6, cta < r5 ? cta : r5, p.dw_Qh, p.dw_Eh) +
         (cta > r5 ? cls_rank(k6, cta - r5, p.dw_Ql, p.dw_El) : 0);
@@ -574,7 +543,7 @@ struct JobIter {
   // fastest: the units in flight hold about G / S row blocks and S W tiles.
   // (DZ: u is the row block itself.)
   __device__ int unit_rb(const TcParams& p, int unit) const {
-    return (mode != MODE_DZ && mode != MODE_BWD && p.split_fast) ? unit / p.S : unit % p.n_rb;
+    return (mode != MODE_DZ && p.split_fast) ? unit / p.S : unit % p.n_rb;
   }
   __device__ int unit_s(const TcParams& p, int unit) const {
     return p.split_fast ? unit % p.S : unit / p.n_rb;
@@ -584,17 +553,16 @@ struct JobIter {
     lo = static_cast<int>(static_cast<int64_t>(s) * p.n_vt / p.S);
     hi = static_cast<int>(static_cast<int64_t>(s + 1) * p.n_vt / p.S);
   }
-  __device__ void init(const TcParams& p, int mode_, int per_slot, const int* zlist_ = nullptr) {
+  __device__ void init(const TcParams& p, int mode_, int per_slot) {
     mode = mode_;
     G = gridDim.x / per_slot;
     cta = blockIdx.x / per_slot;
-    zlist = zlist_;
     if (mode == MODE_DZ) {
       lin = cta;
       u = lin % p.n_rb;
       vt = lin / p.n_rb;
       vt_hi = vt + 1;
-    } else if (mode != MODE_DHDW && mode != MODE_BWD) {
+    } else if (mode != MODE_DHDW) {
       u = cta;
       vt = vt_hi = 0;
       if (u < p.n_units) vt_range(p, u, vt, vt_hi);
@@ -609,9 +577,7 @@ struct JobIter {
   }
   __device__ bool valid(const TcParams& p) const {
     if (mode == MODE_DZ) return lin < p.n_units;
-    if (mode == MODE_DHDW) return phase < 2;
-    if (mode == MODE_BWD) return phase < 3;
-    return u < p.n_units;
+    return (mode != MODE_DHDW) ? (u < p.n_units) : (phase < 2);
   }
   __device__ void next(const TcParams& p) {
     if (mode == MODE_DZ) {
@@ -619,7 +585,7 @@ struct JobIter {
       u = lin % p.n_rb;
       vt = lin / p.n_rb;
       vt_hi = vt + 1;
-    } else if (mode != MODE_DHDW && mode != MODE_BWD) {
+    } else if (mode != MODE_DHDW) {
       if (++vt >= vt_hi) {
         u += G;
         if (u < p.n_units) vt_range(p, u, vt, vt_hi);
@@ -630,12 +596,9 @@ struct JobIter {
         phase = 1;
         dw_start(p);
       }
-    } else if (phase == 1) {
+    } else {
       ++k6;
       dw_pick(p);
-    } else {
-      if (++k7 >= q7) phase = 3;
-      else dz_set(p);
     }
   }
   __device__ void dw_start(const TcParams& p) {
@@ -649,7 +612,7 @@ struct JobIter {
   // FWD / DZ: is this the first / last tile of its unit?  (DZ: every tile
   // starts its row state afresh.)
   __device__ bool first_of_unit(const TcParams& p) const {
-    if (mode == MODE_DZ || mode == MODE_BWD) return true;
+    if (mode == MODE_DZ) return true;
     int lo, hi;
     vt_range(p, u, lo, hi);
     return vt == lo;
@@ -697,7 +660,7 @@ tc_kernel(const __grid_constant__ TcParams p) {
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::BAR_OFF + 8 * (2 * STAGES + 9));
 
   if (warp == 0 && lane == 0) {
-    const int n_maps = (MODE == MODE_FWD) ? 2 : (MODE == MODE_DHDW) ? 6 : (MODE == MODE_BWD) ? 9 : 3;
+    const int n_maps = (MODE == MODE_FWD) ? 2 : (MODE == MODE_DHDW) ? 6 : 3;
 #pragma unroll 1
     for (int i = 0; i < n_maps; ++i) prefetch_tmap(&p.tm[i]);
     for (int s = 0; s < STAGES; ++s) {
@@ -724,24 +687,6 @@ tc_kernel(const __grid_constant__ TcParams p) {
       tmem_relinquish();
     }
   }
-  // BWD: this slot's dZ tiles of the next block, dealt in rounds: in round k
-  // every slot whose count exceeds k takes the next tile, so the k-th tile of
-  // slot j is  sum_i min(zq_i, k) + #{i < j : zq_i > k}.  Both CTAs of a pair
-  // compute the same list.
-  int* zlist = reinterpret_cast<int*>(gbase + C::ZLIST_OFF);
-  if (MODE == MODE_BWD && warp == 1) {
-    const int G = gridDim.x / (PAIR ? 2 : 1);
-    const int j = blockIdx.x / (PAIR ? 2 : 1);
-    const int qj = p.zq[j];
-    for (int k = lane; k < qj; k += 32) {
-      int idx = 0;
-      for (int i = 0; i < G; ++i) {
-        const int qi = p.zq[i];
-        idx += min(qi, k) + ((i < j && qi > k) ? 1 : 0);
-      }
-      zlist[k] = idx;
-    }
-  }
   tc_fence_before();
   __syncthreads();
   if (PAIR) cluster_sync();  // the peer may signal the leader's barriers from here on
@@ -756,15 +701,12 @@ tc_kernel(const __grid_constant__ TcParams p) {
       uint32_t issued = 0;
       bool ok = true;
       JobIter it;
-      it.init(p, MODE, PAIR ? 2 : 1, zlist);
+      it.init(p, MODE, PAIR ? 2 : 1);
       for (; ok && it.valid(p); it.next(p)) {
         int nkb;
         int a_x = 0, a_y = 0, b_x = 0, b_y = 0, kind = 0;
         const int half_n = PAIR ? p.bn / 2 : p.bn;  // B rows / columns this CTA stages
-        // a logit tile (FWD, DZ, FWDZ, and BWD's dZ tiles) or a dH / dW job
-        const bool zj = (MODE == MODE_BWD) ? (it.phase == 2) : (MODE != MODE_DHDW);
-        const int zb = (MODE == MODE_BWD) ? 6 : 0;  // tensor maps of the logit tiles
-        if (zj) {
+        if (MODE != MODE_DHDW) {
           const int rb = it.unit_rb(p, it.u);
           nkb = (p.d + KE - 1) / KE;
           a_y = rb * MB + static_cast<int>(rank) * BM;
@@ -780,7 +722,7 @@ tc_kernel(const __grid_constant__ TcParams p) {
           a_x = (it.u / p.n_nt) * MB + static_cast<int>(rank) * BM;      // vocabulary rows
           b_x = (it.u % p.n_nt) * p.bn + static_cast<int>(rank) * half_n;
         }
-        const uint32_t bytes = zj ? A_BYTES + B_STAGE : A_BYTES + half_n * 128;
+        const uint32_t bytes = (MODE != MODE_DHDW) ? A_BYTES + B_STAGE : A_BYTES + half_n * 128;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, p.status)) { ok = false; break; }
           uint32_t fb = bar_full + 8 * stage;
@@ -794,13 +736,13 @@ tc_kernel(const __grid_constant__ TcParams p) {
           }
           const uint32_t sa = sbase + C::A_OFF + stage * A_BYTES;
           const uint32_t sb = sbase + C::B_OFF + stage * B_STAGE;
-          if (zj) {
+          if (MODE != MODE_DHDW) {
             if (PAIR) {
-              tma_load_2d_pair(sa, &p.tm[zb], fb, kb * KE, a_y);
-              tma_load_2d_pair(sb, &p.tm[zb + 1], fb, kb * KE, b_y);
+              tma_load_2d_pair(sa, &p.tm[0], fb, kb * KE, a_y);
+              tma_load_2d_pair(sb, &p.tm[1], fb, kb * KE, b_y);
             } else {
-              tma_load_2d(sa, &p.tm[zb], fb, kb * KE, a_y);
-              tma_load_2d(sb, &p.tm[zb + 1], fb, kb * KE, b_y);
+              tma_load_2d(sa, &p.tm[0], fb, kb * KE, a_y);
+              tma_load_2d(sb, &p.tm[1], fb, kb * KE, b_y);
             }
           } else if (kind == 5) {
             // dZ is stored as 64-column panels: k-block kb is panel kb.  W is
@@ -859,14 +801,13 @@ tc_kernel(const __grid_constant__ TcParams p) {
       uint32_t acc_phase = 0;
       bool ok = true;
       JobIter it;
-      it.init(p, MODE, PAIR ? 2 : 1, zlist);
+      it.init(p, MODE, PAIR ? 2 : 1);
       for (; ok && it.valid(p); it.next(p)) {
         int nkb;
         uint32_t idesc;
         uint32_t a_step, b_step, a_lbo, b_lbo;
         bool a_mn = false, b_mn = false;
-        const bool zj = (MODE == MODE_BWD) ? (it.phase == 2) : (MODE != MODE_DHDW);
-        if (zj) {
+        if (MODE != MODE_DHDW) {
           nkb = (p.d + KE - 1) / KE;
           idesc = F32 ? idesc_tf32(MMA_M, BN_V, 0, 0) : idesc_bf16(MMA_M, BN_V, 0, 0);
           a_step = 32; b_step = 32; a_lbo = 16; b_lbo = 16;
@@ -895,10 +836,6 @@ tc_kernel(const __grid_constant__ TcParams p) {
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(bar_full + 8 * stage, phase, p.status)) { ok = false; break; }
           tc_fence_after();
-          // BWD: the last stage of a dH / dW job has landed, so the job has
-          // read all of its dZ: announce it to the next block's dZ tiles
-          if (MODE == MODE_BWD && !zj && kb == nkb - 1)
-            red_release_add(p.dep + (it.phase == 0 ? 0 : 1 + it.u / p.n_nt), 1);
           const uint64_t ads = ad0 + static_cast<uint64_t>((stage * A_BYTES) >> 4);
           const uint64_t bds = bd0 + static_cast<uint64_t>((stage * B_STAGE) >> 4);
 #pragma unroll
@@ -972,7 +909,7 @@ tc_kernel(const __grid_constant__ TcParams p) {
         good = mbar_wait(bar_staged + 8 * sb, static_cast<uint32_t>(nstore >> 1) & 1u, p.status);
         if (good) {
           const uint32_t buf = stage_base + sb * EPI_STAGE;
-          if (kind == 0) tma_store_3d(&p.tm[(MODE == MODE_BWD) ? 8 : 2], buf, x, y, z);
+          if (kind == 0) tma_store_3d(&p.tm[2], buf, x, y, z);
           else if (kind == 1) tma_store_2d(&p.tm[4], buf, x, y);
           else if (kind == 2) tma_store_2d(&p.tm[5], buf, x, y);
           else if (kind == 3) tma_reduce_add_2d(&p.tm[5], buf, x, y);
@@ -999,20 +936,16 @@ tc_kernel(const __grid_constant__ TcParams p) {
     float run_m = -INFINITY, run_s = 0.f, run_pz = 0.f;
     float lse2 = 0.f;
     float scale = 0.f;
-    if (MODE == MODE_DHDW || MODE == MODE_BWD) {
+    if (MODE == MODE_DHDW) {
       const int n = *p.countN;
       const float g = (p.grad_loss != nullptr) ? *p.grad_loss : 1.f;
       scale = (n > 0) ? g / static_cast<float>(n) : 0.f;
     }
 
     JobIter it;
-    it.init(p, MODE, PAIR ? 2 : 1, zlist);
+    it.init(p, MODE, PAIR ? 2 : 1);
     for (; ok && it.valid(p); it.next(p)) {
-      // a logit tile (FWD, DZ, FWDZ, BWD's dZ tiles) or a dH / dW job; dzj:
-      // a logit tile whose epilogue writes dZ
-      const bool zj = (MODE == MODE_BWD) ? (it.phase == 2) : (MODE != MODE_DHDW);
-      const bool dzj = (MODE == MODE_DZ) || (MODE == MODE_BWD && it.phase == 2);
-      if (zj && it.first_of_unit(p)) {
+      if (MODE != MODE_DHDW && it.first_of_unit(p)) {
         const int rb = it.unit_rb(p, it.u);
         const int r = rb * MB + row_in_tile;  // row within T (FWD) or the chunk (DZ)
         row_ok = r < p.rows;
@@ -1020,8 +953,8 @@ tc_kernel(const __grid_constant__ TcParams p) {
         counts = row_ok && (p.mask == nullptr || p.mask[t] != 0);
         run_m = -INFINITY; run_s = 0.f; run_pz = 0.f;
         nidx = INT_MAX;
-        if (dzj && row_ok) lse2 = p.lse[t] * LOG2E;
-        const bool want_ids = dzj ? counts : row_ok;
+        if (MODE == MODE_DZ && row_ok) lse2 = p.lse[t] * LOG2E;
+        const bool want_ids = (MODE == MODE_DZ) ? counts : row_ok;
         if (want_ids) {
           const int2* pr = p.pairs + t * p.K;
           const int v_lo = p.v_off + (p.vt0 + it.vt) * BN_V;
@@ -1083,23 +1016,11 @@ tc_kernel(const __grid_constant__ TcParams p) {
             else nidx = INT_MAX;
           }
         }
-      } else if (dzj) {
+      } else if (MODE == MODE_DZ) {
         const int rb = it.u % p.n_rb;
         const int y0 = rb * MB + row0_cta;  // first chunk row of this CTA's 128
         const int v_end = (p.V + 63) & ~63;  // dZ panels span round_up(V, 64) columns
-        if (MODE == MODE_BWD) {
-          // this tile's place in the dZ buffer is read by the launch's dH units
-          // (every one) and by its dW tiles of the same vocabulary block: the
-          // store waits until they have all read it
-          bool good = true;
-          if (issuer) {
-            good = wait_counter(p.dep, p.n5, p.status) &&
-                   (it.vt >= p.n_mt || wait_counter(p.dep + 1 + it.vt, p.n_nt, p.status));
-            fence_proxy_async_global();
-          }
-          if (ew == 0 && __shfl_sync(0xffffffffu, good ? 1 : 0, 0) == 0) ok = false;
-        }
-        for (int c = 0; ok && c < BN_V / 32; ++c) {
+        for (int c = 0; c < BN_V / 32; ++c) {
           const int v0 = (p.vt0 + it.vt) * BN_V + c * 32;
           if (v0 >= v_end) break;
           float x[32];

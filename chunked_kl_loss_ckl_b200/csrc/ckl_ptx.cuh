@@ -75,39 +75,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* st
   return mbar_wait_ns(bar, parity, status, CKL_WAIT_NS);
 }
 
-// ---------------------------------------------------------------- counters
-// Counters in global memory that order work across the CTAs of one launch:
-// the writer adds with release semantics once what it announces is done, the
-// reader acquires before acting on it (both at GPU scope).
-__device__ __forceinline__ void red_release_add(int* ptr, int v) {
-  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
-}
-__device__ __forceinline__ int ld_acquire(const int* ptr) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
-  return v;
-}
-// Orders this thread's earlier generic-proxy accesses to global memory (an
-// acquire above) before its later async-proxy ones (TMA stores).
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-// Bounded wait until *ptr >= target: false, with CKL_DEV_TIMEOUT recorded,
-// after CKL_WAIT_NS.
-__device__ __forceinline__ bool wait_counter(const int* ptr, int target, int* status) {
-  if (ld_acquire(ptr) >= target) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (ld_acquire(ptr) >= target) return true;
-    if (globaltimer_ns() - t0 > CKL_WAIT_NS) {
-      atomicOr(status, CKL_DEV_TIMEOUT);
-      return false;
-    }
-  }
-}
-
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");

@@ -59,7 +59,7 @@ __device__ __forceinline__ uint32_t bf16_key2(uint32_t w) {
 
 constexpr int TK_UNROLL = 2;  // independent 16-byte loads in flight per thread
 #ifndef CKL_TS_UNROLL
-#define CKL_TS_UNROLL 8
+#define CKL_TS_UNROLL 4
 #endif
 constexpr int TS_UNROLL = CKL_TS_UNROLL;  // the same, in the streaming form's pass
 
@@ -350,9 +350,12 @@ topk_cache_kernel(const uint16_t* __restrict__ logits, int64_t T, int V, int K, 
 // Blocks of TS_THREADS threads, TS_BLOCKS per SM: enough rows in flight to
 // keep HBM busy, few enough (TS_BLOCKS x SMs x 256 KB at V = 128 256) that
 // pass 2 finds its row still in L2; needs K <= TS_THREADS.
-constexpr int TS_THREADS = 256;
+#ifndef CKL_TS_THREADS
+#define CKL_TS_THREADS 256
+#endif
+constexpr int TS_THREADS = CKL_TS_THREADS;
 #ifndef CKL_TS_BLOCKS
-#define CKL_TS_BLOCKS 2
+#define CKL_TS_BLOCKS 4
 #endif
 constexpr int TS_BLOCKS = CKL_TS_BLOCKS;  // blocks per SM
 
@@ -369,42 +372,41 @@ struct TsShared {
 // by two 256-bucket rounds: high byte, then low byte.
 __device__ __forceinline__ uint32_t ts_kth_largest_key(TsShared& sm, uint32_t key, int K) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int NW = TS_THREADS / 32;
-  constexpr int PER = 256 / TS_THREADS > 0 ? 256 / TS_THREADS : 1;  // buckets per thread
-  static_assert(TS_THREADS * PER == 256, "one or more whole buckets per thread");
+  static_assert(TS_THREADS >= 256 && TS_THREADS % 256 == 0, "threads 0-255 own one bucket each");
   uint32_t prefix = 0, need = static_cast<uint32_t>(K);
+  bool few = false;  // fewer than K keys: every key counts
   for (int round = 0; round < 2; ++round) {
-    for (int j = tid; j < 256; j += TS_THREADS) sm.hist[j] = 0;
+    if (tid < 256) sm.hist[tid] = 0;
     __syncthreads();
-    if (round == 0 || (key >> 8) == prefix)
+    if (key != 0u && (round == 0 || (key >> 8) == prefix))
       atomicAdd(&sm.hist[(round == 0) ? (key >> 8) : (key & 0xFFu)], 1u);
     __syncthreads();
-    // thread tid owns buckets 255 - PER tid - j, j < PER (descending keys)
-    uint32_t own = 0;
+    // thread tid < 256 owns bucket 255 - tid (descending keys)
+    uint32_t own = 0, incl = 0;
+    if (tid < 256) {
+      own = sm.hist[255 - tid];
+      incl = own;
 #pragma unroll
-    for (int j = 0; j < PER; ++j) own += sm.hist[255 - (PER * tid + j)];
-    uint32_t incl = own;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    if (lane == 31) sm.s_part[warp] = incl;
-    __syncthreads();
-    uint32_t before = incl - own;
-    for (int w = 0; w < warp && w < NW; ++w) before += sm.s_part[w];
-    if (before < need && before + own >= need) {
-      uint32_t c = before;
-      for (int j = 0; j < PER; ++j) {
-        const uint32_t b = 255u - static_cast<uint32_t>(PER * tid + j);
-        const uint32_t h = sm.hist[b];
-        if (c + h >= need) {
-          sm.s_thr = (round == 0) ? b : ((prefix << 8) | b);
-          sm.s_total = c;  // keys above this bucket
-          break;
-        }
-        c += h;
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
       }
+      if (lane == 31) sm.s_part[warp] = incl;
+    }
+    __syncthreads();
+    uint32_t before = incl - own, total = 0;
+    for (int w = 0; w < 8; ++w) {
+      if (w < warp) before += sm.s_part[w];
+      total += sm.s_part[w];
+    }
+    if (round == 0 && total < need) {  // the same on every thread
+      few = true;
+      break;
+    }
+    if (tid < 256 && before < need && before + own >= need) {
+      const uint32_t b = 255u - static_cast<uint32_t>(tid);
+      sm.s_thr = (round == 0) ? b : ((prefix << 8) | b);
+      sm.s_total = before;  // keys above this bucket
     }
     __syncthreads();
     if (round == 0) {
@@ -413,7 +415,9 @@ __device__ __forceinline__ uint32_t ts_kth_largest_key(TsShared& sm, uint32_t ke
     }
     __syncthreads();
   }
-  return sm.s_thr;
+  const uint32_t r = few ? 0u : sm.s_thr;
+  __syncthreads();
+  return r;
 }
 
 __global__ void __launch_bounds__(TS_THREADS, TS_BLOCKS)

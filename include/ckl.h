@@ -82,8 +82,7 @@ enum {
   CKL_KERNEL_OTHER = 6,
   CKL_KERNEL_TOPK = 7,        /* teacher top-K cache producer */
   CKL_KERNEL_SP_GEMM = 8,     /* single pass: one chunk's logit GEMM, stores fp32 z too */
-  CKL_KERNEL_SP_ROWS = 9,     /* single pass: lse, loss terms and dZ from the stored z */
-  CKL_KERNEL_BWD_FUSED = 10   /* dH and dW of one block + the next block's dZ, one launch */
+  CKL_KERNEL_SP_ROWS = 9      /* single pass: lse, loss terms and dZ from the stored z */
 };
 
 /*

@@ -66,13 +66,13 @@ def test_cpu_description_names_the_host():
 
 
 def test_backward_flops_add_up_to_6dV_per_token():
-    # the per-kernel split of the backward (first block's dZ, fused dH/dW +
-    # next dZ launches, last block's dH/dW) covers 6 d V per token exactly
+    # the per-kernel split of the backward (each block's dZ recompute and its
+    # dH + dW) covers 6 d V per token exactly, whatever the blocking
     for T, d, V, plan in ((8192, 3072, 128256, (8192, 14336, 9)),
                           (262144, 4096, 128256, (6144, 64256, 2)),
                           (1000, 64, 3000, (256, 3008, 1))):
         f = bench.kernel_flops_per_step(T, d, V, plan)
-        back = f["bwd_dz"] + f["bwd_fused"] + f["bwd_dhdw"]
+        back = f["bwd_dz"] + f["bwd_dhdw"]
         assert abs(back - 6.0 * T * V * d) <= 1e-9 * back
         n = bench.backward_launches(T, V, plan)
-        assert n["bwd_fused"] == len(bench.backward_blocks(T, V, plan)) - 1
+        assert n["bwd_dz"] == n["bwd_dhdw"] == len(bench.backward_blocks(T, V, plan))
