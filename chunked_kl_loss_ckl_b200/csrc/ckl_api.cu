@@ -239,8 +239,15 @@ constexpr CUtensorMapDataType kDT =
 template <bool F32>
 constexpr uint32_t kKE = F32 ? 32 : 64;  // K (and panel) elements per 128-byte row
 
+// attr: room for 2.  The backward's GEMMs (DZ, DHDW) may start before the
+// launch ahead of them ends (programmatic stream serialisation; the kernel
+// waits where it depends on it).
+#ifndef CKL_PDL
+#define CKL_PDL 1
+#endif
 template <int MODE>
-cudaLaunchConfig_t tc_config(int slots, cudaStream_t st, cudaLaunchAttribute* attr) {
+cudaLaunchConfig_t tc_config(int slots, cudaStream_t st, cudaLaunchAttribute* attr,
+                             bool dependent = true) {
   using C = ckl::Cfg<MODE, kPair>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(slots * kSlotCTAs));
@@ -253,6 +260,11 @@ cudaLaunchConfig_t tc_config(int slots, cudaStream_t st, cudaLaunchAttribute* at
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (CKL_PDL && dependent && (MODE == ckl::MODE_DZ || MODE == ckl::MODE_DHDW)) {
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.numAttrs = 2;
+  }
   return cfg;
 }
 
@@ -270,8 +282,8 @@ bool setup_mode(DevInfo& di) {
         cudaSuccess)
       return false;
   }
-  cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = tc_config<MODE>(di.sms / kSlotCTAs, nullptr, attr);
+  cudaLaunchAttribute attr[2];
+  cudaLaunchConfig_t cfg = tc_config<MODE>(di.sms / kSlotCTAs, nullptr, attr, false);
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, ckl::tc_kernel<MODE, kPair>, &cfg) != cudaSuccess ||
       n <= 0) {
@@ -286,7 +298,7 @@ bool setup_mode(DevInfo& di) {
 template <int MODE, bool F32 = false>
 int launch_tc(const TcParams& p, int64_t units, const DevInfo& di, cudaStream_t st) {
   const int slots = static_cast<int>(std::min<int64_t>(di.slots[MODE], units));
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   cudaLaunchConfig_t cfg = tc_config<MODE>(slots, st, attr);
   return cudaLaunchKernelEx(&cfg, ckl::tc_kernel<MODE, kPair, F32>, p) == cudaSuccess
              ? CKL_OK

@@ -692,6 +692,15 @@ tc_kernel(const __grid_constant__ TcParams p) {
   if (PAIR) cluster_sync();  // the peer may signal the leader's barriers from here on
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+  // The backward's GEMMs are launched so that the next one may start while
+  // this one finishes (its CTAs take the SMs this one's CTAs leave): allow
+  // that now.  Whatever reads or writes memory that an earlier launch of the
+  // stream writes or reads waits below for that launch (griddep_wait), and
+  // only after that: the dH / dW producer before its first dZ load, every
+  // epilogue before its first global access.  The logit GEMMs' producers read
+  // H and W alone, so a recompute launch computes its first tiles while the
+  // dH / dW launch ahead of it drains.
+  griddep_launch();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -700,6 +709,7 @@ tc_kernel(const __grid_constant__ TcParams p) {
       uint32_t phase = 0;
       uint32_t issued = 0;
       bool ok = true;
+      if (MODE == MODE_DHDW) griddep_wait();  // dZ, H_c^T: written by the launches ahead
       JobIter it;
       it.init(p, MODE, PAIR ? 2 : 1);
       for (; ok && it.valid(p); it.next(p)) {
@@ -936,6 +946,7 @@ tc_kernel(const __grid_constant__ TcParams p) {
     float run_m = -INFINITY, run_s = 0.f, run_pz = 0.f;
     float lse2 = 0.f;
     float scale = 0.f;
+    griddep_wait();  // every epilogue reads or writes what earlier launches touch
     if (MODE == MODE_DHDW) {
       const int n = *p.countN;
       const float g = (p.grad_loss != nullptr) ? *p.grad_loss : 1.f;

@@ -75,6 +75,19 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* st
   return mbar_wait_ns(bar, parity, status, CKL_WAIT_NS);
 }
 
+// ---------------------------------------------------------------- dependent launches
+// A kernel launched with programmatic stream serialisation may start before
+// the kernel ahead of it in the stream has finished; griddep_wait() returns
+// once that kernel has completed and its writes are visible (at once for a
+// kernel launched without it).  griddep_launch() lets the next such kernel
+// start as soon as every CTA of this one has called it or exited.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
