@@ -420,10 +420,16 @@ int clear_and_prep(const int32_t* idx, const float* logp, const uint8_t* mask, i
   if (T > 0) {
     Header* hdr = reinterpret_cast<Header*>(w8);
     TraceScope ts(trace, st, CKL_KERNEL_PREP);
-    const unsigned grid = static_cast<unsigned>(cdiv(T, ckl::PREP_WARPS));
-    ckl::prep_kernel<<<grid, ckl::PREP_WARPS * 32, 0, st>>>(
-        idx, logp, mask, T, K, V, reinterpret_cast<int2*>(w8 + L.pairs),
-        reinterpret_cast<float*>(w8 + L.hp), &hdr->status, &hdr->countN);
+    if (K <= ckl::PREP_MAXK) {
+      const unsigned grid = static_cast<unsigned>(cdiv(T, ckl::PREP_WARPS));
+      ckl::prep_kernel<<<grid, ckl::PREP_WARPS * 32, 0, st>>>(
+          idx, logp, mask, T, K, V, reinterpret_cast<int2*>(w8 + L.pairs),
+          reinterpret_cast<float*>(w8 + L.hp), &hdr->status, &hdr->countN);
+    } else {
+      ckl::prep_large_kernel<<<static_cast<unsigned>(T), ckl::PREPL_THREADS, 0, st>>>(
+          idx, logp, mask, T, K, V, reinterpret_cast<int2*>(w8 + L.pairs),
+          reinterpret_cast<float*>(w8 + L.hp), &hdr->status, &hdr->countN);
+    }
     if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
   }
   return CKL_OK;
@@ -439,7 +445,7 @@ int common_prep(const void* H, const void* W, const int32_t* idx, const float* l
   if (!W || !ws || (T > 0 && (!H || !idx || !logp))) return CKL_ERR_INVALID_ARG;
   if (!aligned16(H) || !aligned16(W) || !aligned16(ws) || !aligned4(idx) || !aligned4(logp))
     return CKL_ERR_INVALID_ARG;
-  if (K > ckl::PREP_MAXK) return CKL_ERR_UNSUPPORTED;
+  if (K > ckl::PREP_MAXK_LARGE) return CKL_ERR_UNSUPPORTED;
   L = layout(T, d, V, K, chunk, single_pass, eb);
   if (ws_bytes < L.total) return CKL_ERR_WORKSPACE;
   if (!device_info(di)) return CKL_ERR_CUDA;
@@ -1094,7 +1100,7 @@ const char* ckl_status_string(int32_t status) {
   switch (status) {
     case CKL_OK: return "ok";
     case CKL_ERR_INVALID_ARG: return "invalid argument (null pointer, size or alignment)";
-    case CKL_ERR_UNSUPPORTED: return "unsupported (needs an sm_100 device and K <= 256)";
+    case CKL_ERR_UNSUPPORTED: return "unsupported (needs an sm_100 device and K <= 2048)";
     case CKL_ERR_WORKSPACE: return "workspace too small";
     case CKL_ERR_CUDA: return "CUDA call or kernel launch failed";
     case CKL_ERR_BAD_INDEX: return "teacher token id outside [0, V)";
@@ -1178,7 +1184,7 @@ int ckl_forward_static_scratch(const uint16_t* H, const uint16_t* W, const int32
   if (!aligned16(H) || !aligned16(W) || !aligned4(topk_idx) || !aligned4(topk_logp) ||
       !aligned4(lse) || !aligned4(device_status))
     return CKL_ERR_INVALID_ARG;
-  if (K > ckl::PREP_MAXK) return CKL_ERR_UNSUPPORTED;
+  if (K > ckl::PREP_MAXK_LARGE) return CKL_ERR_UNSUPPORTED;
   // The forward's own layout (as in ckl_forward, partials sized for the largest
   // split count), so the limit depends on T and K only; checked before any
   // device call.

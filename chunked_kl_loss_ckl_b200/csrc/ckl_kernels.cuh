@@ -205,6 +205,110 @@ prep_kernel(const int32_t* __restrict__ idx, const float* __restrict__ logp,
   }
 }
 
+// The same for 256 < K <= PREP_MAXK_LARGE: one 256-thread CTA per row; the
+// (id, position) keys are put in order by a bitonic sort in shared memory,
+// which gives the warp kernel's order (id, then position in the cache).
+constexpr int PREPL_THREADS = 256;
+constexpr int PREP_MAXK_LARGE = 2048;
+
+__device__ __forceinline__ float prepl_block_max(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float r = -INFINITY;
+  for (int w = 0; w < PREPL_THREADS / 32; ++w) r = fmaxf(r, red[w]);
+  __syncthreads();
+  return r;
+}
+__device__ __forceinline__ float prepl_block_sum(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float r = 0.f;
+  for (int w = 0; w < PREPL_THREADS / 32; ++w) r += red[w];
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(PREPL_THREADS)
+prep_large_kernel(const int32_t* __restrict__ idx, const float* __restrict__ logp,
+                  const uint8_t* __restrict__ mask, int64_t T, int K, int64_t V,
+                  int2* __restrict__ pairs, float* __restrict__ Hp, int* status, int* countN) {
+  __shared__ unsigned long long key[PREP_MAXK_LARGE];  // id << 32 | position
+  __shared__ float lps[PREP_MAXK_LARGE];
+  __shared__ float red[PREPL_THREADS / 32];
+  const int tid = threadIdx.x;
+  const int64_t t = blockIdx.x;
+  const int64_t base = t * K;
+  int flags = 0;
+  for (int k = tid; k < K; k += PREPL_THREADS) {
+    int v = idx[base + k];
+    float l = logp[base + k];
+    if (v < 0 || static_cast<int64_t>(v) >= V) {
+      flags |= CKL_DEV_BAD_INDEX;
+      v = INT_MAX;  // never matches a vocabulary column
+      l = -INFINITY;
+    }
+    if (isnan(l) || l == INFINITY) {
+      flags |= CKL_DEV_BAD_LOGP;
+      l = -INFINITY;
+    }
+    key[k] = (static_cast<unsigned long long>(static_cast<uint32_t>(v)) << 32) |
+             static_cast<uint32_t>(k);
+    lps[k] = l;
+  }
+  int P = 1;
+  while (P < K) P <<= 1;
+  for (int k = K + tid; k < P; k += PREPL_THREADS) key[k] = ~0ull;
+  __syncthreads();
+  // renormalisation over the K entries
+  float m = -INFINITY;
+  for (int k = tid; k < K; k += PREPL_THREADS) m = fmaxf(m, lps[k]);
+  m = prepl_block_max(m, red);
+  if (m == -INFINITY) {
+    flags |= CKL_DEV_BAD_LOGP;  // no finite log-prob in this row
+    m = 0.f;
+  }
+  float se = 0.f;
+  for (int k = tid; k < K; k += PREPL_THREADS) se += (lps[k] == -INFINITY) ? 0.f : expf(lps[k] - m);
+  const float ell = m + logf(prepl_block_sum(se, red));
+  float hp = 0.f;
+  for (int k = tid; k < K; k += PREPL_THREADS) {
+    const float pk = (lps[k] == -INFINITY) ? 0.f : expf(lps[k] - ell);
+    hp += (pk > 0.f) ? pk * (lps[k] - ell) : 0.f;
+  }
+  hp = prepl_block_sum(hp, red);
+  // bitonic sort of the keys, ascending: id, then position
+  for (int k2 = 2; k2 <= P; k2 <<= 1) {
+    for (int j = k2 >> 1; j > 0; j >>= 1) {
+      for (int i = tid; i < P; i += PREPL_THREADS) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const unsigned long long a = key[i], b = key[ixj];
+          const bool up = (i & k2) == 0;
+          if (up ? (a > b) : (a < b)) { key[i] = b; key[ixj] = a; }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int k = tid; k < K; k += PREPL_THREADS) {
+    const unsigned long long e = key[k];
+    const int pos = static_cast<int>(e & 0xFFFFFFFFull);
+    const float l = lps[pos];
+    const float pk = (l == -INFINITY) ? 0.f : expf(l - ell);
+    pairs[base + k] = make_int2(static_cast<int>(e >> 32), __float_as_int(pk));
+  }
+  if (tid == 0) {
+    Hp[t] = hp;
+    if (mask == nullptr || mask[t] != 0) atomicAdd(countN, 1);
+  }
+  flags = __reduce_or_sync(0xffffffffu, flags);
+  if ((tid & 31) == 0 && flags) atomicOr(status, flags);
+}
+
 // ------------------------------------------------------------------ combine
 constexpr int COMBINE_THREADS = 256;
 

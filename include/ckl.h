@@ -30,7 +30,7 @@
  *    nothing between calls (it only caches per-device properties such as the
  *    SM count).
  *  - Sizes: T >= 0 tokens, d >= 8 with d % 8 == 0 (16-byte rows for the TMA
- *    unit), V >= 1, 1 <= K <= 256, chunk >= 1.  T, d and V are below 2^31.
+ *    unit), V >= 1, 1 <= K <= 2048, chunk >= 1.  T, d and V are below 2^31.
  *  - Alignment: H, W, dH, dW and the workspace must be 16-byte aligned.
  *  - Errors detectable on the host (null pointer, bad size, misalignment,
  *    small workspace) return a status before anything is enqueued.  A
@@ -63,7 +63,7 @@ extern "C" {
 typedef enum ckl_status {
   CKL_OK = 0,
   CKL_ERR_INVALID_ARG = 1, /* null pointer, size out of range, misalignment */
-  CKL_ERR_UNSUPPORTED = 2, /* no sm_100 device, or K above 256 */
+  CKL_ERR_UNSUPPORTED = 2, /* no sm_100 device, or K above 2048 */
   CKL_ERR_WORKSPACE = 3,   /* workspace smaller than ckl_workspace_bytes() */
   CKL_ERR_CUDA = 4,        /* a CUDA runtime/driver call or launch failed */
   CKL_ERR_BAD_INDEX = 5,   /* device: a teacher id outside [0, V) */

@@ -125,6 +125,23 @@ def test_smallest_and_largest_K(gpu_lib, K):
     assert_parity(run_library(gpu_lib, c, chunk=128), _ref(c), f"K={K}")
 
 
+@pytest.mark.parametrize("K", [257, 1000, 2048])
+def test_large_K_takes_the_block_prep(gpu_lib, K):
+    # K above 256: the prep runs one CTA per row; ids uniform and distinct per
+    # row (a Zipf draw of 2048 distinct ids out of a few thousand is slow to
+    # make), with repeats in some rows, -inf entries and a few masked rows
+    rng = np.random.default_rng(K)
+    c = make_inputs(150, 64, 3000, 4, seed=13, w_std=0.4, mask=("bernoulli", 0.1))
+    idx = np.stack([rng.permutation(3000)[:K] for _ in range(150)]).astype(np.int32)
+    idx[:10, 1] = idx[:10, 0]                      # repeated ids
+    logp = np.log(rng.dirichlet(np.ones(K), 150)).astype(np.float32)
+    logp[10:20, -5:] = -np.inf
+    c = dict(c, idx=idx, logp=logp, K=K)
+    assert_parity(run_library(gpu_lib, c, chunk=64), _ref(c), f"K={K}")
+    out = run_library(gpu_lib, c, chunk=64)
+    assert out["status_f"][0] == 0
+
+
 def test_minus_inf_teacher_entries(gpu_lib):
     c = make_inputs(140, 64, 800, 10, seed=12, w_std=0.4)
     logp = c["logp"].copy()
