@@ -7,8 +7,8 @@
 // writes it, given the teacher's logits.
 //
 // One CTA per row (persistent over rows).  The streaming form (below, K up
-// to the CTA's 512 threads) reads each row once from HBM and once more from
-// L2.  The histogram form, used for larger K and for rows the streaming form
+// to its TS_THREADS = 256 threads) reads each row once from HBM and once more
+// from L2.  The histogram form, used for larger K and for rows the streaming form
 // cannot settle, makes three passes over the row (the first from HBM, the
 // others mostly from L2):
 //   1. the largest logit (packed bf16 maxima, two per instruction);
