@@ -80,11 +80,13 @@ def workload_desc(c):
 
 
 def kernel_source_hash() -> str:
-    """Hash of the CUDA sources; ncu traffic figures are valid only for it."""
+    """Hash of the sources of the tensor-core kernels and their launches (all
+    CUDA sources but the top-K producer's); ncu traffic figures are valid only
+    for it."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "chunked_kl_loss_ckl_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in sorted(x for x in os.listdir(csrc) if x != "ckl_topk.cuh"):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]

@@ -940,9 +940,23 @@ int ckl_topk_cache(const uint16_t* teacher_logits, int64_t T, int64_t V, int32_t
   const int vec8 = (V % 8 == 0 && aligned16(teacher_logits)) ? 1 : 0;
   const int grid = static_cast<int>(std::min<int64_t>(T, static_cast<int64_t>(di.sms) * 2));
   if (K <= ckl::TS_THREADS) {
-    const int sgrid = static_cast<int>(std::min<int64_t>(T, static_cast<int64_t>(di.sms) * ckl::TS_BLOCKS));
-    ckl::topk_stream_kernel<<<sgrid, ckl::TS_THREADS, 0, st>>>(
-        teacher_logits, T, static_cast<int>(V), K, vec8, topk_idx, topk_logp, device_status);
+    // the vector maxima in dynamic shared memory (2 bytes per 8 logits, in
+    // whole passes of the block) when they fit
+    const int mark = (vec8 && V <= ckl::TS_MARK_MAX_V) ? 1 : 0;
+    const int64_t passes = (V / 8 + ckl::TS_PER_PASS - 1) / ckl::TS_PER_PASS;
+    const size_t dyn = mark ? static_cast<size_t>(passes) * ckl::TS_THREADS * 8 : 0;
+    if (cudaFuncSetAttribute(ckl::topk_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             ckl::TS_MARK_MAX_V / 8 * 2) != cudaSuccess)
+      return CKL_ERR_CUDA;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ckl::topk_stream_kernel,
+                                                      ckl::TS_THREADS, dyn) != cudaSuccess ||
+        per_sm < 1)
+      return CKL_ERR_CUDA;
+    per_sm = std::min(per_sm, ckl::TS_BLOCKS);
+    const int sgrid = static_cast<int>(std::min<int64_t>(T, static_cast<int64_t>(di.sms) * per_sm));
+    ckl::topk_stream_kernel<<<sgrid, ckl::TS_THREADS, dyn, st>>>(
+        teacher_logits, T, static_cast<int>(V), K, vec8, mark, topk_idx, topk_logp, device_status);
     if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
     ckl::topk_fallback_kernel<<<grid, ckl::TK_THREADS, 0, st>>>(
         teacher_logits, T, static_cast<int>(V), K, vec8, topk_idx, topk_logp, device_status);

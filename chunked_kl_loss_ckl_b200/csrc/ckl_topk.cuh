@@ -178,6 +178,17 @@ __device__ __forceinline__ void tk_sort_and_write(SM& sm, uint32_t n, int K, flo
   __syncthreads();
 }
 
+// Adds element i (value v, bf16 bits raw) to the candidates if v >= v_thr.
+template <typename SM>
+__device__ __forceinline__ void tk_put(SM& sm, float v, uint32_t raw, int i, float v_thr) {
+  if (v >= v_thr) {
+    const uint32_t slot = atomicAdd(&sm.s_ncand, 1u);
+    if (slot < TK_CAP)
+      sm.cand[slot] = (static_cast<unsigned long long>(bf16_key(raw)) << 32) |
+                      (0xFFFFFFFFu - static_cast<uint32_t>(i));
+  }
+}
+
 // Gathers every element of the row whose value is >= v_thr into the
 // candidates; returns their count (the array holds at most TK_CAP).
 template <int NT = TK_THREADS, int UNROLL = TK_UNROLL, typename SM>
@@ -185,14 +196,7 @@ __device__ __forceinline__ uint32_t tk_gather(SM& sm, const uint16_t* z, int V, 
                                               float v_thr) {
   if (threadIdx.x == 0) sm.s_ncand = 0;
   __syncthreads();
-  auto put = [&](float v, uint32_t raw, int i) {
-    if (v >= v_thr) {
-      const uint32_t slot = atomicAdd(&sm.s_ncand, 1u);
-      if (slot < TK_CAP)
-        sm.cand[slot] = (static_cast<unsigned long long>(bf16_key(raw)) << 32) |
-                        (0xFFFFFFFFu - static_cast<uint32_t>(i));
-    }
-  };
+  auto put = [&](float v, uint32_t raw, int i) { tk_put(sm, v, raw, i, v_thr); };
   if (vec8) {
     // a whole 8-element vector below the threshold is skipped on its maximum
     const uint4* z4 = reinterpret_cast<const uint4*>(z);
@@ -335,21 +339,24 @@ topk_cache_kernel(const uint16_t* __restrict__ logits, int64_t T, int V, int K, 
 }
 
 // ------------------------------------------------------------ streaming form
-// Two passes per row.  Pass 1 (the only one from HBM): every thread keeps
-// its running maximum c and the sum of 2^((z - c) log2 e) over its own
-// elements, rescaled when c grows (at most once per 8-element vector); the
-// block merges the (c, sum) pairs into the row's log-sum-exp.  The K-th
-// largest of the threads' maxima is at most the row's K-th largest value
-// (those K maxima are K elements of the row), so it is a valid threshold:
-// pass 2 (from L2) gathers every element at or above it, vectors whose
-// maximum is below it skipped whole, and the sort keeps the first K.  With
-// the row's top K spread over the threads, the threshold sits just below the
-// K-th value and a few more than K elements are gathered.  When more than
-// TK_CAP would be (the row's large values crowded into few threads), the
-// row is marked and done again by histogram windows in topk_fallback_kernel.
-// Blocks of TS_THREADS threads, TS_BLOCKS per SM: enough rows in flight to
-// keep HBM busy, few enough (TS_BLOCKS x SMs x 256 KB at V = 128 256) that
-// pass 2 finds its row still in L2; needs K <= TS_THREADS.
+// One read of the row from HBM.  Pass 1: every thread keeps its running
+// maximum c and the sum of 2^((z - c) log2 e) over its own elements,
+// rescaled when c grows (at most once per 8-element vector), and writes each
+// of its vectors' maximum (a bf16) to shared memory; the block merges the
+// (c, sum) pairs into the row's log-sum-exp.  The K-th largest of the
+// threads' maxima is at most the row's K-th largest value (those K maxima
+// are K elements of the row), so it is a valid threshold.  Pass 2 scans the
+// vector maxima in shared memory and loads again only the vectors whose
+// maximum reaches the threshold (a few hundred of the row's 16 032 at
+// V = 128 256); their elements at or above it are gathered and the sort
+// keeps the first K.  With the row's top K spread over the threads, the
+// threshold sits just below the K-th value and a few more than K elements are
+// gathered.  When more than TK_CAP would be (the row's large values crowded
+// into few threads), the row is marked and done again by histogram windows
+// in topk_fallback_kernel.  Rows whose vector maxima do not fit the dynamic
+// shared memory the launch gives (V above TS_MARK_MAX_V), or whose length is
+// not a multiple of 8, gather by reading the row again instead.  Blocks of
+// TS_THREADS threads, up to TS_BLOCKS per SM; needs K <= TS_THREADS.
 #ifndef CKL_TS_THREADS
 #define CKL_TS_THREADS 256
 #endif
@@ -357,11 +364,16 @@ constexpr int TS_THREADS = CKL_TS_THREADS;
 #ifndef CKL_TS_BLOCKS
 #define CKL_TS_BLOCKS 4
 #endif
-constexpr int TS_BLOCKS = CKL_TS_BLOCKS;  // blocks per SM
+constexpr int TS_BLOCKS = CKL_TS_BLOCKS;  // blocks per SM (at most)
+constexpr int TS_MARK_MAX_V = 262144;     // vector maxima of up to 64 KB per block
+
+constexpr int TS_MARKS = 512;  // marked vectors a row may have (more: the fallback)
 
 struct TsShared {
   unsigned long long cand[TK_CAP];
   uint32_t hist[256];
+  uint32_t marked[TS_MARKS];  // indices of the vectors pass 2 loads again
+  uint32_t s_nmarked;
   float s_c[TS_THREADS / 32];
   float s_s[TS_THREADS / 32];
   uint32_t s_part[TS_THREADS / 32];
@@ -420,84 +432,166 @@ __device__ __forceinline__ uint32_t ts_kth_largest_key(TsShared& sm, uint32_t ke
   return r;
 }
 
+// The vector maxima of a row, as pass 1 leaves them: for each of a thread's
+// passes over TS_UNROLL x TS_THREADS vectors, its TS_UNROLL = 4 maxima (bf16
+// bits, -inf past the row's end) packed into one uint2 at [pass][thread], so
+// that a thread writes and reads its own four with one 8-byte access.
+static_assert(TS_UNROLL == 4, "the packed vector maxima hold four per thread and pass");
+constexpr int TS_PER_PASS = TS_THREADS * TS_UNROLL;  // vectors per pass of the block
+
+// Pass 2 from the vector maxima.  Each thread scans its own packed maxima
+// (four compared at once, one bf16x2 max) and lists the vectors whose maximum
+// reaches v_thr; then the block loads the listed vectors, one per thread, so
+// that the loads of a row are in flight together, and gathers their elements
+// at or above v_thr.  Returns the number of candidates, or TK_CAP + 1 when
+// more than TS_MARKS vectors are marked (the row then goes to the fallback).
+template <typename SM>
+__device__ __forceinline__ uint32_t ts_gather_marked(SM& sm, const uint2* vmax,
+                                                     const uint16_t* z, int n8, float v_thr) {
+  if (threadIdx.x == 0) { sm.s_ncand = 0; sm.s_nmarked = 0; }
+  __syncthreads();
+  const int passes = (n8 + TS_PER_PASS - 1) / TS_PER_PASS;
+  for (int it = 0; it < passes; ++it) {
+    const uint2 e = vmax[it * TS_THREADS + threadIdx.x];
+    const uint32_t m = bf16x2_max(e.x, e.y);
+    if (fmaxf(bf16_lo(m), bf16_hi(m)) < v_thr) continue;
+#pragma unroll
+    for (int u = 0; u < TS_UNROLL; ++u) {
+      const uint32_t word = (u < 2) ? e.x : e.y;
+      const float vm = (u & 1) ? bf16_hi(word) : bf16_lo(word);
+      const int i = it * TS_PER_PASS + u * TS_THREADS + threadIdx.x;
+      if (vm >= v_thr && i < n8) {
+        const uint32_t slot = atomicAdd(&sm.s_nmarked, 1u);
+        if (slot < static_cast<uint32_t>(TS_MARKS)) sm.marked[slot] = static_cast<uint32_t>(i);
+      }
+    }
+  }
+  __syncthreads();
+  const uint32_t nm = sm.s_nmarked;
+  if (nm > static_cast<uint32_t>(TS_MARKS)) return TK_CAP + 1;  // uniform over the block
+  const uint4* z4 = reinterpret_cast<const uint4*>(z);
+  for (uint32_t k = threadIdx.x; k < nm; k += TS_THREADS) {
+    const int i = static_cast<int>(sm.marked[k]);
+    const uint4 v = z4[i];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      tk_put(sm, bf16_lo(w[j]), w[j] & 0xFFFFu, 8 * i + 2 * j, v_thr);
+      tk_put(sm, bf16_hi(w[j]), w[j] >> 16, 8 * i + 2 * j + 1, v_thr);
+    }
+  }
+  __syncthreads();
+  return sm.s_ncand;
+}
+
+// Per-thread pass-1 state of one row: running maximum and sum of exp.
+struct TsAcc {
+  float cmax = -INFINITY;  // this thread's largest value so far
+  float s = 0.f;           // sum of 2^((z - cmax) log2 e)
+  __device__ __forceinline__ void rescale(float vm) {
+    if (vm > cmax) {
+      s *= ex2_approx((cmax - vm) * LOG2E);  // 0 while nothing was summed
+      cmax = vm;
+    }
+  }
+  // one 8-element vector; returns its maximum
+  __device__ __forceinline__ float add8(const uint4& v) {
+    const uint32_t m2 = bf16x2_max(bf16x2_max(v.x, v.y), bf16x2_max(v.z, v.w));
+    const float vm = fmaxf(bf16_lo(m2), bf16_hi(m2));
+    rescale(vm);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float a = 0.f, b = 0.f;
+    // z - cmax is exact for the values that matter (near the maximum)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      a += ex2_approx((bf16_lo(w[j]) - cmax) * LOG2E);
+      b += ex2_approx((bf16_hi(w[j]) - cmax) * LOG2E);
+    }
+    s += a + b;
+    return vm;
+  }
+};
+
+// The end of a row once every thread has its pass-1 state: log-sum-exp,
+// threshold, gather (from the vector maxima when vmax is given), sort, write.
+__device__ __forceinline__ void ts_finish_row(TsShared& sm, const TsAcc& acc, const uint16_t* z,
+                                              int V, bool vec8, const uint2* vmax, int K,
+                                              int64_t row, int32_t* idx_out, float* logp_out) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float wc = acc.cmax, ws = acc.s;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float oc = __shfl_xor_sync(0xffffffffu, wc, o);
+    const float os = __shfl_xor_sync(0xffffffffu, ws, o);
+    const float nc = fmaxf(wc, oc);
+    ws = (nc == -INFINITY) ? 0.f
+                           : ws * ex2_approx((wc - nc) * LOG2E) + os * ex2_approx((oc - nc) * LOG2E);
+    wc = nc;
+  }
+  if (lane == 0) { sm.s_c[warp] = wc; sm.s_s[warp] = ws; }
+  // threshold: the K-th largest of the threads' maxima
+  const uint32_t my_key = (acc.cmax == -INFINITY) ? 0u : bf16_key(__float_as_uint(acc.cmax) >> 16);
+  const uint32_t thr = ts_kth_largest_key(sm, my_key, K);  // synchronises the block
+  float C = -INFINITY;
+  for (int w = 0; w < TS_THREADS / 32; ++w) C = fmaxf(C, sm.s_c[w]);
+  float S = 0.f;
+  for (int w = 0; w < TS_THREADS / 32; ++w) S += sm.s_s[w] * ex2_approx((sm.s_c[w] - C) * LOG2E);
+  const float lse = C + logf(S);
+  const float v_thr = (thr == 0u) ? -INFINITY : key_value(thr);
+  const uint32_t ncand = vmax ? ts_gather_marked(sm, vmax, z, V / 8, v_thr)
+                              : tk_gather<TS_THREADS, TS_UNROLL>(sm, z, V, vec8, v_thr);
+  if (ncand <= static_cast<uint32_t>(TK_CAP)) {
+    tk_sort_and_write<TS_THREADS>(sm, ncand, K, lse, row, idx_out, logp_out);
+  } else if (threadIdx.x == 0) {
+    idx_out[row * K] = -1;  // left to topk_fallback_kernel
+  }
+}
+
+// Pass 1 of rows of 8-element vectors: TS_UNROLL independent 16-byte loads in
+// flight per thread, then their arithmetic.
 __global__ void __launch_bounds__(TS_THREADS, TS_BLOCKS)
 topk_stream_kernel(const uint16_t* __restrict__ logits, int64_t T, int V, int K, int vec8,
-                   int32_t* __restrict__ idx_out, float* __restrict__ logp_out, int* status) {
+                   int mark, int32_t* __restrict__ idx_out, float* __restrict__ logp_out,
+                   int* status) {
   __shared__ TsShared sm;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // the packed vector maxima of the row when mark != 0 (then vec8 != 0)
+  extern __shared__ uint2 ts_vmax[];
+  const int tid = threadIdx.x;
   for (int64_t row = blockIdx.x; row < T; row += gridDim.x) {
     const uint16_t* z = logits + row * static_cast<int64_t>(V);
-    // ---- pass 1: per-thread maximum and sum of exp against it
-    float cmax = -INFINITY;  // this thread's largest value so far
-    float s = 0.f;           // sum of 2^((z - cmax) log2 e)
-    auto rescale = [&](float vm) {
-      if (vm > cmax) {
-        s *= ex2_approx((cmax - vm) * LOG2E);  // 0 while nothing was summed
-        cmax = vm;
-      }
-    };
+    TsAcc acc;
     if (vec8) {
       const uint4* z4 = reinterpret_cast<const uint4*>(z);
       const int n8 = V / 8;
-      for (int base = tid; base < n8; base += TS_THREADS * TS_UNROLL) {
+      int it = 0;
+      for (int base = tid; base < n8; base += TS_PER_PASS, ++it) {
         uint4 v[TS_UNROLL];
 #pragma unroll
         for (int u = 0; u < TS_UNROLL; ++u) {
           const int i = base + u * TS_THREADS;
           if (i < n8) v[u] = z4[i];
         }
+        uint32_t mb[TS_UNROLL];
 #pragma unroll
         for (int u = 0; u < TS_UNROLL; ++u) {
-          const int i = base + u * TS_THREADS;
-          if (i >= n8) continue;
-          const uint32_t m2 = bf16x2_max(bf16x2_max(v[u].x, v[u].y), bf16x2_max(v[u].z, v[u].w));
-          rescale(fmaxf(bf16_lo(m2), bf16_hi(m2)));
-          const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-          float a = 0.f, b = 0.f;
-          // z - cmax is exact for the values that matter (near the maximum)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            a += ex2_approx((bf16_lo(w[j]) - cmax) * LOG2E);
-            b += ex2_approx((bf16_hi(w[j]) - cmax) * LOG2E);
-          }
-          s += a + b;
+          mb[u] = 0xFF80u;  // -inf: past the row's end
+          if (base + u * TS_THREADS < n8) mb[u] = __float_as_uint(acc.add8(v[u])) >> 16;
         }
+        if (mark) ts_vmax[it * TS_THREADS + tid] = make_uint2(mb[0] | (mb[1] << 16), mb[2] | (mb[3] << 16));
       }
+      // a thread whose first vector is past the row's end still owns the
+      // entries of the passes it skipped
+      if (mark)
+        for (int k = it; k * TS_PER_PASS < n8; ++k)
+          ts_vmax[k * TS_THREADS + tid] = make_uint2(0xFF80FF80u, 0xFF80FF80u);
     } else {
       for (int i = tid; i < V; i += TS_THREADS) {
         const float v = __uint_as_float(static_cast<uint32_t>(z[i]) << 16);
-        rescale(v);
-        s += ex2_approx((v - cmax) * LOG2E);
+        acc.rescale(v);
+        acc.s += ex2_approx((v - acc.cmax) * LOG2E);
       }
     }
-    // ---- the row's log-sum-exp from the threads' (cmax, s) pairs
-    float wc = cmax, ws = s;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float oc = __shfl_xor_sync(0xffffffffu, wc, o);
-      const float os = __shfl_xor_sync(0xffffffffu, ws, o);
-      const float nc = fmaxf(wc, oc);
-      ws = (nc == -INFINITY) ? 0.f
-                             : ws * ex2_approx((wc - nc) * LOG2E) + os * ex2_approx((oc - nc) * LOG2E);
-      wc = nc;
-    }
-    if (lane == 0) { sm.s_c[warp] = wc; sm.s_s[warp] = ws; }
-    // ---- threshold: the K-th largest of the threads' maxima
-    const uint32_t my_key = (cmax == -INFINITY) ? 0u : bf16_key(__float_as_uint(cmax) >> 16);
-    const uint32_t thr = ts_kth_largest_key(sm, my_key, K);  // synchronises the block
-    float C = -INFINITY;
-    for (int w = 0; w < TS_THREADS / 32; ++w) C = fmaxf(C, sm.s_c[w]);
-    float S = 0.f;
-    for (int w = 0; w < TS_THREADS / 32; ++w) S += sm.s_s[w] * ex2_approx((sm.s_c[w] - C) * LOG2E);
-    const float lse = C + logf(S);
-    const float v_thr = (thr == 0u) ? -INFINITY : key_value(thr);
-    // ---- pass 2: gather, sort, write
-    const uint32_t ncand = tk_gather<TS_THREADS, TS_UNROLL>(sm, z, V, vec8 != 0, v_thr);
-    if (ncand <= static_cast<uint32_t>(TK_CAP)) {
-      tk_sort_and_write<TS_THREADS>(sm, ncand, K, lse, row, idx_out, logp_out);
-    } else if (tid == 0) {
-      idx_out[row * K] = -1;  // left to topk_fallback_kernel
-    }
+    ts_finish_row(sm, acc, z, V, vec8 != 0, mark ? ts_vmax : nullptr, K, row, idx_out, logp_out);
   }
 }
 
@@ -508,10 +602,22 @@ __global__ void __launch_bounds__(TK_THREADS, 2)
 topk_fallback_kernel(const uint16_t* __restrict__ logits, int64_t T, int V, int K, int vec8,
                      int32_t* __restrict__ idx_out, float* __restrict__ logp_out, int* status) {
   __shared__ TkShared sm;
-  for (int64_t row = blockIdx.x; row < T; row += gridDim.x) {
-    if (idx_out[row * K] != -1) continue;  // uniform over the block
-    tk_row_hist(sm, logits + row * static_cast<int64_t>(V), V, vec8 != 0, K, row, idx_out,
-                logp_out, status);
+  // the block's rows are checked in parallel (one load each), TK_THREADS at a time
+  for (int64_t first = blockIdx.x; first < T; first += static_cast<int64_t>(gridDim.x) * TK_THREADS) {
+    const int64_t mine = first + static_cast<int64_t>(threadIdx.x) * gridDim.x;
+    const bool left = mine < T && idx_out[mine * K] == -1;
+    if (!__syncthreads_or(left)) continue;
+    __shared__ uint32_t s_left[TK_THREADS / 32];
+    const uint32_t bits = __ballot_sync(0xffffffffu, left);
+    if ((threadIdx.x & 31) == 0) s_left[threadIdx.x >> 5] = bits;
+    __syncthreads();
+    for (int t = 0; t < TK_THREADS; ++t) {
+      if (!((s_left[t >> 5] >> (t & 31)) & 1u)) continue;  // uniform over the block
+      const int64_t row = first + static_cast<int64_t>(t) * gridDim.x;
+      tk_row_hist(sm, logits + row * static_cast<int64_t>(V), V, vec8 != 0, K, row, idx_out,
+                  logp_out, status);
+    }
+    __syncthreads();
   }
 }
 

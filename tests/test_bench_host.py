@@ -34,8 +34,9 @@ def test_committed_traffic_file_is_well_formed():
     # bench.py reports these figures only while the sources hash the same
     with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
         t = json.load(f)
-    assert len(t["source_hash"]) == 16 and "ncu" in t["command"]
+    assert len(t["source_hash"]) == 16
     for k in ("fwd_gemm", "bwd_dz", "bwd_dhdw"):
+        assert "ncu" in t["commands"][k] and "--clock-control none" in t["commands"][k]
         e = t["kernels"]["8k"][k]
         assert e["dram_bytes_per_launch"] > e["algorithmic_bytes"] > 0
 

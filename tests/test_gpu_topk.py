@@ -125,6 +125,18 @@ def test_rows_whose_large_values_crowd_into_few_threads(gpu_lib):
     _check(gpu_lib, f32_to_bf16_bits(z), K)
 
 
+@pytest.mark.parametrize("V", [262144, 262152])
+def test_widest_rows_with_and_without_vector_marks(gpu_lib, V):
+    # 262 144 is the widest row whose 8-element vector maxima the streaming
+    # kernel keeps in shared memory (64 KB per CTA, fewer CTAs per SM); one
+    # vector wider and it reads the row a second time to gather instead.
+    # Row 3 has 150 equal logits across the K-th value.
+    rng = np.random.default_rng(10)
+    z = rng.normal(0, 2, (5, V)).astype(np.float32)
+    z[3, rng.choice(V, 150, replace=False)] = 9.0
+    _check(gpu_lib, f32_to_bf16_bits(z), 100)
+
+
 def test_cache_feeds_the_loss(gpu_lib):
     # The producer's output is a valid teacher cache for the fused loss.
     from ckl_synth import make_inputs
