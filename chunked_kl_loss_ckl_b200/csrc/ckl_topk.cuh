@@ -484,6 +484,36 @@ __device__ __forceinline__ uint32_t ts_gather_marked(SM& sm, const uint2* vmax,
   return sm.s_ncand;
 }
 
+// Packed pairs of fp32 (lane 0 in the low word), for the sm_100 two-lane
+// add / sub / mul instructions.
+__device__ __forceinline__ uint64_t f32x2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float f32x2_lo(uint64_t r) { return __uint_as_float(static_cast<uint32_t>(r)); }
+__device__ __forceinline__ float f32x2_hi(uint64_t r) { return __uint_as_float(static_cast<uint32_t>(r >> 32)); }
+__device__ __forceinline__ uint64_t bf16x2_widen(uint32_t w) {  // both halves, exactly
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(w << 16), "r"(w & 0xFFFF0000u));
+  return r;
+}
+__device__ __forceinline__ uint64_t f32x2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f32x2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 // Per-thread pass-1 state of one row: running maximum and sum of exp.
 struct TsAcc {
   float cmax = -INFINITY;  // this thread's largest value so far
@@ -500,17 +530,41 @@ struct TsAcc {
     const float vm = fmaxf(bf16_lo(m2), bf16_hi(m2));
     rescale(vm);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    float a = 0.f, b = 0.f;
-    // z - cmax is exact for the values that matter (near the maximum)
+    // (z - cmax) log2 e for the two halves of a word at once (packed fp32
+    // pairs, each lane rounded as the scalar form); z - cmax is exact for
+    // the values that matter (near the maximum)
+    const uint64_t c2 = f32x2_pack(cmax, cmax), l2 = f32x2_pack(LOG2E, LOG2E);
+    uint64_t ab = 0;  // (+0, +0): the sums of the low and the high halves
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      a += ex2_approx((bf16_lo(w[j]) - cmax) * LOG2E);
-      b += ex2_approx((bf16_hi(w[j]) - cmax) * LOG2E);
+      const uint64_t d = f32x2_mul(f32x2_sub(bf16x2_widen(w[j]), c2), l2);
+      ab = f32x2_add(ab, f32x2_pack(ex2_approx(f32x2_lo(d)), ex2_approx(f32x2_hi(d))));
     }
-    s += a + b;
+    s += f32x2_lo(ab) + f32x2_hi(ab);
     return vm;
   }
 };
+
+// Writes the first K of the row's n candidates in order (descending value,
+// equal values by smaller id: the candidates' keys are distinct) by ranking:
+// each candidate counts the candidates above it, and the one of rank r < K
+// writes output r.  One barrier instead of a sort's log^2; n <= 2 TS_THREADS.
+template <typename SM>
+__device__ __forceinline__ void ts_rank_and_write(SM& sm, uint32_t n, int K, float lse,
+                                                  int64_t row, int32_t* idx_out,
+                                                  float* logp_out) {
+  for (uint32_t c = threadIdx.x; c < n; c += TS_THREADS) {
+    const unsigned long long mine = sm.cand[c];
+    uint32_t rank = 0;
+#pragma unroll 4
+    for (uint32_t q = 0; q < n; ++q) rank += (sm.cand[q] > mine) ? 1u : 0u;
+    if (rank < static_cast<uint32_t>(K)) {
+      idx_out[row * K + rank] = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(mine));
+      logp_out[row * K + rank] = key_value(static_cast<uint32_t>(mine >> 32)) - lse;
+    }
+  }
+  __syncthreads();
+}
 
 // The end of a row once every thread has its pass-1 state: log-sum-exp,
 // threshold, gather (from the vector maxima when vmax is given), sort, write.
@@ -541,7 +595,10 @@ __device__ __forceinline__ void ts_finish_row(TsShared& sm, const TsAcc& acc, co
   const uint32_t ncand = vmax ? ts_gather_marked(sm, vmax, z, V / 8, v_thr)
                               : tk_gather<TS_THREADS, TS_UNROLL>(sm, z, V, vec8, v_thr);
   if (ncand <= static_cast<uint32_t>(TK_CAP)) {
-    tk_sort_and_write<TS_THREADS>(sm, ncand, K, lse, row, idx_out, logp_out);
+    if (ncand >= static_cast<uint32_t>(K) && ncand <= 2u * TS_THREADS)
+      ts_rank_and_write(sm, ncand, K, lse, row, idx_out, logp_out);
+    else
+      tk_sort_and_write<TS_THREADS>(sm, ncand, K, lse, row, idx_out, logp_out);
   } else if (threadIdx.x == 0) {
     idx_out[row * K] = -1;  // left to topk_fallback_kernel
   }
