@@ -378,9 +378,12 @@ int choose_splits(int64_t n_rb, int64_t n_vt, int sms, int smin = 1, int smax_in
 // row blocks' H (kMB x d each) does not fit in 48 MiB of L2 together, number
 // the units split-fastest with S near sqrt(slots), so that the units in
 // flight share about slots / S row blocks and S W tiles.
+#ifndef CKL_FWD_H_L2_MIB
+#define CKL_FWD_H_L2_MIB 48
+#endif
 void forward_schedule(TcParams& p, int64_t d, int eb, int slots) {
   const int64_t hblk = kMB * d * eb;
-  if (static_cast<int64_t>(p.n_rb) * hblk > (int64_t(48) << 20)) {
+  if (static_cast<int64_t>(p.n_rb) * hblk > (int64_t(CKL_FWD_H_L2_MIB) << 20)) {
     p.split_fast = 1;
     p.S = choose_splits(p.n_rb, p.n_vt, slots, 4, 16);
   } else {
