@@ -25,7 +25,7 @@ __all__ = [
     "topk_cache", "single_pass_workspace_bytes", "forward_backward", "backward_plan",
     "DW_READY_FN", "forward_f32", "backward_f32", "selftest_wait_timeout", "dp_local_stats",
     "dp_finish", "forward_vocab_shard", "combine_vocab_shards", "backward_vocab_shard",
-    "dh_to_bf16",
+    "dh_to_bf16", "find_duplicate_ids",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libckl.so")
@@ -34,7 +34,7 @@ CKL_OK = 0
 STATUS_NAMES = {
     0: "CKL_OK", 1: "CKL_ERR_INVALID_ARG", 2: "CKL_ERR_UNSUPPORTED", 3: "CKL_ERR_WORKSPACE",
     4: "CKL_ERR_CUDA", 5: "CKL_ERR_BAD_INDEX", 6: "CKL_ERR_BAD_LOGP", 7: "CKL_ERR_TIMEOUT",
-    8: "CKL_ERR_TOPK_TIES",
+    8: "CKL_ERR_TOPK_TIES", 9: "CKL_ERR_DUP_INDEX",
 }
 KERNEL_NAMES = {1: "prep", 2: "fwd_gemm", 3: "fwd_combine", 4: "bwd_dz", 5: "bwd_dhdw", 6: "other",
                 7: "topk", 8: "sp_gemm", 9: "sp_rows"}
@@ -95,6 +95,8 @@ def _load() -> ctypes.CDLL:
     L.ckl_forward_backward.restype = ctypes.c_int
     L.ckl_topk_cache.argtypes = [vp, i64, i64, i32, vp, vp, vp, vp]
     L.ckl_topk_cache.restype = ctypes.c_int
+    L.ckl_find_duplicate_ids.argtypes = [vp, i64, i32, vp, vp]
+    L.ckl_find_duplicate_ids.restype = ctypes.c_int
     L.ckl_selftest_wait_timeout.argtypes = [i64, vp, sz, vp]
     L.ckl_selftest_wait_timeout.restype = ctypes.c_int
     L.ckl_forward_vocab_shard.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i32, i64,
@@ -384,6 +386,20 @@ def topk_cache(logits, K: int, stream=None, status=None):
     if rc != CKL_OK:
         raise CklError(rc, "ckl_topk_cache")
     return idx, logp, st
+
+
+def find_duplicate_ids(idx, stream=None):
+    """ckl_find_duplicate_ids on a [T, K] int32 CUDA tensor of teacher ids:
+    returns a [1] int32 device tensor holding the smallest row with a
+    repeated id, or -1."""
+    if not idx.is_cuda or idx.dim() != 2 or not idx.is_contiguous() or idx.dtype != torch.int32:
+        raise ValueError("idx must be a contiguous 2-D int32 CUDA tensor")
+    out = torch.empty(1, dtype=torch.int32, device=idx.device)
+    rc = lib.ckl_find_duplicate_ids(_ptr(idx), idx.shape[0], idx.shape[1], _ptr(out),
+                                    _stream_handle(stream))
+    if rc != CKL_OK:
+        raise CklError(rc, "ckl_find_duplicate_ids")
+    return out
 
 
 def selftest_wait_timeout(limit_s: float, workspace, stream=None) -> None:

@@ -969,6 +969,27 @@ int ckl_topk_cache(const uint16_t* teacher_logits, int64_t T, int64_t V, int32_t
   return cudaGetLastError() == cudaSuccess ? CKL_OK : CKL_ERR_CUDA;
 }
 
+int ckl_find_duplicate_ids(const int32_t* topk_idx, int64_t T, int32_t K,
+                           int32_t* first_dup_row, void* stream) {
+  const int64_t lim = (int64_t(1) << 31) - 1;
+  if (T < 0 || T >= lim || K < 1) return CKL_ERR_INVALID_ARG;
+  if (K > ckl::PREP_MAXK_LARGE) return CKL_ERR_UNSUPPORTED;
+  if (!first_dup_row || !aligned4(first_dup_row) || (T > 0 && (!topk_idx || !aligned4(topk_idx))))
+    return CKL_ERR_INVALID_ARG;
+  if (T * static_cast<int64_t>(K) >= lim) return CKL_ERR_INVALID_ARG;
+  DevInfo di;
+  if (!device_info(di)) return CKL_ERR_CUDA;
+  if (di.major != 10) return CKL_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(first_dup_row, 0xFF, sizeof(int32_t), st) != cudaSuccess)  // -1
+    return CKL_ERR_CUDA;
+  if (T == 0) return CKL_OK;
+  const int grid = static_cast<int>(std::min<int64_t>(T, static_cast<int64_t>(di.sms) * 8));
+  ckl::dup_ids_kernel<<<grid, ckl::DUP_THREADS, 0, st>>>(topk_idx, T, K,
+                                                        reinterpret_cast<uint32_t*>(first_dup_row));
+  return cudaGetLastError() == cudaSuccess ? CKL_OK : CKL_ERR_CUDA;
+}
+
 int ckl_selftest_wait_timeout(int64_t limit_ns, void* workspace, size_t workspace_bytes,
                               void* stream) {
   if (!workspace || !aligned16(workspace) || workspace_bytes < kHeaderBytes)
@@ -1124,6 +1145,7 @@ const char* ckl_status_string(int32_t status) {
     case CKL_ERR_BAD_LOGP: return "teacher log-prob NaN/+inf, or a row with none finite";
     case CKL_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out of time";
     case CKL_ERR_TOPK_TIES: return "too many teacher logits tie at a row's K-th value";
+    case CKL_ERR_DUP_INDEX: return "a teacher token id repeated within a row";
     default: return "unknown status";
   }
 }

@@ -232,6 +232,33 @@ __device__ __forceinline__ float prepl_block_sum(float v, float* red) {
   return r;
 }
 
+// The smallest row of idx [T, K] that holds some id more than once, by
+// atomicMin into *first_dup_row (pre-set to -1, i.e. 0xFFFFFFFF unsigned).
+// One CTA per row, persistent; the row's ids in shared memory, each thread
+// comparing its ids with every later one (K^2 / 2 comparisons per row).
+constexpr int DUP_THREADS = 256;
+__global__ void __launch_bounds__(DUP_THREADS)
+dup_ids_kernel(const int32_t* __restrict__ idx, int64_t T, int K, uint32_t* first_dup_row) {
+  __shared__ int32_t ids[PREP_MAXK_LARGE];
+  __shared__ int s_found;
+  for (int64_t row = blockIdx.x; row < T; row += gridDim.x) {
+    if (threadIdx.x == 0) s_found = 0;
+    for (int k = threadIdx.x; k < K; k += DUP_THREADS) ids[k] = idx[row * K + k];
+    __syncthreads();
+    bool dup = false;
+    for (int a = threadIdx.x; a < K && !dup; a += DUP_THREADS) {
+      const int32_t v = ids[a];
+      for (int b = a + 1; b < K; ++b)
+        if (ids[b] == v) { dup = true; break; }
+    }
+    if (dup) s_found = 1;
+    __syncthreads();
+    if (threadIdx.x == 0 && s_found) atomicMin(first_dup_row, static_cast<uint32_t>(row));
+    __syncthreads();
+  }
+}
+
+
 __global__ void __launch_bounds__(PREPL_THREADS)
 prep_large_kernel(const int32_t* __restrict__ idx, const float* __restrict__ logp,
                   const uint8_t* __restrict__ mask, int64_t T, int K, int64_t V,

@@ -69,7 +69,8 @@ typedef enum ckl_status {
   CKL_ERR_BAD_INDEX = 5,   /* device: a teacher id outside [0, V) */
   CKL_ERR_BAD_LOGP = 6,    /* device: NaN/+inf log-prob, or a row with none finite */
   CKL_ERR_TIMEOUT = 7,     /* device: a bounded wait inside a kernel ran out */
-  CKL_ERR_TOPK_TIES = 8    /* device: too many logits tie at a row's K-th value */
+  CKL_ERR_TOPK_TIES = 8,   /* device: too many logits tie at a row's K-th value */
+  CKL_ERR_DUP_INDEX = 9    /* a teacher id repeated within a row (ckl_find_duplicate_ids) */
 } ckl_status;
 
 /* Kernel ids written by the optional launch trace. */
@@ -375,6 +376,26 @@ CKL_API int ckl_read_device_status(const void* workspace, void* stream, int32_t*
 CKL_API int ckl_topk_cache(const uint16_t* teacher_logits, int64_t T, int64_t V, int32_t K,
                            int32_t* topk_idx, float* topk_logp, int32_t* device_status,
                            void* stream);
+
+/*
+ * Optional duplicate-id check of a teacher cache.  The pages' cache keeps
+ * each position's 100 most likely tokens ("Дистилляция LLM на одной GPU:
+ * offline-кэш и chunked KL loss", section «Два приёма»), so its ids are
+ * distinct; ckl_forward / ckl_backward take a repeated id literally (its
+ * log-probs' renormalised p are summed at that token).  A caller whose policy
+ * is to refuse repeats runs this check first and treats a row >= 0 as
+ * CKL_ERR_DUP_INDEX.
+ *   topk_idx        [T, K] int32 device, row-major
+ *   first_dup_row   [1]    int32 device out: the smallest row holding some id
+ *                                more than once, or -1 when every row's ids
+ *                                are distinct
+ * Requires 1 <= K <= 2048.  Needs no workspace; one small kernel enqueued on
+ * `stream` (the result is ready when the stream reaches it).  Returns
+ * CKL_ERR_INVALID_ARG for a null or misaligned pointer or a bad size,
+ * CKL_ERR_UNSUPPORTED for K above 2048.
+ */
+CKL_API int ckl_find_duplicate_ids(const int32_t* topk_idx, int64_t T, int32_t K,
+                                   int32_t* first_dup_row, void* stream);
 
 /* Static, human-readable text for a status code. */
 CKL_API const char* ckl_status_string(int32_t status);

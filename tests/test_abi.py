@@ -25,7 +25,8 @@ def test_header_declares_the_entry_points():
     assert _declared() == ["ckl_backward", "ckl_backward_ex", "ckl_backward_f32",
                            "ckl_backward_plan", "ckl_backward_vocab_shard",
                            "ckl_combine_vocab_shards", "ckl_dh_to_bf16", "ckl_dp_finish",
-                           "ckl_dp_local_stats", "ckl_forward", "ckl_forward_backward",
+                           "ckl_dp_local_stats", "ckl_find_duplicate_ids", "ckl_forward",
+                           "ckl_forward_backward",
                            "ckl_forward_f32", "ckl_forward_static_scratch",
                            "ckl_forward_vocab_shard",
                            "ckl_read_device_status", "ckl_selftest_wait_timeout",
@@ -41,7 +42,7 @@ def test_library_exports_every_declared_symbol(ckl):
 
 
 def test_status_strings_and_version(ckl):
-    for code in range(9):
+    for code in range(10):
         assert ckl.status_string(code) and ckl.status_string(code) != "unknown status"
     assert ckl.status_string(99) == "unknown status"
     assert ckl.lib.ckl_version() >= 100
@@ -187,6 +188,13 @@ def test_host_checks_return_before_any_device_work(ckl):
     assert L.ckl_combine_vocab_shards(fake, 2, nul, 4, 4, fake, fake, fake, 16, nul, nul) == 3
     assert L.ckl_dh_to_bf16(fake, fake, 6, nul) == 1
     assert L.ckl_dh_to_bf16(ctypes.c_void_p(4100), fake, 8, nul) == 1
+    # duplicate-id check: K in [1, 2048], aligned non-null buffers
+    assert L.ckl_find_duplicate_ids(fake, 4, 0, fake, nul) == 1
+    assert L.ckl_find_duplicate_ids(fake, -1, 4, fake, nul) == 1
+    assert L.ckl_find_duplicate_ids(fake, 4, 4, nul, nul) == 1
+    assert L.ckl_find_duplicate_ids(nul, 4, 4, fake, nul) == 1
+    assert L.ckl_find_duplicate_ids(fake, 4, 4, ctypes.c_void_p(4098), nul) == 1
+    assert L.ckl_find_duplicate_ids(fake, 4, 3000, fake, nul) == 2
 
 
 def test_static_scratch_limit_is_checked_on_the_host(ckl):

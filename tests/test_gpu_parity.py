@@ -223,3 +223,25 @@ def test_comparator_losses_agree_with_the_library(gpu_lib):
         gw = w.grad.float().cpu().numpy()
         assert np.linalg.norm(gh - out["dH"]) / np.linalg.norm(out["dH"]) < 2e-2
         assert np.linalg.norm(gw - out["dW"]) / np.linalg.norm(out["dW"]) < 2e-2
+
+
+def _first_dup_row(idx):
+    return next((r for r in range(idx.shape[0]) if len(np.unique(idx[r])) < idx.shape[1]), -1)
+
+
+@pytest.mark.parametrize("T,K", [(700, 100), (40, 2048), (5, 1), (0, 16)])
+def test_duplicate_id_check_finds_the_first_repeat(gpu_lib, T, K):
+    # distinct ids everywhere (-1), then repeats planted in three rows: the
+    # smallest of them is reported; 700 rows > the CTAs' rows per pass
+    rng = np.random.default_rng(T + K)
+    idx = np.zeros((T, K), dtype=np.int32)
+    for r in range(T):
+        idx[r] = rng.permutation(200000)[:K]
+    got = gpu_lib.find_duplicate_ids(torch.from_numpy(idx).cuda()).item()
+    assert got == -1 == _first_dup_row(idx)
+    if K > 1 and T > 0:
+        for r in rng.choice(T, min(3, T), replace=False):
+            a, b = rng.choice(K, 2, replace=False)
+            idx[r, b] = idx[r, a]
+        got = gpu_lib.find_duplicate_ids(torch.from_numpy(idx).cuda()).item()
+        assert got == _first_dup_row(idx) >= 0
