@@ -125,6 +125,21 @@ def test_rows_whose_large_values_crowd_into_few_threads(gpu_lib):
     _check(gpu_lib, f32_to_bf16_bits(z), K)
 
 
+@pytest.mark.parametrize("n_top", [300, 700])
+def test_many_marked_vectors_rank_or_fallback(gpu_lib, n_top):
+    # n_top equal top logits, each in its own 8-element vector: 300 are
+    # ranked in the streaming kernel (more candidates than threads), 700 mark
+    # more vectors than its list holds and the row goes to the histogram
+    # kernel; both must return the first K of the ties by id
+    rng = np.random.default_rng(11 + n_top)
+    T, V, K = 4, 128256, 100
+    z = rng.normal(0, 2, (T, V)).astype(np.float32)
+    for r in (0, 2):
+        vecs = rng.choice(V // 8, n_top, replace=False)
+        z[r, 8 * vecs + rng.integers(0, 8, n_top)] = 11.0
+    _check(gpu_lib, f32_to_bf16_bits(z), K)
+
+
 @pytest.mark.parametrize("V", [262144, 262152])
 def test_widest_rows_with_and_without_vector_marks(gpu_lib, V):
     # 262 144 is the widest row whose 8-element vector maxima the streaming
