@@ -32,6 +32,11 @@
 
 #include "ckl_ptx.cuh"
 
+// DHDW: alternate the k direction of a slot's consecutive jobs (1) or not (0).
+#ifndef CKL_SERPENTINE
+#define CKL_SERPENTINE 1
+#endif
+
 namespace ckl {
 
 constexpr int BM = 128;           // rows per tile (TMEM lanes)
@@ -641,6 +646,7 @@ struct JobIter {
   int lin;
   int phase;  // DHDW: 0 = dH units, 1 = dW tiles, 2 = done
   int k6, e6;
+  int ord;  // jobs of this slot before this one
   // tiles of a class (n slots, quota Q for the first E, Q - 1 for the rest)
   // dealt in rounds before round k, and those of its first m slots in round k
   __device__ static int cls_before(int k, int n, int Q, int E) {
@@ -686,6 +692,7 @@ struct JobIter {
   }
   __device__ void init(const TcParams& p, int mode_, int per_slot) {
     mode = mode_;
+    ord = 0;
     G = gridDim.x / per_slot;
     cta = blockIdx.x / per_slot;
     if (mode == MODE_DZ) {
@@ -710,7 +717,14 @@ struct JobIter {
     if (mode == MODE_DZ) return lin < p.n_units;
     return (mode != MODE_DHDW) ? (u < p.n_units) : (phase < 2);
   }
+  // DHDW: sweep this job's k-blocks backwards?  A slot's consecutive jobs
+  // alternate direction, so that a job starts on the operand rows the slot's
+  // (and, in step, the other slots') previous jobs read last, which L2 still
+  // holds: the slab's W rows for the dH units, H_c^T and dZ panels for the
+  // dW tiles.
+  __device__ bool reverse_k() const { return CKL_SERPENTINE && mode == MODE_DHDW && (ord & 1); }
   __device__ void next(const TcParams& p) {
+    ++ord;
     if (mode == MODE_DZ) {
       lin += G;
       u = lin % p.n_rb;
@@ -864,7 +878,9 @@ tc_kernel(const __grid_constant__ TcParams p) {
           b_x = (it.u % p.n_nt) * p.bn + static_cast<int>(rank) * half_n;
         }
         const uint32_t bytes = (MODE != MODE_DHDW) ? A_BYTES + B_STAGE : A_BYTES + half_n * 128;
-        for (int kb = 0; kb < nkb; ++kb) {
+        const bool rev = it.reverse_k();
+        for (int kq = 0; kq < nkb; ++kq) {
+          const int kb = rev ? nkb - 1 - kq : kq;  // the k-block this stage carries
           if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, p.status)) { ok = false; break; }
           uint32_t fb = bar_full + 8 * stage;
           if (PAIR) {
