@@ -133,7 +133,7 @@ __device__ __forceinline__ void tk_for_row(const uint16_t* z, int V, bool vec8, 
   }
 }
 
-// Shared memory of one row's selection.
+// Shared memory of one row's selection (histogram form).
 struct TkShared {
   uint32_t hist[TK_WIN];
   unsigned long long cand[TK_CAP];
@@ -369,68 +369,53 @@ constexpr int TS_MARK_MAX_V = 262144;     // vector maxima of up to 64 KB per bl
 
 constexpr int TS_MARKS = 512;  // marked vectors a row may have (more: the fallback)
 
-struct TsShared {
+struct alignas(16) TsShared {
   unsigned long long cand[TK_CAP];
-  uint32_t hist[256];
+  uint32_t keys[TS_THREADS];  // the threads' maximum keys, for the threshold
   uint32_t marked[TS_MARKS];  // indices of the vectors pass 2 loads again
   uint32_t s_nmarked;
   float s_c[TS_THREADS / 32];
   float s_s[TS_THREADS / 32];
-  uint32_t s_part[TS_THREADS / 32];
-  uint32_t s_thr, s_total, s_ncand;
+  uint32_t s_thr, s_ncand;
 };
 
 // The K-th largest of the block's keys (one per thread; 0 = no element),
-// by two 256-bucket rounds: high byte, then low byte.
-__device__ __forceinline__ uint32_t ts_kth_largest_key(TsShared& sm, uint32_t key, int K) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  static_assert(TS_THREADS >= 256 && TS_THREADS % 256 == 0, "threads 0-255 own one bucket each");
-  uint32_t prefix = 0, need = static_cast<uint32_t>(K);
-  bool few = false;  // fewer than K keys: every key counts
-  for (int round = 0; round < 2; ++round) {
-    if (tid < 256) sm.hist[tid] = 0;
-    __syncthreads();
-    if (key != 0u && (round == 0 || (key >> 8) == prefix))
-      atomicAdd(&sm.hist[(round == 0) ? (key >> 8) : (key & 0xFFu)], 1u);
-    __syncthreads();
-    // thread tid < 256 owns bucket 255 - tid (descending keys)
-    uint32_t own = 0, incl = 0;
-    if (tid < 256) {
-      own = sm.hist[255 - tid];
-      incl = own;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      if (lane == 31) sm.s_part[warp] = incl;
-    }
-    __syncthreads();
-    uint32_t before = incl - own, total = 0;
-    for (int w = 0; w < 8; ++w) {
-      if (w < warp) before += sm.s_part[w];
-      total += sm.s_part[w];
-    }
-    if (round == 0 && total < need) {  // the same on every thread
-      few = true;
-      break;
-    }
-    if (tid < 256 && before < need && before + own >= need) {
-      const uint32_t b = 255u - static_cast<uint32_t>(tid);
-      sm.s_thr = (round == 0) ? b : ((prefix << 8) | b);
-      sm.s_total = before;  // keys above this bucket
-    }
-    __syncthreads();
-    if (round == 0) {
-      prefix = sm.s_thr;
-      need -= sm.s_total;
-    }
-    __syncthreads();
-  }
-  const uint32_t r = few ? 0u : sm.s_thr;
+// or 0 when fewer than K are non-zero.  The keys go to shared memory and
+// warp 0 selects the answer bit by bit from the most significant: at each
+// bit it counts, with ballots, the keys that agree with the bits chosen so
+// far and have this one set; if at least the remaining rank are, the answer
+// has the bit, otherwise those keys all rank above it.  Two barriers.
+__device__ __forceinline__ uint32_t ts_kth_key(TsShared& sm, uint32_t key, int K) {
+  constexpr int KPL = TS_THREADS / 32;  // keys per lane
+  sm.keys[threadIdx.x] = key;
   __syncthreads();
-  return r;
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    uint32_t k[KPL];
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) k[j] = sm.keys[j * 32 + lane];
+    uint32_t total = 0;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) total += __popc(__ballot_sync(0xffffffffu, k[j] != 0u));
+    uint32_t prefix = 0;
+    if (total >= static_cast<uint32_t>(K)) {
+      uint32_t need = static_cast<uint32_t>(K);
+#pragma unroll 1
+      for (int bit = 15; bit >= 0; --bit) {
+        const uint32_t hi = (prefix >> bit) | 1u;  // the chosen bits, then this one set
+        uint32_t cnt = 0;
+#pragma unroll
+        for (int j = 0; j < KPL; ++j) cnt += __popc(__ballot_sync(0xffffffffu, (k[j] >> bit) == hi));
+        if (cnt >= need) prefix |= 1u << bit;
+        else need -= cnt;
+      }
+    }
+    if (lane == 0) sm.s_thr = prefix;
+  }
+  __syncthreads();
+  return sm.s_thr;
 }
+
 
 // The vector maxima of a row, as pass 1 leaves them: for each of a thread's
 // passes over TS_UNROLL x TS_THREADS vectors, its TS_UNROLL = 4 maxima (bf16
@@ -553,11 +538,15 @@ template <typename SM>
 __device__ __forceinline__ void ts_rank_and_write(SM& sm, uint32_t n, int K, float lse,
                                                   int64_t row, int32_t* idx_out,
                                                   float* logp_out) {
+  const ulonglong2* c2 = reinterpret_cast<const ulonglong2*>(sm.cand);
   for (uint32_t c = threadIdx.x; c < n; c += TS_THREADS) {
     const unsigned long long mine = sm.cand[c];
-    uint32_t rank = 0;
+    uint32_t rank = (n & 1u) && sm.cand[n - 1] > mine ? 1u : 0u;
 #pragma unroll 4
-    for (uint32_t q = 0; q < n; ++q) rank += (sm.cand[q] > mine) ? 1u : 0u;
+    for (uint32_t q = 0; q < n / 2; ++q) {  // two candidates per 16-byte read
+      const ulonglong2 e = c2[q];
+      rank += (e.x > mine ? 1u : 0u) + (e.y > mine ? 1u : 0u);
+    }
     if (rank < static_cast<uint32_t>(K)) {
       idx_out[row * K + rank] = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(mine));
       logp_out[row * K + rank] = key_value(static_cast<uint32_t>(mine >> 32)) - lse;
@@ -585,7 +574,7 @@ __device__ __forceinline__ void ts_finish_row(TsShared& sm, const TsAcc& acc, co
   if (lane == 0) { sm.s_c[warp] = wc; sm.s_s[warp] = ws; }
   // threshold: the K-th largest of the threads' maxima
   const uint32_t my_key = (acc.cmax == -INFINITY) ? 0u : bf16_key(__float_as_uint(acc.cmax) >> 16);
-  const uint32_t thr = ts_kth_largest_key(sm, my_key, K);  // synchronises the block
+  const uint32_t thr = ts_kth_key(sm, my_key, K);  // synchronises the block
   float C = -INFINITY;
   for (int w = 0; w < TS_THREADS / 32; ++w) C = fmaxf(C, sm.s_c[w]);
   float S = 0.f;
