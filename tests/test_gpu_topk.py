@@ -125,6 +125,17 @@ def test_rows_whose_large_values_crowd_into_few_threads(gpu_lib):
     _check(gpu_lib, f32_to_bf16_bits(z), K)
 
 
+@pytest.mark.parametrize("V,K", [(1024, 200), (2048, 256), (4096, 256), (8, 8)])
+def test_rows_with_fewer_vectors_than_threads(gpu_lib, V, K):
+    # 8-element vectors: 1024 logits give 128 thread maxima, fewer than K =
+    # 200, so every element is a candidate (and they are sorted, not ranked);
+    # 2048 and 4096 give exactly and twice 256 maxima at the largest K the
+    # streaming form takes; V = K = 8 is one vector
+    rng = np.random.default_rng(V + K)
+    z = np.round(rng.normal(0, 2, (37, V)) * 8) / 8   # ties on a 1/8 grid
+    _check(gpu_lib, f32_to_bf16_bits(z.astype(np.float32)), K)
+
+
 @pytest.mark.parametrize("n_top", [300, 700])
 def test_many_marked_vectors_rank_or_fallback(gpu_lib, n_top):
     # n_top equal top logits, each in its own 8-element vector: 300 are
