@@ -346,14 +346,16 @@ topk_cache_kernel(const uint16_t* __restrict__ logits, int64_t T, int V, int K, 
 // (c, sum) pairs into the row's log-sum-exp.  The K-th largest of the
 // threads' maxima is at most the row's K-th largest value (those K maxima
 // are K elements of the row), so it is a valid threshold.  Pass 2 scans the
-// vector maxima in shared memory and loads again only the vectors whose
-// maximum reaches the threshold (a few hundred of the row's 16 032 at
-// V = 128 256); their elements at or above it are gathered and the sort
-// keeps the first K.  With the row's top K spread over the threads, the
+// vector maxima in shared memory, lists the vectors whose maximum reaches the
+// threshold (about 130 of the row's 16 032 at V = 128 256) and loads them
+// again, one per thread; their elements at or above it are the candidates,
+// and each candidate's rank among them (their keys are distinct) places the
+// first K in order.  With the row's top K spread over the threads, the
 // threshold sits just below the K-th value and a few more than K elements are
-// gathered.  When more than TK_CAP would be (the row's large values crowded
-// into few threads), the row is marked and done again by histogram windows
-// in topk_fallback_kernel.  Rows whose vector maxima do not fit the dynamic
+// gathered.  When more than TS_MARKS vectors are marked or more than TK_CAP
+// elements would be gathered (the row's large values crowded into few
+// threads, or heavy ties), the row is marked and done again by histogram
+// windows in topk_fallback_kernel.  Rows whose vector maxima do not fit the dynamic
 // shared memory the launch gives (V above TS_MARK_MAX_V), or whose length is
 // not a multiple of 8, gather by reading the row again instead.  Blocks of
 // TS_THREADS threads, up to TS_BLOCKS per SM; needs K <= TS_THREADS.
