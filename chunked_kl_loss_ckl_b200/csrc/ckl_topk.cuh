@@ -378,6 +378,7 @@ struct alignas(16) TsShared {
   uint32_t s_nmarked;
   float s_c[TS_THREADS / 32];
   float s_s[TS_THREADS / 32];
+  float s_lse;
   uint32_t s_thr, s_ncand;
 };
 
@@ -386,36 +387,32 @@ struct alignas(16) TsShared {
 // warp 0 selects the answer bit by bit from the most significant: at each
 // bit it counts, with ballots, the keys that agree with the bits chosen so
 // far and have this one set; if at least the remaining rank are, the answer
-// has the bit, otherwise those keys all rank above it.  Two barriers.
-__device__ __forceinline__ uint32_t ts_kth_key(TsShared& sm, uint32_t key, int K) {
+// has the bit, otherwise those keys all rank above it.  Called by one warp
+// on the keys in sm.keys.
+__device__ __forceinline__ uint32_t ts_kth_key_warp(const TsShared& sm, int K) {
   constexpr int KPL = TS_THREADS / 32;  // keys per lane
-  sm.keys[threadIdx.x] = key;
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    uint32_t k[KPL];
+  const int lane = threadIdx.x & 31;
+  uint32_t k[KPL];
 #pragma unroll
-    for (int j = 0; j < KPL; ++j) k[j] = sm.keys[j * 32 + lane];
-    uint32_t total = 0;
+  for (int j = 0; j < KPL; ++j) k[j] = sm.keys[j * 32 + lane];
+  uint32_t mine = 0;
 #pragma unroll
-    for (int j = 0; j < KPL; ++j) total += __popc(__ballot_sync(0xffffffffu, k[j] != 0u));
-    uint32_t prefix = 0;
-    if (total >= static_cast<uint32_t>(K)) {
-      uint32_t need = static_cast<uint32_t>(K);
+  for (int j = 0; j < KPL; ++j) mine += (k[j] != 0u) ? 1u : 0u;
+  uint32_t prefix = 0;
+  if (__reduce_add_sync(0xffffffffu, mine) >= static_cast<uint32_t>(K)) {
+    uint32_t need = static_cast<uint32_t>(K);
 #pragma unroll 1
-      for (int bit = 15; bit >= 0; --bit) {
-        const uint32_t hi = (prefix >> bit) | 1u;  // the chosen bits, then this one set
-        uint32_t cnt = 0;
+    for (int bit = 15; bit >= 0; --bit) {
+      const uint32_t hi = (prefix >> bit) | 1u;  // the chosen bits, then this one set
+      uint32_t c = 0;
 #pragma unroll
-        for (int j = 0; j < KPL; ++j) cnt += __popc(__ballot_sync(0xffffffffu, (k[j] >> bit) == hi));
-        if (cnt >= need) prefix |= 1u << bit;
-        else need -= cnt;
-      }
+      for (int j = 0; j < KPL; ++j) c += ((k[j] >> bit) == hi) ? 1u : 0u;
+      const uint32_t cnt = __reduce_add_sync(0xffffffffu, c);
+      if (cnt >= need) prefix |= 1u << bit;
+      else need -= cnt;
     }
-    if (lane == 0) sm.s_thr = prefix;
   }
-  __syncthreads();
-  return sm.s_thr;
+  return prefix;
 }
 
 
@@ -574,14 +571,23 @@ __device__ __forceinline__ void ts_finish_row(TsShared& sm, const TsAcc& acc, co
     wc = nc;
   }
   if (lane == 0) { sm.s_c[warp] = wc; sm.s_s[warp] = ws; }
-  // threshold: the K-th largest of the threads' maxima
-  const uint32_t my_key = (acc.cmax == -INFINITY) ? 0u : bf16_key(__float_as_uint(acc.cmax) >> 16);
-  const uint32_t thr = ts_kth_key(sm, my_key, K);  // synchronises the block
-  float C = -INFINITY;
-  for (int w = 0; w < TS_THREADS / 32; ++w) C = fmaxf(C, sm.s_c[w]);
-  float S = 0.f;
-  for (int w = 0; w < TS_THREADS / 32; ++w) S += sm.s_s[w] * ex2_approx((sm.s_c[w] - C) * LOG2E);
-  const float lse = C + logf(S);
+  // the threshold, the K-th largest of the threads' maxima, by warp 0 while
+  // warp 1 merges the warps' (max, sum) pairs into the row's log-sum-exp
+  sm.keys[threadIdx.x] = (acc.cmax == -INFINITY) ? 0u : bf16_key(__float_as_uint(acc.cmax) >> 16);
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t t = ts_kth_key_warp(sm, K);
+    if (lane == 0) sm.s_thr = t;
+  } else if (warp == 1 && lane == 0) {
+    float C = -INFINITY;
+    for (int w = 0; w < TS_THREADS / 32; ++w) C = fmaxf(C, sm.s_c[w]);
+    float S = 0.f;
+    for (int w = 0; w < TS_THREADS / 32; ++w) S += sm.s_s[w] * ex2_approx((sm.s_c[w] - C) * LOG2E);
+    sm.s_lse = C + logf(S);
+  }
+  __syncthreads();
+  const uint32_t thr = sm.s_thr;
+  const float lse = sm.s_lse;
   const float v_thr = (thr == 0u) ? -INFINITY : key_value(thr);
   const uint32_t ncand = vmax ? ts_gather_marked(sm, vmax, z, V / 8, v_thr)
                               : tk_gather<TS_THREADS, TS_UNROLL>(sm, z, V, vec8, v_thr);
